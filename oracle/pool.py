@@ -1,0 +1,274 @@
+"""Reference model of the mixed-format page pool: allocator, block tables, anchor policy.
+
+ORACLE -- test infrastructure only (see ``oracle/formats.py`` for the rule on who may use it).
+
+Written from the pages' description of the page hierarchy ("Minima-KV ..." summary,
+brainszone.ai pt page, sections "O que os autores propõem" and "Âncoras em FP8, arquivo em
+TQ3"): every page of a live request stays addressable through the request's page table;
+recently used pages and pages marked protected ("anchor") stay FP8; older non-anchor pages
+are converted to packed TQ3.  Readings of what the pages leave open:
+
+* Page = 16 tokens.  A page p of a sequence of length L is an anchor iff
+  p < sink_pages (page 0 by default), or 16p + 16 > L - W (it holds one of the last W
+  tokens), or it is flagged protected.  Demotion converts every full FP8 page that is not
+  an anchor; the TQ3 page is computed from the FP8 page (pages are *converted*).
+* Slots are handed out lowest rank first (rank = position in a per-format slot order,
+  identity unless set), sequences in the order the call lists them, pages ascending.
+  Slots freed by a call return to the free list at the end of that call.
+* Block-table entry: -1 unmapped, else (format << 30) | slot with format 0 = FP8, 1 = TQ3.
+* A call that fails changes nothing.
+"""
+from __future__ import annotations
+
+import heapq
+
+import numpy as np
+
+from . import formats as F
+
+FP8, TQ3 = 0, 1
+PAGE = F.PAGE_TOKENS
+
+
+class PoolError(Exception):
+    """Raised for the error cases of the pool API; ``code`` names the case."""
+
+    def __init__(self, code: str, msg: str = ""):
+        super().__init__(f"{code}: {msg}")
+        self.code = code
+
+
+class _Allocator:
+    def __init__(self, n: int):
+        self.n = n
+        self.rank = np.arange(n, dtype=np.int64)
+        self.heap = [(i, i) for i in range(n)]
+        self.free = set(range(n))
+
+    def set_order(self, order):
+        order = np.asarray(order, dtype=np.int64)
+        if sorted(order.tolist()) != list(range(self.n)):
+            raise PoolError("INVALID_ARG", "slot order must be a permutation")
+        self.rank = np.empty(self.n, dtype=np.int64)
+        self.rank[order] = np.arange(self.n)
+        self.heap = [(int(self.rank[s]), s) for s in self.free]
+        heapq.heapify(self.heap)
+
+    def take(self) -> int:
+        while True:
+            r, s = heapq.heappop(self.heap)
+            if s in self.free:
+                self.free.discard(s)
+                return s
+
+    def give(self, s: int):
+        self.free.add(s)
+        heapq.heappush(self.heap, (int(self.rank[s]), s))
+
+
+class RefPool:
+    """The pool's whole observable state: tables, lengths, flags and every slot's contents."""
+
+    def __init__(self, Hkv, D, max_seqs, max_pages_per_seq, fp8_slots, tq3_slots,
+                 sink_pages=1):
+        if D % F.TQ3_GROUP:
+            raise PoolError("INVALID_ARG", "head_dim must be a multiple of 32")
+        self.Hkv, self.D, self.G = Hkv, D, D // F.TQ3_GROUP
+        self.max_seqs, self.max_pages = max_seqs, max_pages_per_seq
+        self.sink_pages = sink_pages
+        self.alloc = [_Allocator(fp8_slots), _Allocator(tq3_slots)]
+        self.table = [[] for _ in range(max_seqs)]      # per seq: list of (fmt, slot)
+        self.ctx = [0] * max_seqs
+        self.protected = [set() for _ in range(max_seqs)]
+        self.fp8 = {}   # slot -> [kcodes [Hkv,16,D], vcodes, kscale [Hkv], vscale [Hkv]]
+        self.tq3 = {}   # slot -> [kq [Hkv,16,D], ks [Hkv,16,G], vq, vs]
+
+    # ------------------------------------------------------------------ helpers
+    def _check_seq(self, s):
+        if not (0 <= s < self.max_seqs):
+            raise PoolError("BAD_SEQ", f"sequence {s}")
+
+    def set_slot_order(self, fmt, order):
+        self.alloc[fmt].set_order(order)
+
+    def entry(self, seq, page) -> int:
+        fmt, slot = self.table[seq][page]
+        return (fmt << 30) | slot
+
+    def block_table(self, seq):
+        return [self.entry(seq, p) for p in range(len(self.table[seq]))]
+
+    # ------------------------------------------------------------------ append
+    def append(self, seq_ids, n_new, k, v):
+        """Append tokens: k, v float64 [sum(n_new), Hkv, D] (bf16 values), rows grouped by
+        sequence in ``seq_ids`` order."""
+        seq_ids = [int(s) for s in seq_ids]
+        n_new = [int(n) for n in n_new]
+        for s in seq_ids:
+            self._check_seq(s)
+        if len(set(seq_ids)) != len(seq_ids) or any(n < 0 for n in n_new):
+            raise PoolError("INVALID_ARG", "repeated sequence or negative count")
+        need = 0
+        for s, n in zip(seq_ids, n_new):
+            pages_after = -(-(self.ctx[s] + n) // PAGE)
+            if pages_after > self.max_pages:
+                raise PoolError("OUT_OF_PAGES", f"sequence {s} exceeds max pages")
+            need += pages_after - len(self.table[s])
+        if need > len(self.alloc[FP8].free):
+            raise PoolError("OUT_OF_PAGES", "FP8 pool exhausted")
+        row = 0
+        for s, n in zip(seq_ids, n_new):
+            L0 = self.ctx[s]
+            pages_after = -(-(L0 + n) // PAGE)
+            for _ in range(len(self.table[s]), pages_after):
+                slot = self.alloc[FP8].take()
+                self.table[s].append((FP8, slot))
+                z = np.zeros((self.Hkv, PAGE, self.D), np.uint8)
+                self.fp8[slot] = [z, z.copy(), np.zeros(self.Hkv), np.zeros(self.Hkv)]
+            t = 0
+            while t < n:
+                pos = L0 + t
+                page, off = divmod(pos, PAGE)
+                cnt = min(PAGE - off, n - t)
+                fmt, slot = self.table[s][page]
+                assert fmt == FP8
+                st = self.fp8[slot]
+                for h in range(self.Hkv):
+                    for which, src in ((0, k), (1, v)):
+                        x = src[row + t:row + t + cnt, h, :]
+                        codes, sc = F.fp8_write(st[which][h], st[2 + which][h], off, x)
+                        st[which][h] = codes
+                        st[2 + which][h] = sc
+                t += cnt
+            self.ctx[s] = L0 + n
+            row += n
+
+    # ------------------------------------------------------------------ policy
+    def is_anchor(self, seq, page, window_tokens) -> bool:
+        L = self.ctx[seq]
+        return (page < self.sink_pages or PAGE * page + PAGE > L - window_tokens
+                or page in self.protected[seq])
+
+    def set_protected(self, seq, page, flag):
+        self._check_seq(seq)
+        if not (0 <= page < len(self.table[seq])):
+            raise PoolError("INVALID_ARG", "page not mapped")
+        if flag:
+            self.protected[seq].add(page)
+        else:
+            self.protected[seq].discard(page)
+
+    def demote_candidates(self, seq, window_tokens):
+        L = self.ctx[seq]
+        out = []
+        for p, (fmt, _) in enumerate(self.table[seq]):
+            if fmt == FP8 and PAGE * (p + 1) <= L and not self.is_anchor(seq, p, window_tokens):
+                out.append(p)
+        return out
+
+    def demote(self, seq_ids, window_tokens):
+        """Convert every full, non-anchor FP8 page of the listed sequences to TQ3.
+        Returns [(seq, page, fp8_slot, tq3_slot)] in processing order."""
+        seq_ids = [int(s) for s in seq_ids]
+        for s in seq_ids:
+            self._check_seq(s)
+        if len(set(seq_ids)) != len(seq_ids) or window_tokens < 0:
+            raise PoolError("INVALID_ARG", "repeated sequence or negative window")
+        work = [(s, p) for s in seq_ids for p in self.demote_candidates(s, window_tokens)]
+        if len(work) > len(self.alloc[TQ3].free):
+            raise PoolError("OUT_OF_PAGES", "TQ3 pool exhausted")
+        done, freed = [], []
+        for s, p in work:
+            _, src = self.table[s][p]
+            dst = self.alloc[TQ3].take()
+            self.tq3[dst] = self.convert(src)
+            self.table[s][p] = (TQ3, dst)
+            done.append((s, p, src, dst))
+            freed.append(src)
+        for src in freed:
+            del self.fp8[src]
+            self.alloc[FP8].give(src)
+        return done
+
+    def convert(self, fp8_slot):
+        """TQ3 contents of a full FP8 page: x = fp32(dec(code) * scale), then per group of
+        32 channels of each (token, head, K-or-V) quantise to 3 bits."""
+        kc, vc, ks, vs = self.fp8[fp8_slot]
+        res = []
+        for codes, scales in ((kc, ks), (vc, vs)):
+            x = F.f32(F.e4m3_decode(codes) * scales[:, None, None])       # [Hkv,16,D]
+            q, s = F.tq3_quantize(x.reshape(self.Hkv, PAGE, self.G, F.TQ3_GROUP))
+            res += [q.reshape(self.Hkv, PAGE, self.D), s]
+        return res
+
+    # ------------------------------------------------------------------ lifecycle
+    def seq_reset(self, seq):
+        self._check_seq(seq)
+        freed = [[], []]
+        for fmt, slot in self.table[seq]:
+            freed[fmt].append(slot)
+        for fmt in (FP8, TQ3):
+            for slot in freed[fmt]:
+                (self.fp8 if fmt == FP8 else self.tq3).pop(slot)
+                self.alloc[fmt].give(slot)
+        self.table[seq] = []
+        self.ctx[seq] = 0
+        self.protected[seq] = set()
+
+    def seq_copy(self, src, dst):
+        """Give ``dst`` (empty) its own copy of every page of ``src``; formats kept."""
+        self._check_seq(src)
+        self._check_seq(dst)
+        if src == dst or self.table[dst] or self.ctx[dst]:
+            raise PoolError("INVALID_ARG", "destination must be a different, empty sequence")
+        need = [0, 0]
+        for fmt, _ in self.table[src]:
+            need[fmt] += 1
+        for fmt in (FP8, TQ3):
+            if need[fmt] > len(self.alloc[fmt].free):
+                raise PoolError("OUT_OF_PAGES", "pool exhausted")
+        for fmt, slot in self.table[src]:
+            new = self.alloc[fmt].take()
+            store = self.fp8 if fmt == FP8 else self.tq3
+            store[new] = [np.array(a, copy=True) for a in store[slot]]
+            self.table[dst].append((fmt, new))
+        self.ctx[dst] = self.ctx[src]
+        self.protected[dst] = set(self.protected[src])
+
+    # ------------------------------------------------------------------ views
+    def slot_bytes(self, entry: int):
+        fmt, slot = entry >> 30, entry & ((1 << 30) - 1)
+        if fmt == FP8:
+            kc, vc, ks, vs = self.fp8[slot]
+            return F.fp8_slot_bytes(kc, vc, ks, vs)
+        kq, ks, vq, vs = self.tq3[slot]
+        return F.tq3_slot_bytes(kq, ks, vq, vs)
+
+    def dequant_seq(self, seq, heads=None):
+        """Dequantised K and V of a sequence: float64 [L, Hkv, D] each (exact values)."""
+        L = self.ctx[seq]
+        heads = range(self.Hkv) if heads is None else heads
+        nh = len(list(heads))
+        K = np.zeros((len(self.table[seq]) * PAGE, nh, self.D))
+        V = np.zeros_like(K)
+        for p, (fmt, slot) in enumerate(self.table[seq]):
+            rows = slice(p * PAGE, (p + 1) * PAGE)
+            for j, h in enumerate(heads):
+                if fmt == FP8:
+                    kc, vc, ks, vs = self.fp8[slot]
+                    K[rows, j] = F.fp8_dequant(kc[h], ks[h])
+                    V[rows, j] = F.fp8_dequant(vc[h], vs[h])
+                else:
+                    kq, kscale, vq, vscale = self.tq3[slot]
+                    K[rows, j] = F.tq3_dequant(kq[h].reshape(PAGE, self.G, F.TQ3_GROUP),
+                                               kscale[h]).reshape(PAGE, self.D)
+                    V[rows, j] = F.tq3_dequant(vq[h].reshape(PAGE, self.G, F.TQ3_GROUP),
+                                               vscale[h]).reshape(PAGE, self.D)
+        return K[:L], V[:L]
+
+    def stats(self):
+        live = sum(self.ctx)
+        n8 = sum(1 for t in self.table for f, _ in t if f == FP8)
+        n3 = sum(1 for t in self.table for f, _ in t if f == TQ3)
+        kv_bytes = n8 * self.Hkv * F.fp8_head_bytes(self.D) + n3 * self.Hkv * F.tq3_head_bytes(self.D)
+        return live, n8, n3, (kv_bytes / live if live else 0.0)
