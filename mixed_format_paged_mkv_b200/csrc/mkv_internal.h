@@ -1,0 +1,118 @@
+// Host <-> kernel parameter blocks of the mixed-format paged KV cache (not part of the ABI).
+//
+// Every kernel takes one parameter block by value (__grid_constant__), so a launch carries its
+// own descriptors: no staging buffer, no host->device copy before the kernel can start.  The
+// blocks stay below the 32 KiB kernel-parameter limit; larger requests are split into several
+// launches by the host code.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mkv {
+
+constexpr int kPageTokens = 16;
+constexpr int kFmtShift = 30;
+constexpr uint32_t kSlotMask = (1u << kFmtShift) - 1u;
+
+// Bits of the device status word.
+constexpr int32_t kStatusCheck = 1;    // invalid table entry, slot or non-finite input
+constexpr int32_t kStatusTimeout = 2;  // a bounded wait ran out
+
+// Bytes of one KV head inside a slot.
+inline int64_t fp8_head_bytes(int D) { return 32LL * D + 16; }
+inline int64_t tq3_head_bytes(int D) { return 14LL * D; }
+
+// ------------------------------------------------------------------ append (FP8 page write)
+struct AppendDesc {
+  int32_t slot;         // FP8 slot of the page
+  int32_t table_index;  // row * max_pages + logical page (written when the page is new)
+  int32_t first_row;    // input row of the first token written into this page
+  int16_t n_old;        // tokens already in the page
+  int16_t n_new;        // tokens written by this call
+};
+constexpr int kAppendMaxDesc = 1536;
+struct AppendParams {
+  uint8_t* fp8_slab;
+  int32_t* tables;
+  int32_t* status;
+  const uint16_t* k;  // bf16 bits [rows][Hkv][D]
+  const uint16_t* v;
+  int64_t slot_bytes;
+  int32_t Hkv, D;
+  int32_t n_desc;
+  AppendDesc desc[kAppendMaxDesc];
+};
+
+// ------------------------------------------------------------------ demote (FP8 -> TQ3)
+struct DemoteDesc {
+  int32_t src_slot;     // FP8 slot
+  int32_t dst_slot;     // TQ3 slot
+  int32_t table_index;  // entry retagged to TQ3
+};
+constexpr int kDemoteMaxDesc = 2560;
+struct DemoteParams {
+  const uint8_t* fp8_slab;
+  uint8_t* tq3_slab;
+  int32_t* tables;
+  int64_t fp8_slot_bytes, tq3_slot_bytes;
+  int32_t Hkv, D;
+  int32_t n_desc;
+  DemoteDesc desc[kDemoteMaxDesc];
+};
+
+// ------------------------------------------------------------------ slot copy
+struct CopyDesc {
+  int32_t src_slot, dst_slot, fmt, table_index;
+};
+constexpr int kCopyMaxDesc = 1920;
+struct CopyParams {
+  uint8_t* fp8_slab;
+  uint8_t* tq3_slab;
+  int32_t* tables;
+  int64_t fp8_slot_bytes, tq3_slot_bytes;
+  int32_t n_desc;
+  CopyDesc desc[kCopyMaxDesc];
+};
+
+// ------------------------------------------------------------------ decode
+struct SeqDesc {
+  int32_t row;             // table row (sequence id)
+  int32_t ctx;             // context length L (includes the q_len new tokens)
+  int32_t n_pages;         // mapped pages
+  int32_t n8, n3;          // FP8 / TQ3 pages (host counts; the plan kernel checks them)
+  int32_t list8, list3;    // offsets of the sequence's FP8 / TQ3 page lists (int2 entries)
+  int32_t split8, split3;  // partial-attention CTAs per KV head for each format
+  int32_t cta0;            // first CTA (grid x) of this sequence
+  int32_t part0;           // first partial-state index of this sequence
+  int32_t out_row;         // position of the sequence in the call (rows of q and out)
+};
+constexpr int kDecodeMaxSeqs = 480;
+struct DecodeParams {
+  const uint8_t* fp8_slab;
+  const uint8_t* tq3_slab;
+  const int32_t* tables;
+  int32_t* status;
+  const uint16_t* q;  // bf16 bits [n][q_len][Hq][D]
+  float* out;         // fp32 [n][q_len][Hq][D]
+  int2* lists;        // page lists: {slot, logical page}
+  float* part_ml;     // [part][Hkv][NC][2]: running max (log2 units), denominator
+  float* part_acc;    // [part][Hkv][NC][D]: unnormalised accumulator
+  int64_t fp8_slot_bytes, tq3_slot_bytes;
+  int32_t Hkv, D, g, q_len, NC, Hq;
+  int32_t max_pages, fp8_slots, tq3_slots;
+  int32_t P8, P3;      // pages per CTA for each format
+  float logit_scale;   // sm_scale * log2(e)
+  int32_t n_seqs;      // sequences in this launch
+  int32_t total_ctas;  // partial CTAs per KV head in this launch
+  SeqDesc seq[kDecodeMaxSeqs];
+};
+
+cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
+cudaError_t launch_demote(const DemoteParams& p, cudaStream_t s);
+cudaError_t launch_copy(const CopyParams& p, cudaStream_t s);
+cudaError_t launch_plan(const DecodeParams& p, cudaStream_t s);
+cudaError_t launch_partial(const DecodeParams& p, cudaStream_t s);
+cudaError_t launch_merge(const DecodeParams& p, cudaStream_t s);
+bool partial_supported(int D, int NC);
+
+}  // namespace mkv

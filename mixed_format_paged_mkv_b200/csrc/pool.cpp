@@ -1,0 +1,739 @@
+// Host side of the mixed-format paged KV cache: allocator, block tables, anchor policy,
+// decode planning and the C ABI declared in include/mkv.h.
+//
+// "Minima-KV ..." (brainszone.ai pt page, sections "O que os autores propõem" and "Âncoras em
+// FP8, arquivo em TQ3"): pages of a live request stay addressable; recent and protected pages
+// are FP8 anchors; older non-anchor pages are converted to packed TQ3.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <functional>
+#include <string>
+#include <vector>
+
+#include "mkv.h"
+#include "mkv_internal.h"
+
+using namespace mkv;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int ok() {
+  g_last_error.clear();
+  return MKV_OK;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(MKV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Free slots handed out lowest rank first; rank = position in the slot order.
+struct Allocator {
+  int32_t n = 0;
+  std::vector<int32_t> rank;
+  std::vector<uint8_t> is_free;
+  std::vector<uint64_t> heap;  // (rank << 32) | slot, min-heap
+  int32_t n_free = 0;
+
+  void init(int32_t slots) {
+    n = slots;
+    rank.resize(n);
+    is_free.assign(n, 1);
+    for (int32_t i = 0; i < n; ++i) rank[i] = i;
+    rebuild();
+  }
+  void rebuild() {
+    heap.clear();
+    n_free = 0;
+    for (int32_t s = 0; s < n; ++s)
+      if (is_free[s]) {
+        heap.push_back((static_cast<uint64_t>(rank[s]) << 32) | static_cast<uint32_t>(s));
+        ++n_free;
+      }
+    std::make_heap(heap.begin(), heap.end(), std::greater<uint64_t>());
+  }
+  int32_t take() {
+    std::pop_heap(heap.begin(), heap.end(), std::greater<uint64_t>());
+    const int32_t s = static_cast<int32_t>(heap.back() & 0xffffffffu);
+    heap.pop_back();
+    is_free[s] = 0;
+    --n_free;
+    return s;
+  }
+  void give(int32_t s) {
+    is_free[s] = 1;
+    ++n_free;
+    heap.push_back((static_cast<uint64_t>(rank[s]) << 32) | static_cast<uint32_t>(s));
+    std::push_heap(heap.begin(), heap.end(), std::greater<uint64_t>());
+  }
+};
+
+struct Seq {
+  std::vector<int32_t> table;     // block-table entries
+  std::vector<int32_t> fp8_pages; // logical pages currently FP8, ascending
+  std::vector<uint8_t> prot;      // protected flag per logical page
+  int32_t ctx = 0;
+  int32_t n3 = 0;
+};
+
+inline int32_t entry_of(int fmt, int32_t slot) {
+  return static_cast<int32_t>((static_cast<uint32_t>(fmt) << kFmtShift) | static_cast<uint32_t>(slot));
+}
+inline int fmt_of(int32_t e) { return static_cast<int>(static_cast<uint32_t>(e) >> kFmtShift); }
+inline int32_t slot_of(int32_t e) { return static_cast<int32_t>(static_cast<uint32_t>(e) & kSlotMask); }
+
+struct TimingRec {
+  cudaEvent_t ev[4];
+};
+
+}  // namespace
+
+struct mkv_pool {
+  mkv_pool_config cfg{};
+  bool host_only = false;
+  uint8_t* fp8_slab = nullptr;
+  uint8_t* tq3_slab = nullptr;
+  int32_t* d_tables = nullptr;
+  int32_t* d_status = nullptr;
+  int64_t fp8_slot_bytes = 0, tq3_slot_bytes = 0;
+  int sm_count = 148;
+  std::vector<Seq> seqs;
+  Allocator alloc[2];
+  int64_t launches = 0;
+  bool timing = false;
+  std::vector<TimingRec> timing_recs;
+  std::vector<cudaEvent_t> spare_events;
+};
+
+namespace {
+
+bool valid_pool(mkv_pool_t p) { return p != nullptr; }
+
+int check_seq(mkv_pool_t p, int32_t s) {
+  if (s < 0 || s >= p->cfg.max_seqs)
+    return fail(MKV_ERR_BAD_SEQ, "sequence %d outside [0, %d)", s, p->cfg.max_seqs);
+  return MKV_OK;
+}
+
+int validate_config(const mkv_pool_config* c) {
+  if (!c) return fail(MKV_ERR_INVALID_ARG, "config is NULL");
+  if (c->num_kv_heads < 1) return fail(MKV_ERR_INVALID_ARG, "num_kv_heads must be >= 1");
+  if (c->head_dim != 64 && c->head_dim != 128 && c->head_dim != 256)
+    return fail(MKV_ERR_UNSUPPORTED, "head_dim %d not built (64, 128, 256)", c->head_dim);
+  if (c->page_size != kPageTokens) return fail(MKV_ERR_INVALID_ARG, "page_size must be 16");
+  if (c->max_seqs < 1 || c->max_pages_per_seq < 1)
+    return fail(MKV_ERR_INVALID_ARG, "max_seqs and max_pages_per_seq must be >= 1");
+  if (c->fp8_slots < 1 || c->tq3_slots < 0 || c->fp8_slots > static_cast<int32_t>(kSlotMask) ||
+      c->tq3_slots > static_cast<int32_t>(kSlotMask))
+    return fail(MKV_ERR_INVALID_ARG, "slot counts out of range");
+  if (c->sink_pages < 0) return fail(MKV_ERR_INVALID_ARG, "sink_pages must be >= 0");
+  if (c->flags & ~MKV_POOL_HOST_ONLY) return fail(MKV_ERR_INVALID_ARG, "unknown flags");
+  if (static_cast<int64_t>(c->max_seqs) * c->max_pages_per_seq > (1LL << 31) - 1)
+    return fail(MKV_ERR_INVALID_ARG, "table too large");
+  return MKV_OK;
+}
+
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+// Pages of work per partial-attention CTA: enough CTAs for about four waves of two CTAs per
+// SM, an FP8 page counting as two TQ3 pages of bytes.
+void choose_split(const mkv_pool_t p, int64_t pages8, int64_t pages3, int32_t* P8, int32_t* P3) {
+  const int64_t work = (2 * pages8 + pages3) * p->cfg.num_kv_heads;
+  const int64_t target_ctas = static_cast<int64_t>(p->sm_count) * 2 * 4;
+  int64_t per = (work + target_ctas - 1) / target_ctas;
+  per = std::max<int64_t>(4, std::min<int64_t>(256, per));
+  *P3 = static_cast<int32_t>(per);
+  *P8 = static_cast<int32_t>(std::max<int64_t>(2, per / 2));
+}
+
+struct DecodePlan {
+  int32_t NC = 0, g = 0, P8 = 0, P3 = 0;
+  std::vector<SeqDesc> seq;
+  int64_t list_entries = 0, parts = 0;
+  size_t off_lists = 0, off_ml = 0, off_acc = 0, bytes = 0;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+int plan_decode(mkv_pool_t p, const int32_t* seq_ids, int32_t n, int32_t q_len, int32_t Hq,
+                DecodePlan* plan) {
+  if (n < 0 || (n > 0 && !seq_ids)) return fail(MKV_ERR_INVALID_ARG, "bad sequence list");
+  if (q_len < 1) return fail(MKV_ERR_INVALID_ARG, "q_len must be >= 1");
+  const int Hkv = p->cfg.num_kv_heads;
+  if (Hq < Hkv || Hq % Hkv) return fail(MKV_ERR_INVALID_ARG, "num_q_heads %d not a multiple of Hkv %d", Hq, Hkv);
+  plan->g = Hq / Hkv;
+  plan->NC = q_len * plan->g;
+  if (!partial_supported(p->cfg.head_dim, plan->NC))
+    return fail(MKV_ERR_UNSUPPORTED, "q_len * num_q_heads / Hkv = %d > 32 is not built", plan->NC);
+  int64_t n8 = 0, n3 = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    if (int e = check_seq(p, seq_ids[i])) return e;
+    const Seq& s = p->seqs[seq_ids[i]];
+    if (s.ctx < q_len || s.ctx == 0)
+      return fail(MKV_ERR_EMPTY_CONTEXT, "sequence %d has %d tokens < q_len %d", seq_ids[i], s.ctx, q_len);
+    n8 += static_cast<int64_t>(s.fp8_pages.size());
+    n3 += s.n3;
+  }
+  choose_split(p, n8, n3, &plan->P8, &plan->P3);
+  plan->seq.resize(n);
+  int64_t lists = 0, parts = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    const Seq& s = p->seqs[seq_ids[i]];
+    SeqDesc& d = plan->seq[i];
+    d.row = seq_ids[i];
+    d.ctx = s.ctx;
+    d.n_pages = static_cast<int32_t>(s.table.size());
+    d.n8 = static_cast<int32_t>(s.fp8_pages.size());
+    d.n3 = s.n3;
+    d.list8 = static_cast<int32_t>(lists);
+    d.list3 = static_cast<int32_t>(lists + d.n8);
+    lists += d.n8 + d.n3;
+    d.split8 = (d.n8 + plan->P8 - 1) / plan->P8;
+    d.split3 = (d.n3 + plan->P3 - 1) / plan->P3;
+    d.part0 = static_cast<int32_t>(parts);
+    parts += d.split8 + d.split3;
+    d.out_row = i;
+    d.cta0 = 0;  // per launch
+  }
+  if (lists > INT32_MAX || parts > INT32_MAX) return fail(MKV_ERR_INVALID_ARG, "call too large");
+  plan->list_entries = lists;
+  plan->parts = parts;
+  const int64_t cols = static_cast<int64_t>(parts) * Hkv * plan->NC;
+  plan->off_lists = 0;
+  plan->off_ml = align256(static_cast<size_t>(lists) * 8);
+  plan->off_acc = plan->off_ml + align256(static_cast<size_t>(cols) * 2 * 4);
+  plan->bytes = plan->off_acc + align256(static_cast<size_t>(cols) * p->cfg.head_dim * 4);
+  if (plan->bytes == 0) plan->bytes = 256;
+  return MKV_OK;
+}
+
+cudaEvent_t get_event(mkv_pool_t p) {
+  if (!p->spare_events.empty()) {
+    cudaEvent_t e = p->spare_events.back();
+    p->spare_events.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+const char* mkv_last_error(void) { return g_last_error.c_str(); }
+
+int mkv_pool_required_bytes(const mkv_pool_config* cfg, size_t* fp8_slab, size_t* tq3_slab,
+                            size_t* tables, size_t* status) {
+  if (int e = validate_config(cfg)) return e;
+  const size_t Hkv = cfg->num_kv_heads, D = cfg->head_dim;
+  if (fp8_slab) *fp8_slab = static_cast<size_t>(cfg->fp8_slots) * Hkv * fp8_head_bytes(D);
+  if (tq3_slab) *tq3_slab = static_cast<size_t>(cfg->tq3_slots) * Hkv * tq3_head_bytes(D);
+  if (tables) *tables = static_cast<size_t>(cfg->max_seqs) * cfg->max_pages_per_seq * 4;
+  if (status) *status = 16;
+  return ok();
+}
+
+int mkv_pool_create(const mkv_pool_config* cfg, void* fp8_slab, void* tq3_slab,
+                    int32_t* d_tables, int32_t* d_status, mkv_pool_t* out) {
+  if (int e = validate_config(cfg)) return e;
+  if (!out) return fail(MKV_ERR_INVALID_ARG, "out is NULL");
+  const bool host_only = (cfg->flags & MKV_POOL_HOST_ONLY) != 0;
+  if (host_only) {
+    if (fp8_slab || tq3_slab || d_tables || d_status)
+      return fail(MKV_ERR_INVALID_ARG, "host-only pools take no device buffers");
+  } else {
+    if (!fp8_slab || (!tq3_slab && cfg->tq3_slots > 0) || !d_tables || !d_status)
+      return fail(MKV_ERR_INVALID_ARG, "device buffers must not be NULL");
+    const uintptr_t a = reinterpret_cast<uintptr_t>(fp8_slab) | reinterpret_cast<uintptr_t>(tq3_slab) |
+                        reinterpret_cast<uintptr_t>(d_tables) | reinterpret_cast<uintptr_t>(d_status);
+    if (a & 255) return fail(MKV_ERR_INVALID_ARG, "device buffers must be 256-byte aligned");
+  }
+  mkv_pool* p = new mkv_pool();
+  p->cfg = *cfg;
+  p->host_only = host_only;
+  p->fp8_slab = static_cast<uint8_t*>(fp8_slab);
+  p->tq3_slab = static_cast<uint8_t*>(tq3_slab);
+  p->d_tables = d_tables;
+  p->d_status = d_status;
+  p->fp8_slot_bytes = static_cast<int64_t>(cfg->num_kv_heads) * fp8_head_bytes(cfg->head_dim);
+  p->tq3_slot_bytes = static_cast<int64_t>(cfg->num_kv_heads) * tq3_head_bytes(cfg->head_dim);
+  p->seqs.resize(cfg->max_seqs);
+  p->alloc[0].init(cfg->fp8_slots);
+  p->alloc[1].init(cfg->tq3_slots);
+  if (!host_only) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&p->sm_count, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess)
+      e = cudaMemsetAsync(d_tables, 0xFF, static_cast<size_t>(cfg->max_seqs) * cfg->max_pages_per_seq * 4, 0);
+    if (e == cudaSuccess) e = cudaMemsetAsync(d_status, 0, 16, 0);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(0);
+    if (e != cudaSuccess) {
+      delete p;
+      return cuda_fail(e, "pool init");
+    }
+  }
+  *out = p;
+  return ok();
+}
+
+void mkv_pool_destroy(mkv_pool_t p) {
+  if (!p) return;
+  for (auto& r : p->timing_recs)
+    for (auto e : r.ev) cudaEventDestroy(e);
+  for (auto e : p->spare_events) cudaEventDestroy(e);
+  delete p;
+}
+
+int mkv_pool_set_slot_order(mkv_pool_t p, int32_t fmt, const int32_t* order, int32_t n) {
+  if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
+  if (fmt != MKV_FMT_FP8 && fmt != MKV_FMT_TQ3) return fail(MKV_ERR_INVALID_ARG, "bad format");
+  Allocator& a = p->alloc[fmt];
+  if (n != a.n || (n > 0 && !order)) return fail(MKV_ERR_INVALID_ARG, "order must list all %d slots", a.n);
+  std::vector<uint8_t> seen(n, 0);
+  for (int32_t i = 0; i < n; ++i) {
+    if (order[i] < 0 || order[i] >= n || seen[order[i]])
+      return fail(MKV_ERR_INVALID_ARG, "order is not a permutation");
+    seen[order[i]] = 1;
+  }
+  for (int32_t i = 0; i < n; ++i) a.rank[order[i]] = i;
+  a.rebuild();
+  return ok();
+}
+
+int mkv_append_kv(mkv_pool_t p, const int32_t* seq_ids, const int32_t* n_new, int32_t n_seqs,
+                  const void* k_bf16, const void* v_bf16, void* stream) {
+  if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
+  if (n_seqs < 0 || (n_seqs > 0 && (!seq_ids || !n_new)))
+    return fail(MKV_ERR_INVALID_ARG, "bad sequence list");
+  const int32_t MP = p->cfg.max_pages_per_seq;
+  int64_t need = 0, rows = 0;
+  std::vector<uint8_t> seen(p->cfg.max_seqs, 0);
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    if (int e = check_seq(p, seq_ids[i])) return e;
+    if (seen[seq_ids[i]]) return fail(MKV_ERR_INVALID_ARG, "sequence %d listed twice", seq_ids[i]);
+    seen[seq_ids[i]] = 1;
+    if (n_new[i] < 0) return fail(MKV_ERR_INVALID_ARG, "negative token count");
+    const Seq& s = p->seqs[seq_ids[i]];
+    const int64_t pages_after = (static_cast<int64_t>(s.ctx) + n_new[i] + kPageTokens - 1) / kPageTokens;
+    if (pages_after > MP)
+      return fail(MKV_ERR_OUT_OF_PAGES, "sequence %d would need %lld pages > %d", seq_ids[i],
+                  static_cast<long long>(pages_after), MP);
+    need += pages_after - static_cast<int64_t>(s.table.size());
+    rows += n_new[i];
+  }
+  if (need > p->alloc[0].n_free)
+    return fail(MKV_ERR_OUT_OF_PAGES, "FP8 slab has %d free slots, %lld needed", p->alloc[0].n_free,
+                static_cast<long long>(need));
+  if (rows > 0 && !p->host_only && (!k_bf16 || !v_bf16))
+    return fail(MKV_ERR_INVALID_ARG, "k/v are NULL");
+  if (rows > INT32_MAX) return fail(MKV_ERR_INVALID_ARG, "too many tokens");
+
+  // ---- commit host state, collect page writes
+  std::vector<AppendDesc> descs;
+  int32_t row = 0;
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    Seq& s = p->seqs[seq_ids[i]];
+    const int32_t L0 = s.ctx, n = n_new[i];
+    const int32_t pages_after = (L0 + n + kPageTokens - 1) / kPageTokens;
+    if (s.prot.size() < static_cast<size_t>(pages_after)) s.prot.resize(pages_after, 0);
+    while (static_cast<int32_t>(s.table.size()) < pages_after) {
+      const int32_t slot = p->alloc[0].take();
+      s.fp8_pages.push_back(static_cast<int32_t>(s.table.size()));
+      s.table.push_back(entry_of(MKV_FMT_FP8, slot));
+    }
+    for (int32_t t = 0; t < n;) {
+      const int32_t pos = L0 + t, page = pos / kPageTokens, off = pos % kPageTokens;
+      const int32_t cnt = std::min(kPageTokens - off, n - t);
+      AppendDesc d;
+      d.slot = slot_of(s.table[page]);
+      d.table_index = seq_ids[i] * MP + page;
+      d.first_row = row + t;
+      d.n_old = static_cast<int16_t>(off);
+      d.n_new = static_cast<int16_t>(cnt);
+      descs.push_back(d);
+      t += cnt;
+    }
+    s.ctx = L0 + n;
+    row += n;
+  }
+  if (p->host_only) return ok();
+  AppendParams* prm = new AppendParams;
+  prm->fp8_slab = p->fp8_slab;
+  prm->tables = p->d_tables;
+  prm->status = p->d_status;
+  prm->k = static_cast<const uint16_t*>(k_bf16);
+  prm->v = static_cast<const uint16_t*>(v_bf16);
+  prm->slot_bytes = p->fp8_slot_bytes;
+  prm->Hkv = p->cfg.num_kv_heads;
+  prm->D = p->cfg.head_dim;
+  for (size_t b = 0; b < descs.size(); b += kAppendMaxDesc) {
+    const size_t m = std::min<size_t>(kAppendMaxDesc, descs.size() - b);
+    prm->n_desc = static_cast<int32_t>(m);
+    std::memcpy(prm->desc, descs.data() + b, m * sizeof(AppendDesc));
+    cudaError_t e = launch_append(*prm, as_stream(stream));
+    ++p->launches;
+    if (e != cudaSuccess) {
+      delete prm;
+      return cuda_fail(e, "append launch");
+    }
+  }
+  delete prm;
+  return ok();
+}
+
+int mkv_set_protected(mkv_pool_t p, int32_t seq, int32_t page, int32_t flag) {
+  if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
+  if (int e = check_seq(p, seq)) return e;
+  Seq& s = p->seqs[seq];
+  if (page < 0 || page >= static_cast<int32_t>(s.table.size()))
+    return fail(MKV_ERR_INVALID_ARG, "page %d of sequence %d is not mapped", page, seq);
+  s.prot[page] = flag ? 1 : 0;
+  return ok();
+}
+
+int mkv_demote_pages(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, int32_t window,
+                     int32_t* n_demoted, void* stream) {
+  if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
+  if (n_seqs < 0 || (n_seqs > 0 && !seq_ids)) return fail(MKV_ERR_INVALID_ARG, "bad sequence list");
+  if (window < 0) return fail(MKV_ERR_INVALID_ARG, "window must be >= 0");
+  std::vector<uint8_t> seen(p->cfg.max_seqs, 0);
+  struct Work { int32_t seq, page; };
+  std::vector<Work> work;
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    if (int e = check_seq(p, seq_ids[i])) return e;
+    if (seen[seq_ids[i]]) return fail(MKV_ERR_INVALID_ARG, "sequence %d listed twice", seq_ids[i]);
+    seen[seq_ids[i]] = 1;
+    const Seq& s = p->seqs[seq_ids[i]];
+    const int64_t L = s.ctx;
+    for (int32_t pg : s.fp8_pages) {
+      const bool full = static_cast<int64_t>(kPageTokens) * (pg + 1) <= L;
+      const bool anchor = pg < p->cfg.sink_pages ||
+                          static_cast<int64_t>(kPageTokens) * pg + kPageTokens > L - window ||
+                          s.prot[pg];
+      if (full && !anchor) work.push_back({seq_ids[i], pg});
+    }
+  }
+  if (static_cast<int64_t>(work.size()) > p->alloc[1].n_free)
+    return fail(MKV_ERR_OUT_OF_PAGES, "TQ3 slab has %d free slots, %zu needed", p->alloc[1].n_free, work.size());
+  std::vector<DemoteDesc> descs;
+  std::vector<int32_t> freed;
+  descs.reserve(work.size());
+  for (const Work& w : work) {
+    Seq& s = p->seqs[w.seq];
+    const int32_t src = slot_of(s.table[w.page]);
+    const int32_t dst = p->alloc[1].take();
+    s.table[w.page] = entry_of(MKV_FMT_TQ3, dst);
+    s.n3 += 1;
+    descs.push_back({src, dst, w.seq * p->cfg.max_pages_per_seq + w.page});
+    freed.push_back(src);
+  }
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    Seq& s = p->seqs[seq_ids[i]];
+    s.fp8_pages.erase(std::remove_if(s.fp8_pages.begin(), s.fp8_pages.end(),
+                                     [&](int32_t pg) { return fmt_of(s.table[pg]) != MKV_FMT_FP8; }),
+                      s.fp8_pages.end());
+  }
+  if (n_demoted) *n_demoted = static_cast<int32_t>(descs.size());
+  if (!p->host_only && !descs.empty()) {
+    DemoteParams* prm = new DemoteParams;
+    prm->fp8_slab = p->fp8_slab;
+    prm->tq3_slab = p->tq3_slab;
+    prm->tables = p->d_tables;
+    prm->fp8_slot_bytes = p->fp8_slot_bytes;
+    prm->tq3_slot_bytes = p->tq3_slot_bytes;
+    prm->Hkv = p->cfg.num_kv_heads;
+    prm->D = p->cfg.head_dim;
+    for (size_t b = 0; b < descs.size(); b += kDemoteMaxDesc) {
+      const size_t m = std::min<size_t>(kDemoteMaxDesc, descs.size() - b);
+      prm->n_desc = static_cast<int32_t>(m);
+      std::memcpy(prm->desc, descs.data() + b, m * sizeof(DemoteDesc));
+      cudaError_t e = launch_demote(*prm, as_stream(stream));
+      ++p->launches;
+      if (e != cudaSuccess) {
+        delete prm;
+        for (int32_t s : freed) p->alloc[0].give(s);
+        return cuda_fail(e, "demote launch");
+      }
+    }
+    delete prm;
+  }
+  for (int32_t s : freed) p->alloc[0].give(s);
+  return ok();
+}
+
+int mkv_decode_workspace_bytes(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs,
+                               int32_t q_len, int32_t Hq, size_t* bytes) {
+  if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
+  if (!bytes) return fail(MKV_ERR_INVALID_ARG, "bytes is NULL");
+  DecodePlan plan;
+  if (int e = plan_decode(p, seq_ids, n_seqs, q_len, Hq, &plan)) return e;
+  *bytes = plan.bytes;
+  return ok();
+}
+
+int mkv_decode_attention(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, int32_t q_len,
+                         const void* q_bf16, int32_t Hq, float sm_scale, float* out,
+                         void* workspace, size_t ws_bytes, void* stream) {
+  if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
+  if (p->host_only) return fail(MKV_ERR_INVALID_ARG, "host-only pool cannot decode");
+  DecodePlan plan;
+  if (int e = plan_decode(p, seq_ids, n_seqs, q_len, Hq, &plan)) return e;
+  if (!std::isfinite(sm_scale)) return fail(MKV_ERR_INVALID_ARG, "sm_scale is not finite");
+  if (n_seqs == 0) return ok();
+  if (!q_bf16 || !out || !workspace) return fail(MKV_ERR_INVALID_ARG, "q/out/workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(workspace) & 255)
+    return fail(MKV_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (ws_bytes < plan.bytes)
+    return fail(MKV_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", ws_bytes, plan.bytes);
+  cudaStream_t st = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DecodeParams* prm = new DecodeParams;
+  prm->fp8_slab = p->fp8_slab;
+  prm->tq3_slab = p->tq3_slab;
+  prm->tables = p->d_tables;
+  prm->status = p->d_status;
+  prm->q = static_cast<const uint16_t*>(q_bf16);
+  prm->out = out;
+  prm->lists = reinterpret_cast<int2*>(ws + plan.off_lists);
+  prm->part_ml = reinterpret_cast<float*>(ws + plan.off_ml);
+  prm->part_acc = reinterpret_cast<float*>(ws + plan.off_acc);
+  prm->fp8_slot_bytes = p->fp8_slot_bytes;
+  prm->tq3_slot_bytes = p->tq3_slot_bytes;
+  prm->Hkv = p->cfg.num_kv_heads;
+  prm->D = p->cfg.head_dim;
+  prm->g = plan.g;
+  prm->q_len = q_len;
+  prm->NC = plan.NC;
+  prm->Hq = Hq;
+  prm->max_pages = p->cfg.max_pages_per_seq;
+  prm->fp8_slots = p->cfg.fp8_slots;
+  prm->tq3_slots = p->cfg.tq3_slots;
+  prm->P8 = plan.P8;
+  prm->P3 = plan.P3;
+  prm->logit_scale = sm_scale * 1.4426950408889634f;
+  TimingRec rec{};
+  bool timed = p->timing;
+  if (timed) {
+    for (auto& e : rec.ev) {
+      e = get_event(p);
+      if (!e) timed = false;
+    }
+  }
+  cudaError_t err = cudaSuccess;
+  for (int32_t b = 0; b < n_seqs && err == cudaSuccess; b += kDecodeMaxSeqs) {
+    const int32_t m = std::min<int32_t>(kDecodeMaxSeqs, n_seqs - b);
+    int32_t ctas = 0;
+    for (int32_t i = 0; i < m; ++i) {
+      prm->seq[i] = plan.seq[b + i];
+      prm->seq[i].cta0 = ctas;
+      ctas += prm->seq[i].split8 + prm->seq[i].split3;
+    }
+    prm->n_seqs = m;
+    prm->total_ctas = ctas;
+    const bool first = b == 0, last = b + m >= n_seqs;
+    if (timed && first) err = cudaEventRecord(rec.ev[0], st);
+    if (err == cudaSuccess) err = launch_plan(*prm, st), ++p->launches;
+    if (timed && first && err == cudaSuccess) err = cudaEventRecord(rec.ev[1], st);
+    if (err == cudaSuccess) err = launch_partial(*prm, st), ++p->launches;
+    if (timed && last && err == cudaSuccess) err = cudaEventRecord(rec.ev[2], st);
+    if (err == cudaSuccess) err = launch_merge(*prm, st), ++p->launches;
+    if (timed && last && err == cudaSuccess) err = cudaEventRecord(rec.ev[3], st);
+  }
+  delete prm;
+  if (timed) {
+    if (err == cudaSuccess && n_seqs <= kDecodeMaxSeqs) p->timing_recs.push_back(rec);
+    else for (auto e : rec.ev) p->spare_events.push_back(e);
+  }
+  if (err != cudaSuccess) return cuda_fail(err, "decode launch");
+  return ok();
+}
+
+int mkv_seq_reset(mkv_pool_t p, int32_t seq, void* stream) {
+  if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
+  if (int e = check_seq(p, seq)) return e;
+  Seq& s = p->seqs[seq];
+  const size_t n = s.table.size();
+  for (int32_t e : s.table) p->alloc[fmt_of(e)].give(slot_of(e));
+  s = Seq();
+  if (!p->host_only && n > 0) {
+    cudaError_t e = cudaMemsetAsync(p->d_tables + static_cast<int64_t>(seq) * p->cfg.max_pages_per_seq,
+                                    0xFF, n * 4, as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "reset");
+  }
+  return ok();
+}
+
+int mkv_seq_copy(mkv_pool_t p, int32_t src, int32_t dst, void* stream) {
+  if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
+  if (int e = check_seq(p, src)) return e;
+  if (int e = check_seq(p, dst)) return e;
+  if (src == dst || !p->seqs[dst].table.empty() || p->seqs[dst].ctx)
+    return fail(MKV_ERR_INVALID_ARG, "destination must be a different, empty sequence");
+  const Seq& s = p->seqs[src];
+  int64_t need[2] = {0, 0};
+  for (int32_t e : s.table) need[fmt_of(e)]++;
+  for (int f = 0; f < 2; ++f)
+    if (need[f] > p->alloc[f].n_free) return fail(MKV_ERR_OUT_OF_PAGES, "slab %d exhausted", f);
+  Seq d;
+  d.ctx = s.ctx;
+  d.prot = s.prot;
+  d.n3 = s.n3;
+  d.fp8_pages = s.fp8_pages;
+  std::vector<CopyDesc> descs;
+  for (size_t pg = 0; pg < s.table.size(); ++pg) {
+    const int f = fmt_of(s.table[pg]);
+    const int32_t ns = p->alloc[f].take();
+    d.table.push_back(entry_of(f, ns));
+    descs.push_back({slot_of(s.table[pg]), ns, f, dst * p->cfg.max_pages_per_seq + static_cast<int32_t>(pg)});
+  }
+  p->seqs[dst] = d;
+  if (p->host_only) return ok();
+  CopyParams* prm = new CopyParams;
+  prm->fp8_slab = p->fp8_slab;
+  prm->tq3_slab = p->tq3_slab;
+  prm->tables = p->d_tables;
+  prm->fp8_slot_bytes = p->fp8_slot_bytes;
+  prm->tq3_slot_bytes = p->tq3_slot_bytes;
+  for (size_t b = 0; b < descs.size(); b += kCopyMaxDesc) {
+    const size_t m = std::min<size_t>(kCopyMaxDesc, descs.size() - b);
+    prm->n_desc = static_cast<int32_t>(m);
+    std::memcpy(prm->desc, descs.data() + b, m * sizeof(CopyDesc));
+    cudaError_t e = launch_copy(*prm, as_stream(stream));
+    ++p->launches;
+    if (e != cudaSuccess) {
+      delete prm;
+      return cuda_fail(e, "copy launch");
+    }
+  }
+  delete prm;
+  return ok();
+}
+
+int mkv_get_block_table(mkv_pool_t p, int32_t seq, int32_t* host_out, int32_t cap,
+                        int32_t* n_pages, int32_t* ctx_len) {
+  if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
+  if (int e = check_seq(p, seq)) return e;
+  const Seq& s = p->seqs[seq];
+  if (cap < 0 || (cap > 0 && !host_out)) return fail(MKV_ERR_INVALID_ARG, "bad output buffer");
+  const int32_t n = static_cast<int32_t>(s.table.size());
+  for (int32_t i = 0; i < std::min(cap, n); ++i) host_out[i] = s.table[i];
+  if (n_pages) *n_pages = n;
+  if (ctx_len) *ctx_len = s.ctx;
+  return ok();
+}
+
+int mkv_slot_bytes(mkv_pool_t p, int32_t fmt, size_t* bytes) {
+  if (!valid_pool(p) || !bytes) return fail(MKV_ERR_INVALID_ARG, "NULL argument");
+  if (fmt == MKV_FMT_FP8) *bytes = p->fp8_slot_bytes;
+  else if (fmt == MKV_FMT_TQ3) *bytes = p->tq3_slot_bytes;
+  else return fail(MKV_ERR_INVALID_ARG, "bad format");
+  return ok();
+}
+
+int mkv_read_slot(mkv_pool_t p, int32_t entry, void* host_out, size_t cap, void* stream) {
+  if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
+  if (p->host_only) return fail(MKV_ERR_INVALID_ARG, "host-only pool has no slabs");
+  if (entry < 0) return fail(MKV_ERR_INVALID_ARG, "unmapped entry");
+  const int f = fmt_of(entry);
+  const int32_t slot = slot_of(entry);
+  if (f > 1 || slot >= (f == 0 ? p->cfg.fp8_slots : p->cfg.tq3_slots))
+    return fail(MKV_ERR_INVALID_ARG, "entry 0x%x names no slot", entry);
+  const int64_t b = f == 0 ? p->fp8_slot_bytes : p->tq3_slot_bytes;
+  if (!host_out || cap < static_cast<size_t>(b)) return fail(MKV_ERR_INVALID_ARG, "output buffer too small");
+  const uint8_t* src = (f == 0 ? p->fp8_slab : p->tq3_slab) + slot * b;
+  cudaStream_t st = as_stream(stream);
+  cudaError_t e = cudaMemcpyAsync(host_out, src, b, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "read slot");
+  return ok();
+}
+
+int mkv_pool_stats(mkv_pool_t p, int64_t* live, int32_t* n8, int32_t* n3, double* bpt) {
+  if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
+  int64_t tokens = 0, c8 = 0, c3 = 0;
+  for (const Seq& s : p->seqs) {
+    tokens += s.ctx;
+    c8 += static_cast<int64_t>(s.fp8_pages.size());
+    c3 += s.n3;
+  }
+  if (live) *live = tokens;
+  if (n8) *n8 = static_cast<int32_t>(c8);
+  if (n3) *n3 = static_cast<int32_t>(c3);
+  if (bpt) *bpt = tokens ? static_cast<double>(c8 * p->fp8_slot_bytes + c3 * p->tq3_slot_bytes) / tokens : 0.0;
+  return ok();
+}
+
+int mkv_get_device_status(mkv_pool_t p, void* stream) {
+  if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
+  if (p->host_only) return ok();
+  cudaStream_t st = as_stream(stream);
+  int32_t h = 0;
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemcpy(&h, p->d_status, 4, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(p->d_status, 0, 4);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (h & kStatusTimeout) return fail(MKV_ERR_DEVICE_TIMEOUT, "a kernel's bounded wait ran out (status 0x%x)", h);
+  if (h & kStatusCheck) return fail(MKV_ERR_DEVICE_CHECK, "a kernel found an invalid entry or input (status 0x%x)", h);
+  return ok();
+}
+
+int mkv_timing_enable(mkv_pool_t p, int32_t enable) {
+  if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
+  p->timing = enable != 0;
+  return ok();
+}
+
+int mkv_timing_read(mkv_pool_t p, double* ms_partial, double* ms_merge, double* ms_plan,
+                    int64_t* calls) {
+  if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
+  double a = 0, b = 0, c = 0;
+  cudaError_t err = cudaSuccess;
+  for (auto& r : p->timing_recs) {
+    float t0 = 0, t1 = 0, t2 = 0;
+    if (err == cudaSuccess) err = cudaEventSynchronize(r.ev[3]);
+    if (err == cudaSuccess) err = cudaEventElapsedTime(&t0, r.ev[0], r.ev[1]);
+    if (err == cudaSuccess) err = cudaEventElapsedTime(&t1, r.ev[1], r.ev[2]);
+    if (err == cudaSuccess) err = cudaEventElapsedTime(&t2, r.ev[2], r.ev[3]);
+    c += t0;
+    a += t1;
+    b += t2;
+  }
+  const int64_t n = static_cast<int64_t>(p->timing_recs.size());
+  for (auto& r : p->timing_recs)
+    for (auto e : r.ev) p->spare_events.push_back(e);
+  p->timing_recs.clear();
+  if (err != cudaSuccess) return cuda_fail(err, "timing read");
+  if (ms_partial) *ms_partial = a;
+  if (ms_merge) *ms_merge = b;
+  if (ms_plan) *ms_plan = c;
+  if (calls) *calls = n;
+  return ok();
+}
+
+int mkv_launch_count(mkv_pool_t p, int64_t* launches) {
+  if (!valid_pool(p) || !launches) return fail(MKV_ERR_INVALID_ARG, "NULL argument");
+  *launches = p->launches;
+  return ok();
+}
+
+}  // extern "C"
