@@ -100,7 +100,7 @@ typedef struct {
 
 /* Device bytes the caller must provide for a pool with this configuration:
  * FP8 slab, TQ3 slab, block table (int32 [max_seqs][max_pages_per_seq]) and the device
- * status word.  Any output pointer may be NULL.  Pure host computation. */
+ * status word (256 bytes).  Any output pointer may be NULL.  Pure host computation. */
 MKV_API int mkv_pool_required_bytes(const mkv_pool_config* cfg, size_t* fp8_slab_bytes,
                                     size_t* tq3_slab_bytes, size_t* table_bytes,
                                     size_t* status_bytes);
@@ -153,14 +153,17 @@ MKV_API int mkv_decode_workspace_bytes(mkv_pool_t pool, const int32_t* seq_ids,
  * parciais são combinados"): for sequence seq_ids[i] of length L, query j < q_len (the new
  * tokens are the last q_len positions), query head hq (KV head hq / (num_q_heads/Hkv)):
  *     out[i][j][hq][:] = sum_t softmax_t(sm_scale * q . K_t) V_t   over t <= L - q_len + j
- * with K, V the dequantised cache.  Each format has its own partial-attention kernel
- * producing (running max, denominator, unnormalised accumulator) per query head and split;
- * a merge kernel combines the partials with global normalisation.  No dense copy of the
- * cache is made; the workspace holds only page lists and partial states.
+ * with K, V the dequantised cache.  Two kernel launches (more only for very large calls):
+ * every sequence is cut into units of one page format and a logical page range; each format
+ * has its own partial-attention code producing (running max, denominator, unnormalised
+ * accumulator) per query column of a unit; the merge kernel combines all partial states of a
+ * (sequence, KV head, column) with global normalisation.  No dense copy of the cache is made;
+ * the workspace holds only partial states.
  *   q_bf16    device bf16 [n_seqs][q_len][num_q_heads][D]
  *   out       device fp32 [n_seqs][q_len][num_q_heads][D]
  *   workspace device scratch of ws_bytes >= mkv_decode_workspace_bytes(...), 256-B aligned
- * Constraints: num_q_heads % Hkv == 0, q_len * (num_q_heads / Hkv) <= 32.
+ * Constraints: num_q_heads % Hkv == 0, q_len * (num_q_heads / Hkv) <= 32,
+ * n_seqs <= max_seqs (rows may repeat).
  * Errors: BAD_SEQ, EMPTY_CONTEXT, INVALID_ARG, UNSUPPORTED, WORKSPACE_TOO_SMALL, CUDA. */
 MKV_API int mkv_decode_attention(mkv_pool_t pool, const int32_t* seq_ids, int32_t n_seqs,
                                  int32_t q_len, const void* q_bf16, int32_t num_q_heads,
@@ -198,12 +201,13 @@ MKV_API int mkv_pool_stats(mkv_pool_t pool, int64_t* live_tokens, int32_t* fp8_p
 MKV_API int mkv_get_device_status(mkv_pool_t pool, void* stream);
 
 /* Kernel timing for measurement: while enabled, every decode call records CUDA events on its
- * stream around each of its kernels.  mkv_timing_read synchronises on the recorded events and
- * returns the summed milliseconds of the partial-attention kernels, the merge kernels and the
- * plan kernels, and the number of decode calls timed; it then clears the record. */
+ * stream before its partial-attention kernel, between it and the merge kernel, and after the
+ * merge.  mkv_timing_read synchronises on the recorded events and returns the summed
+ * milliseconds of each kernel and the number of decode calls timed; it then clears the record.
+ * (Calls split into several launch groups record the span of all of them as partial time.) */
 MKV_API int mkv_timing_enable(mkv_pool_t pool, int32_t enable);
 MKV_API int mkv_timing_read(mkv_pool_t pool, double* ms_partial, double* ms_merge,
-                            double* ms_plan, int64_t* calls);
+                            int64_t* calls);
 
 /* Number of kernels this pool has launched since creation. */
 MKV_API int mkv_launch_count(mkv_pool_t pool, int64_t* launches);

@@ -59,7 +59,6 @@ SIGNATURES = {
     "mkv_timing_enable": (ctypes.c_int, [_P, _I32]),
     "mkv_timing_read": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_double),
                                        ctypes.POINTER(ctypes.c_double),
-                                       ctypes.POINTER(ctypes.c_double),
                                        ctypes.POINTER(ctypes.c_int64)]),
     "mkv_launch_count": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int64)]),
     "mkv_last_error": (ctypes.c_char_p, []),
@@ -208,9 +207,9 @@ class Pool:
         if out is None:
             out = torch.empty((n, q_len, Hq, D), dtype=torch.float32, device=q.device)
         op = _dev_ptr(out, torch.float32, "out")
-        need = self.workspace_bytes(s, q_len, Hq)
-        if workspace is None:
-            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        if workspace is None:   # the library checks a caller-given workspace's size itself
+            workspace = torch.empty(self.workspace_bytes(s, q_len, Hq), dtype=torch.uint8,
+                                    device=q.device)
         wp = _dev_ptr(workspace, torch.uint8, "workspace")
         scale = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
         _check(lib().mkv_decode_attention(self.handle, sp, s.size, q_len, qp, Hq,
@@ -265,11 +264,12 @@ class Pool:
         _check(lib().mkv_timing_enable(self.handle, 1 if enable else 0), "mkv_timing_enable")
 
     def timing_read(self):
-        v = [ctypes.c_double() for _ in range(3)]
+        """{'partial_ms', 'merge_ms': summed device time of each decode kernel, 'calls'}."""
+        v = [ctypes.c_double(), ctypes.c_double()]
         n = ctypes.c_int64()
-        _check(lib().mkv_timing_read(self.handle, *[ctypes.byref(x) for x in v], ctypes.byref(n)),
-               "mkv_timing_read")
-        return dict(partial_ms=v[0].value, merge_ms=v[1].value, plan_ms=v[2].value, calls=n.value)
+        _check(lib().mkv_timing_read(self.handle, ctypes.byref(v[0]), ctypes.byref(v[1]),
+                                     ctypes.byref(n)), "mkv_timing_read")
+        return dict(partial_ms=v[0].value, merge_ms=v[1].value, calls=n.value)
 
     def launch_count(self):
         n = ctypes.c_int64()

@@ -6,16 +6,16 @@
 // normalisation combines them -- no page is converted to a common format first and no dense
 // copy of the cache is made (section "... sem a chamada sombra densa").
 //
-// Three launches per call:
-//   plan_kernel     per sequence, compacts the block-table row into an FP8 page list and a TQ3
-//                   page list ({slot, logical page}), in logical order.
-//   partial_kernel  per (sequence, KV head, split of one format's list): streams the pages of
-//                   the split through a shared-memory ring with bulk async copies and computes
-//                   (m, l, acc) for the GQA group's query columns.  FP8 CTAs and TQ3 CTAs run
-//                   different code (fp8_page / tq3_page) and write separate partial states;
-//                   they share one grid so the small FP8 share does not run alone on a few SMs.
-//   merge_kernel    per (sequence, query column): M = max m, L = sum l 2^(m-M),
-//                   O = sum acc 2^(m-M) / L.
+// Two launches per call.  The host cuts every sequence into work units -- (format, logical page
+// range) -- and orders them largest first.  A CTA takes one (unit, KV head):
+//   1. its producer warp scans the block-table entries of the range and keeps the pages of the
+//      unit's format (FP8 units run fp8_page, TQ3 units tq3_page: separate per-format code and
+//      separate partial states);
+//   2. the producer streams those pages through a shared-memory ring with bulk async copies
+//      completing on mbarriers; consumer warps compute (m, l, acc) per query column;
+//   3. the CTA writes its partial state.
+// A second kernel merges, per (sequence, KV head, query column), all partial states of both
+// formats: M = max m, L = sum l 2^(m-M), O = sum acc 2^(m-M) / L.
 //
 // Tensor-core use: per page the logits are a 16-token x 8-column tile (tokens are the MMA M
 // dimension, the q_len*g query columns of one KV head the N dimension) and P.V is a
@@ -37,45 +37,51 @@ namespace mkv {
 namespace {
 
 constexpr float kLazyRescale = 8.f;  // log2 units
-constexpr int kMaxListPerCta = 256;
 
 template <int D, int NT>
 struct Cfg {
-  static constexpr int G = D / 32;
   static constexpr int PW = NT == 1 ? 4 : (NT == 2 ? 2 : 1);  // page-parallel warps
   static constexpr int NWC = NT * PW;                          // consumer warps
   static constexpr int THREADS = 32 * (NWC + 1);               // + 1 producer warp
   static constexpr int FP8_STAGE = 32 * D + 16;
   static constexpr int TQ3_STAGE = 14 * D;
-  static constexpr int FP8_NST = 8;
+  static constexpr int FP8_NST = 6;
   static constexpr int TQ3_NST = 16;
   static constexpr int RING_FP8 = FP8_NST * FP8_STAGE;
   static constexpr int RING_TQ3 = TQ3_NST * TQ3_STAGE;
   static constexpr int COMBINE = (PW - 1) * NT * 8 * (D + 2) * 4;
   static constexpr int RING = RING_FP8 > RING_TQ3 ? (RING_FP8 > COMBINE ? RING_FP8 : COMBINE)
                                                   : (RING_TQ3 > COMBINE ? RING_TQ3 : COMBINE);
-  // header: 2 x 16 mbarriers, 16 stage tags, abort flag, list buffer
-  static constexpr int HDR = 256 + 64 + 16 + kMaxListPerCta * 8;
-  static constexpr int SMEM = HDR + RING;
+  // Q fragments: per n-tile, D/32 x 32 lanes x 16 bytes
+  static constexpr int QF = NT * D * 16;
+  // header: 2 x 16 mbarriers | 16 stage tags | misc ints | page list | Q fragments | ring
+  static constexpr int OFF_TAG = 256, OFF_MISC = 320, OFF_LIST = 384;
+  static constexpr int OFF_QF = OFF_LIST + kMaxPagesPerUnit * 8;
+  static constexpr int OFF_RING = OFF_QF + QF;
+  static constexpr int SMEM = OFF_RING + RING;
 };
 
 struct Smem {
   uint64_t* full;
   uint64_t* empty;
   int32_t* tag;    // logical page of each stage (-1: invalid entry)
-  int32_t* abort;
-  int2* list;
+  int32_t* misc;   // [0] page count, [1] abort flag, [4..7] logit scales
+  int2* list;      // {slot, logical page} of the unit's pages
+  uint4* qf;       // Q fragments [NT][D/32][32 lanes]
   uint8_t* ring;
 };
 
+template <int D, int NT>
 __device__ __forceinline__ Smem carve(uint8_t* base) {
+  using C = Cfg<D, NT>;
   Smem s;
   s.full = reinterpret_cast<uint64_t*>(base);
   s.empty = s.full + 16;
-  s.tag = reinterpret_cast<int32_t*>(base + 256);
-  s.abort = reinterpret_cast<int32_t*>(base + 256 + 64);
-  s.list = reinterpret_cast<int2*>(base + 256 + 64 + 16);
-  s.ring = base + 256 + 64 + 16 + kMaxListPerCta * 8;
+  s.tag = reinterpret_cast<int32_t*>(base + C::OFF_TAG);
+  s.misc = reinterpret_cast<int32_t*>(base + C::OFF_MISC);
+  s.list = reinterpret_cast<int2*>(base + C::OFF_LIST);
+  s.qf = reinterpret_cast<uint4*>(base + C::OFF_QF);
+  s.ring = base + C::OFF_RING;
   return s;
 }
 
@@ -146,7 +152,7 @@ __device__ __forceinline__ void mask_page(float (&x)[4], int tok0, int r, int li
 // 8c+0, 8c+4 (k-block 0), 8c+1, 8c+5 (k-block 0, upper k), 8c+2, 8c+6 / 8c+3, 8c+7 (k-block 1).
 template <int D>
 __device__ __forceinline__ void tq3_page(WarpState<D>& st, const uint8_t* pg,
-                                         const uint32_t (&qb)[D / 32][4], int lane,
+                                         const uint4* qf, int lane,
                                          float ls, int tok0, bool masked, int lim0, int lim1,
                                          int kw, int ks5, int vw, int vs1) {
   constexpr int G = D / 32;
@@ -171,9 +177,10 @@ __device__ __forceinline__ void tq3_page(WarpState<D>& st, const uint8_t* pg,
       a[j] = hsub2_u32(((xa >> (3 * j)) & kMask) | kMagic, kSub);
       b[j] = hsub2_u32(((xb >> (3 * j)) & kMask) | kMagic, kSub);
     }
+    const uint4 qb = qf[32 * g + lane];
     float cg[4] = {0.f, 0.f, 0.f, 0.f};
-    mma_f16_16816(cg, a[0], b[0], a[1], b[1], qb[g][0], qb[g][1], cg);
-    mma_f16_16816(cg, a[2], b[2], a[3], b[3], qb[g][2], qb[g][3], cg);
+    mma_f16_16816(cg, a[0], b[0], a[1], b[1], qb.x, qb.y, cg);
+    mma_f16_16816(cg, a[2], b[2], a[3], b[3], qb.z, qb.w, cg);
     const float sa = __half2float(kscale[16 * g + r]);
     const float sb = __half2float(kscale[16 * g + r + 8]);
     x[0] = fmaf(sa, cg[0], x[0]);
@@ -220,7 +227,7 @@ __device__ __forceinline__ void tq3_page(WarpState<D>& st, const uint8_t* pg,
 // 64j+16c+4i+{0,1}, k 2c+8,2c+9 <- 64j+16c+4i+{2,3}.
 template <int D>
 __device__ __forceinline__ void fp8_page(WarpState<D>& st, const uint8_t* pg,
-                                         const uint32_t (&qb)[D / 16][2], int lane, float ls,
+                                         const uint4* qf, int lane, float ls,
                                          int tok0, bool masked, int lim0, int lim1) {
   const int r = lane >> 2, c = lane & 3;
   const float sk = *reinterpret_cast<const float*>(pg + 32 * D);
@@ -232,11 +239,13 @@ __device__ __forceinline__ void fp8_page(WarpState<D>& st, const uint8_t* pg,
     const uint4 wb = *reinterpret_cast<const uint4*>(pg + (r + 8) * D + 64 * j + 16 * c);
     const uint32_t va[4] = {wa.x, wa.y, wa.z, wa.w};
     const uint32_t vb[4] = {wb.x, wb.y, wb.z, wb.w};
+    const uint4 q01 = qf[32 * (2 * j) + lane], q23 = qf[32 * (2 * j + 1) + lane];
+    const uint32_t qq[8] = {q01.x, q01.y, q01.z, q01.w, q23.x, q23.y, q23.z, q23.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       mma_f16_16816(cg, e4m3x2_to_f16x2(va[i]), e4m3x2_to_f16x2(vb[i]),
                     e4m3x2_to_f16x2(va[i] >> 16), e4m3x2_to_f16x2(vb[i] >> 16),
-                    qb[4 * j + i][0], qb[4 * j + i][1], cg);
+                    qq[2 * i], qq[2 * i + 1], cg);
     }
   }
   float x[4];
@@ -270,8 +279,7 @@ __device__ __forceinline__ void fp8_page(WarpState<D>& st, const uint8_t* pg,
   }
 }
 
-// Query column n of this CTA's KV head -> (query index, query head).  Returns a pointer to the
-// bf16 row or nullptr for padding columns.
+// Query column n of this CTA's KV head -> its bf16 row, or nullptr for padding columns.
 __device__ __forceinline__ const uint16_t* q_row(const DecodeParams& p, const SeqDesc& sd,
                                                  int h, int n) {
   if (n >= p.NC) return nullptr;
@@ -279,79 +287,143 @@ __device__ __forceinline__ const uint16_t* q_row(const DecodeParams& p, const Se
   return p.q + ((static_cast<int64_t>(sd.out_row) * p.q_len + qi) * p.Hq + hq) * p.D;
 }
 
-__device__ __forceinline__ uint32_t q_pair(float a, float b, float scale) {
-  return pack_f16x2(a * scale, b * scale);
-}
-
-// Power-of-two factor bringing the warp's largest |q| into [2^13, 2^14) so that the f16 images
-// of the bf16 queries keep their precision; returns the factor, *inv its inverse.
-__device__ __forceinline__ float q_prescale(float amax, float* inv) {
+// Build the f16 Q fragments of n-tile nt (columns 8nt..8nt+7) in this format's channel order
+// into shared memory, scaled by a power of two that brings the tile's largest |q| into
+// [2^13, 2^14) (f16 images of the bf16 queries keep their precision); returns the logit scale
+// with the power of two undone.
+template <int D, bool FP8>
+__device__ __forceinline__ float build_q(const DecodeParams& p, const SeqDesc& sd, int h, int nt,
+                                         int lane, uint4* qf) {
+  const int r = lane >> 2, c = lane & 3;
+  const uint16_t* qr = q_row(p, sd, h, 8 * nt + r);
+  float qv[D / 4];
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < D / 4; ++i) {
+    // FP8 order: channels 64j+16c+e (j = i/16, e = i%16); TQ3 order: 32g+8c+e (g = i/8)
+    const int ch = FP8 ? 64 * (i / 16) + 16 * c + (i % 16) : 32 * (i / 8) + 8 * c + (i % 8);
+    const float v = qr ? bf16_bits_to_float(qr[ch]) : 0.f;
+    qv[i] = v;
+    amax = fmaxf(amax, fabsf(v));
+  }
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   int e = 0;
   if (amax > 0.f && isfinite(amax)) {
     frexpf(amax, &e);  // amax in [2^(e-1), 2^e)
-    e = 14 - e;
-    e = max(-100, min(100, e));
+    e = max(-100, min(100, 14 - e));
   }
-  *inv = ldexpf(1.f, -e);
-  return ldexpf(1.f, e);
+  const float qs = ldexpf(1.f, e);
+#pragma unroll
+  for (int w = 0; w < D / 32; ++w) {
+    uint4 f;
+    if constexpr (FP8) {
+      // two k-blocks (4j+i, 4j+i+1) per uint4: channels +0,+1 | +2,+3 of each
+      const float* v = qv + 8 * w;
+      f.x = pack_f16x2(v[0] * qs, v[1] * qs);
+      f.y = pack_f16x2(v[2] * qs, v[3] * qs);
+      f.z = pack_f16x2(v[4] * qs, v[5] * qs);
+      f.w = pack_f16x2(v[6] * qs, v[7] * qs);
+    } else {
+      // k-block pairs (8c+0, 8c+4), (8c+1, 8c+5), (8c+2, 8c+6), (8c+3, 8c+7) of group w
+      const float* v = qv + 8 * w;
+      f.x = pack_f16x2(v[0] * qs, v[4] * qs);
+      f.y = pack_f16x2(v[1] * qs, v[5] * qs);
+      f.z = pack_f16x2(v[2] * qs, v[6] * qs);
+      f.w = pack_f16x2(v[3] * qs, v[7] * qs);
+    }
+    qf[32 * w + lane] = f;
+  }
+  return p.logit_scale * ldexpf(1.f, -e);
+}
+
+// Producer warp: collect the unit's pages of format fmt from table entries [first, last).
+__device__ __forceinline__ int scan_range(const DecodeParams& p, const int32_t* row, int first,
+                                          int last, int fmt, int lane, int2* list) {
+  const int nslots = fmt == 0 ? p.fp8_slots : p.tq3_slots;
+  const unsigned lt = (1u << lane) - 1u;
+  int count = 0;
+  bool bad = false;
+  for (int base = first; base < last; base += 256) {
+    int32_t e[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int idx = base + 32 * j + lane;
+      e[j] = idx < last ? row[idx] : -2;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int idx = base + 32 * j + lane;
+      const uint32_t f = static_cast<uint32_t>(e[j]) >> kFmtShift;
+      const int slot = static_cast<int>(static_cast<uint32_t>(e[j]) & kSlotMask);
+      const bool mapped = e[j] >= 0;
+      bad |= (idx < last) && (!mapped || f > 1 || slot >= (f == 0 ? p.fp8_slots : p.tq3_slots));
+      const bool take = mapped && static_cast<int>(f) == fmt && slot < nslots;
+      const unsigned b = __ballot_sync(0xffffffffu, take);
+      const int pos = count + __popc(b & lt);
+      if (take && pos < kMaxPagesPerUnit) list[pos] = make_int2(slot, idx);
+      count += __popc(b);
+    }
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) flag_status(p.status, kStatusCheck);
+  if (count > kMaxPagesPerUnit) {
+    if (lane == 0) flag_status(p.status, kStatusCheck);
+    count = kMaxPagesPerUnit;
+  }
+  return count;
 }
 
 template <int D, int NT, bool FP8>
-__device__ void run_partial(const DecodeParams& p, const SeqDesc& sd, int h, int list_off,
-                            int count, int part, Smem sm) {
+__device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDesc& u, int h,
+                         Smem sm) {
   using C = Cfg<D, NT>;
   constexpr int STAGE = FP8 ? C::FP8_STAGE : C::TQ3_STAGE;
   constexpr int NST = FP8 ? C::FP8_NST : C::TQ3_NST;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = lane >> 2, c = lane & 3;
+  const int nt = warp % NT, pw = warp / NT;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], NT);
     }
-    *sm.abort = 0;
+    sm.misc[1] = 0;
     mbar_fence_init();
   }
   if (warp == C::NWC) {
-    const int2* lst = p.lists + list_off;
-    for (int i = lane; i < count; i += 32) sm.list[i] = lst[i];
+    const int32_t* row = p.tables + static_cast<int64_t>(sd.row) * p.max_pages;
+    const int n = scan_range(p, row, u.first, u.last, FP8 ? 0 : 1, lane, sm.list);
+    if (lane == 0) sm.misc[0] = n;
+  } else if (pw == 0) {
+    const float ls = build_q<D, FP8>(p, sd, h, nt, lane, sm.qf + nt * (D / 32) * 32);
+    if (lane == 0) reinterpret_cast<float*>(sm.misc)[4 + nt] = ls;
   }
   __syncthreads();
+  const int count = sm.misc[0];
 
   WarpState<D> st;
-  const int nt = warp % NT, pw = warp / NT;
-
   if (warp == C::NWC) {
-    // ---------------- producer: one lane streams the split's pages into the ring
+    // ---------------- producer: one lane streams the unit's pages into the ring
     if (lane == 0) {
       const uint8_t* slab = FP8 ? p.fp8_slab : p.tq3_slab;
       const int64_t slot_bytes = FP8 ? p.fp8_slot_bytes : p.tq3_slot_bytes;
-      const int nslots = FP8 ? p.fp8_slots : p.tq3_slots;
       int issued = 0;
       for (int i = 0; i < count; ++i) {
         const int s = i % NST;
         if (i >= NST && !mbar_wait(&sm.empty[s], ((i / NST) - 1) & 1)) {
           flag_status(p.status, kStatusTimeout);
-          atomicExch(sm.abort, 1);
+          atomicExch(&sm.misc[1], 1);
           break;
         }
         const int2 e = sm.list[i];
-        const bool ok = static_cast<unsigned>(e.x) < static_cast<unsigned>(nslots) && e.y >= 0;
-        sm.tag[s] = ok ? e.y : -1;
-        if (ok) {
-          mbar_arrive_expect_tx(&sm.full[s], STAGE);
-          bulk_g2s(sm.ring + s * STAGE,
-                   slab + static_cast<int64_t>(e.x) * slot_bytes + static_cast<int64_t>(h) * STAGE,
-                   STAGE, &sm.full[s]);
-        } else {
-          flag_status(p.status, kStatusCheck);
-          mbar_arrive(&sm.full[s]);
-        }
+        sm.tag[s] = e.y;
+        mbar_arrive_expect_tx(&sm.full[s], STAGE);
+        bulk_g2s(sm.ring + s * STAGE,
+                 slab + static_cast<int64_t>(e.x) * slot_bytes + static_cast<int64_t>(h) * STAGE,
+                 STAGE, &sm.full[s]);
         issued = i + 1;
       }
-      if (*reinterpret_cast<volatile int32_t*>(sm.abort)) {
+      if (*reinterpret_cast<volatile int32_t*>(&sm.misc[1])) {
         // drain: wait (bounded) for the last fill of every stage so no copy is in flight
         for (int i = max(0, issued - NST); i < issued; ++i)
           mbar_wait(&sm.full[i % NST], (i / NST) & 1, 100000000ull);
@@ -363,52 +435,8 @@ __device__ void run_partial(const DecodeParams& p, const SeqDesc& sd, int h, int
     const int lim0 = n0 < p.NC ? sd.ctx - p.q_len + n0 / p.g : sd.ctx - 1;
     const int lim1 = n1 < p.NC ? sd.ctx - p.q_len + n1 / p.g : sd.ctx - 1;
     const int min_lim = sd.ctx - p.q_len;
-    // Q fragment of column 8nt + r, in this format's channel order
-    const uint16_t* qr = q_row(p, sd, h, 8 * nt + r);
-    constexpr int QW = FP8 ? D / 16 : D / 32;
-    constexpr int QB = FP8 ? 2 : 4;
-    uint32_t qb[QW][QB];
-    float qv[D / 4];  // this lane's D/4 query values in fragment order
-    float amax = 0.f;
-    if constexpr (FP8) {
-#pragma unroll
-      for (int j = 0; j < D / 64; ++j) {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float v = qr ? bf16_bits_to_float(qr[64 * j + 16 * c + e]) : 0.f;
-          qv[16 * j + e] = v;
-          amax = fmaxf(amax, fabsf(v));
-        }
-      }
-    } else {
-#pragma unroll
-      for (int g = 0; g < D / 32; ++g) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float v = qr ? bf16_bits_to_float(qr[32 * g + 8 * c + e]) : 0.f;
-          qv[8 * g + e] = v;
-          amax = fmaxf(amax, fabsf(v));
-        }
-      }
-    }
-    float inv;
-    const float qs = q_prescale(amax, &inv);
-    if constexpr (FP8) {
-#pragma unroll
-      for (int kb = 0; kb < D / 16; ++kb) {
-        const float* v = qv + 4 * kb;  // channels 64j+16c+4i+{0..3}, kb = 4j+i
-        qb[kb][0] = q_pair(v[0], v[1], qs);
-        qb[kb][1] = q_pair(v[2], v[3], qs);
-      }
-    } else {
-#pragma unroll
-      for (int g = 0; g < D / 32; ++g) {
-        const float* v = qv + 8 * g;   // channels 32g+8c+{0..7}
-#pragma unroll
-        for (int j = 0; j < 4; ++j) qb[g][j % QB] = q_pair(v[j], v[j + 4], qs);
-      }
-    }
-    const float ls = p.logit_scale * inv;
+    const float ls = reinterpret_cast<const float*>(sm.misc)[4 + nt];
+    const uint4* qf = sm.qf + nt * (D / 32) * 32;
     // TQ3 lane constants: K chunk c of a record starts at bit 24c; we read bits from 24c-5
     // (codes land at 5+3k); V field of row r starts at bit 12r; we read from 12r-1.
     const int kbit = 24 * c - 5, vbit = 12 * r - 1;
@@ -426,19 +454,16 @@ __device__ void run_partial(const DecodeParams& p, const SeqDesc& sd, int h, int
       const int s = i % NST;
       if (!mbar_wait(&sm.full[s], (i / NST) & 1)) {
         flag_status(p.status, kStatusTimeout);
-        atomicExch(sm.abort, 1);
+        atomicExch(&sm.misc[1], 1);
         break;
       }
-      const int logical = sm.tag[s];
-      if (logical >= 0) {
-        const int tok0 = 16 * logical;
-        const bool masked = tok0 + 15 > min_lim;
-        const uint8_t* pg = sm.ring + s * STAGE;
-        if constexpr (FP8)
-          fp8_page<D>(st, pg, qb, lane, ls, tok0, masked, lim0, lim1);
-        else
-          tq3_page<D>(st, pg, qb, lane, ls, tok0, masked, lim0, lim1, kw, ks5, vw, vs1);
-      }
+      const int tok0 = 16 * sm.tag[s];
+      const bool masked = tok0 + 15 > min_lim;
+      const uint8_t* pg = sm.ring + s * STAGE;
+      if constexpr (FP8)
+        fp8_page<D>(st, pg, qf, lane, ls, tok0, masked, lim0, lim1);
+      else
+        tq3_page<D>(st, pg, qf, lane, ls, tok0, masked, lim0, lim1, kw, ks5, vw, vs1);
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.empty[s]);
     }
@@ -494,6 +519,7 @@ __device__ void run_partial(const DecodeParams& p, const SeqDesc& sd, int h, int
       }
     }
     // write the partial state of columns 8nt + 2c + k
+    const int part = sd.part0 + u.part;
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const int n = 8 * nt + 2 * c + k;
@@ -514,135 +540,106 @@ __device__ void run_partial(const DecodeParams& p, const SeqDesc& sd, int h, int
   }
 }
 
-template <int D, int NT>
-__global__ void __launch_bounds__(Cfg<D, NT>::THREADS, 2)
-    partial_kernel(const __grid_constant__ DecodeParams p) {
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  const Smem sm = carve(smem_raw);
-  const int x = blockIdx.x, h = blockIdx.y;
-  // sequence of this CTA: last s with seq[s].cta0 <= x
-  int lo = 0, hi = p.n_seqs - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (p.seq[mid].cta0 <= x) lo = mid; else hi = mid - 1;
-  }
-  const SeqDesc& sd = p.seq[lo];
-  const int local = x - sd.cta0;
-  const int part = sd.part0 + local;
-  if (local < sd.split8) {
-    const int first = local * p.P8;
-    const int count = min(p.P8, sd.n8 - first);
-    run_partial<D, NT, true>(p, sd, h, sd.list8 + first, count, part, sm);
-  } else {
-    const int first = (local - sd.split8) * p.P3;
-    const int count = min(p.P3, sd.n3 - first);
-    run_partial<D, NT, false>(p, sd, h, sd.list3 + first, count, part, sm);
-  }
-}
-
-// ------------------------------------------------------------------ plan
-__global__ void __launch_bounds__(256) plan_kernel(const __grid_constant__ DecodeParams p) {
-  __shared__ int w8[8], w3[8];
-  const SeqDesc& sd = p.seq[blockIdx.x];
-  const int32_t* row = p.tables + static_cast<int64_t>(sd.row) * p.max_pages;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const unsigned lt = (1u << lane) - 1u;
-  int base8 = 0, base3 = 0;
-  for (int b = 0; b < sd.n_pages; b += 256) {
-    const int idx = b + threadIdx.x;
-    const bool valid = idx < sd.n_pages;
-    const int32_t e = valid ? row[idx] : -1;
-    const uint32_t fmt = static_cast<uint32_t>(e) >> kFmtShift;
-    const int slot = static_cast<int>(static_cast<uint32_t>(e) & kSlotMask);
-    const bool good = valid && e >= 0 && fmt <= 1 &&
-                      slot < (fmt == 0 ? p.fp8_slots : p.tq3_slots);
-    if (valid && !good) flag_status(p.status, kStatusCheck);
-    const bool is8 = good && fmt == 0, is3 = good && fmt == 1;
-    const unsigned b8 = __ballot_sync(0xffffffffu, is8), b3 = __ballot_sync(0xffffffffu, is3);
-    if (lane == 0) {
-      w8[warp] = __popc(b8);
-      w3[warp] = __popc(b3);
-    }
-    __syncthreads();
-    int off8 = 0, off3 = 0, tot8 = 0, tot3 = 0;
-    for (int w = 0; w < 8; ++w) {
-      if (w < warp) {
-        off8 += w8[w];
-        off3 += w3[w];
-      }
-      tot8 += w8[w];
-      tot3 += w3[w];
-    }
-    if (is8) {
-      const int rank = base8 + off8 + __popc(b8 & lt);
-      if (rank < sd.n8) p.lists[sd.list8 + rank] = make_int2(slot, idx);
-      else flag_status(p.status, kStatusCheck);
-    }
-    if (is3) {
-      const int rank = base3 + off3 + __popc(b3 & lt);
-      if (rank < sd.n3) p.lists[sd.list3 + rank] = make_int2(slot, idx);
-      else flag_status(p.status, kStatusCheck);
-    }
-    base8 += tot8;
-    base3 += tot3;
-    __syncthreads();
-  }
-  if (base8 != sd.n8 || base3 != sd.n3) {
-    if (threadIdx.x == 0) flag_status(p.status, kStatusCheck);
-    for (int i = base8 + threadIdx.x; i < sd.n8; i += 256) p.lists[sd.list8 + i] = make_int2(-1, -1);
-    for (int i = base3 + threadIdx.x; i < sd.n3; i += 256) p.lists[sd.list3 + i] = make_int2(-1, -1);
-  }
-}
-
-// ------------------------------------------------------------------ merge
-// grid (sequence, KV head * NC); one thread per channel.
-__global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ DecodeParams p) {
-  const SeqDesc& sd = p.seq[blockIdx.x];
-  const int h = blockIdx.y / p.NC, n = blockIdx.y % p.NC;
-  const int S = sd.split8 + sd.split3;
+// Merge of the partial states of one (sequence, KV head, query column): the globally
+// normalised combination M = max m, L = sum l 2^(m-M), O = sum acc 2^(m-M) / L.  The maximum and
+// the weights are computed once in shared memory; the accumulation over partials is then a
+// branch-free sum of independent float4 loads, split over thread groups and reduced at the end.
+constexpr int kMergeThreads = 256;
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_constant__ DecodeParams p) {
+  __shared__ float w[kDecodeMaxUnits];
+  __shared__ float red[kMergeThreads / 32];
+  __shared__ float4 part[kMergeThreads];
+  const int pair = blockIdx.x / p.NC, n = blockIdx.x % p.NC;
+  const SeqDesc& sd = p.seq[pair / p.Hkv];
+  const int h = pair % p.Hkv;
+  const int S = sd.n_parts, D = p.D, tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+  const int64_t base0 = (static_cast<int64_t>(sd.part0) * p.Hkv + h) * p.NC + n;
   const int64_t stride = static_cast<int64_t>(p.Hkv) * p.NC;
-  const int64_t first = (static_cast<int64_t>(sd.part0) * p.Hkv + h) * p.NC + n;
+  const float2* ml = reinterpret_cast<const float2*>(p.part_ml);
+  float mloc = -INFINITY;
+  for (int j = tid; j < S; j += kMergeThreads) mloc = fmaxf(mloc, ml[base0 + j * stride].x);
+  for (int o = 16; o > 0; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
+  if (lane == 0) red[wp] = mloc;
+  __syncthreads();
   float M = -INFINITY;
-  for (int j = 0; j < S; ++j) M = fmaxf(M, p.part_ml[2 * (first + j * stride)]);
-  const int qi = n / p.g, hq = h * p.g + n % p.g;
-  float* out = p.out + ((static_cast<int64_t>(sd.out_row) * p.q_len + qi) * p.Hq + hq) * p.D;
-  for (int d = threadIdx.x; d < p.D; d += blockDim.x) {
-    float L = 0.f, O = 0.f;
-    if (M != -INFINITY) {
-      for (int j = 0; j < S; ++j) {
-        const int64_t b = first + j * stride;
-        const float m = p.part_ml[2 * b];
-        if (m == -INFINITY) continue;
-        const float w = exp2f(m - M);
-        L = fmaf(w, p.part_ml[2 * b + 1], L);
-        O = fmaf(w, p.part_acc[b * p.D + d], O);
-      }
+  for (int i = 0; i < kMergeThreads / 32; ++i) M = fmaxf(M, red[i]);
+  __syncthreads();
+  float lloc = 0.f;
+  for (int j = tid; j < S; j += kMergeThreads) {
+    const float2 v = ml[base0 + j * stride];
+    const float wj = (v.x == -INFINITY || M == -INFINITY) ? 0.f : exp2f(v.x - M);
+    w[j] = wj;
+    lloc = fmaf(wj, v.y, lloc);
+  }
+  for (int o = 16; o > 0; o >>= 1) lloc += __shfl_xor_sync(0xffffffffu, lloc, o);
+  if (lane == 0) red[wp] = lloc;
+  __syncthreads();
+  float L = 0.f;
+  for (int i = 0; i < kMergeThreads / 32; ++i) L += red[i];
+  // accumulation: thread = (subset k of the partials, group c4 of 4 channels)
+  const int groups = D / 4, nsub = kMergeThreads / groups;
+  const int c4 = tid % groups, k = tid / groups;
+  float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+  const float4* acc = reinterpret_cast<const float4*>(p.part_acc);
+#pragma unroll 8
+  for (int j = k; j < S; j += nsub) {
+    const float4 a = acc[(base0 + j * stride) * groups + c4];
+    const float wj = w[j];
+    O.x = fmaf(wj, a.x, O.x);
+    O.y = fmaf(wj, a.y, O.y);
+    O.z = fmaf(wj, a.z, O.z);
+    O.w = fmaf(wj, a.w, O.w);
+  }
+  part[tid] = O;
+  __syncthreads();
+  if (tid < groups) {
+    float4 t = part[tid];
+    for (int i = 1; i < nsub; ++i) {
+      const float4 u = part[tid + i * groups];
+      t.x += u.x; t.y += u.y; t.z += u.z; t.w += u.w;
     }
-    out[d] = L > 0.f ? O / L : 0.f;
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    const int qi = n / p.g, hq = h * p.g + n % p.g;
+    float* out = p.out + ((static_cast<int64_t>(sd.out_row) * p.q_len + qi) * p.Hq + hq) * D;
+    reinterpret_cast<float4*>(out)[tid] = make_float4(t.x * inv, t.y * inv, t.z * inv, t.w * inv);
   }
 }
 
 template <int D, int NT>
-cudaError_t launch_partial_t(const DecodeParams& p, cudaStream_t s) {
+__global__ void __launch_bounds__(Cfg<D, NT>::THREADS, 3)
+    decode_kernel(const __grid_constant__ DecodeParams p) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  const Smem sm = carve<D, NT>(smem_raw);
+  const int h = blockIdx.x % p.Hkv;
+  const UnitDesc& u = p.unit[blockIdx.x / p.Hkv];
+  const SeqDesc& sd = p.seq[u.seq];
+  if (u.fmt == 0)
+    run_unit<D, NT, true>(p, sd, u, h, sm);
+  else
+    run_unit<D, NT, false>(p, sd, u, h, sm);
+}
+
+template <int D, int NT>
+cudaError_t launch_t(const DecodeParams& p, cudaStream_t s) {
   using C = Cfg<D, NT>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(partial_kernel<D, NT>,
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, NT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  partial_kernel<D, NT><<<dim3(p.total_ctas, p.Hkv), C::THREADS, C::SMEM, s>>>(p);
+  decode_kernel<D, NT><<<p.n_units * p.Hkv, C::THREADS, C::SMEM, s>>>(p);
   return cudaGetLastError();
 }
 
 template <int D>
-cudaError_t launch_partial_d(const DecodeParams& p, cudaStream_t s) {
+cudaError_t launch_d(const DecodeParams& p, cudaStream_t s) {
   switch ((p.NC + 7) / 8) {
-    case 1: return launch_partial_t<D, 1>(p, s);
-    case 2: return launch_partial_t<D, 2>(p, s);
-    case 3: return launch_partial_t<D, 3>(p, s);
-    case 4: return launch_partial_t<D, 4>(p, s);
+    case 1: return launch_t<D, 1>(p, s);
+    case 2: return launch_t<D, 2>(p, s);
+    case 3: return launch_t<D, 3>(p, s);
+    case 4: return launch_t<D, 4>(p, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -653,24 +650,20 @@ bool partial_supported(int D, int NC) {
   return (D == 64 || D == 128 || D == 256) && NC >= 1 && NC <= 32;
 }
 
-cudaError_t launch_plan(const DecodeParams& p, cudaStream_t s) {
-  plan_kernel<<<p.n_seqs, 256, 0, s>>>(p);
+cudaError_t launch_merge(const DecodeParams& p, cudaStream_t s) {
+  if (p.n_seqs <= 0) return cudaSuccess;
+  merge_kernel<<<p.n_seqs * p.Hkv * p.NC, kMergeThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_partial(const DecodeParams& p, cudaStream_t s) {
-  if (p.total_ctas <= 0) return cudaSuccess;
+  if (p.n_units <= 0) return cudaSuccess;
   switch (p.D) {
-    case 64: return launch_partial_d<64>(p, s);
-    case 128: return launch_partial_d<128>(p, s);
-    case 256: return launch_partial_d<256>(p, s);
+    case 64: return launch_d<64>(p, s);
+    case 128: return launch_d<128>(p, s);
+    case 256: return launch_d<256>(p, s);
     default: return cudaErrorInvalidValue;
   }
-}
-
-cudaError_t launch_merge(const DecodeParams& p, cudaStream_t s) {
-  merge_kernel<<<dim3(p.n_seqs, p.Hkv * p.NC), p.D < 256 ? p.D : 256, 0, s>>>(p);
-  return cudaGetLastError();
 }
 
 }  // namespace mkv

@@ -75,42 +75,51 @@ struct CopyParams {
 };
 
 // ------------------------------------------------------------------ decode
+// Decode = partial kernel + merge kernel.  Work unit = (sequence, format, logical page range);
+// a partial CTA takes one (unit, KV head): it scans the block-table entries of its range,
+// streams the pages of its format through a shared-memory ring and writes one partial state
+// per query column.  The merge kernel combines every partial state of a (sequence, KV head,
+// column).
 struct SeqDesc {
-  int32_t row;             // table row (sequence id)
-  int32_t ctx;             // context length L (includes the q_len new tokens)
-  int32_t n_pages;         // mapped pages
-  int32_t n8, n3;          // FP8 / TQ3 pages (host counts; the plan kernel checks them)
-  int32_t list8, list3;    // offsets of the sequence's FP8 / TQ3 page lists (int2 entries)
-  int32_t split8, split3;  // partial-attention CTAs per KV head for each format
-  int32_t cta0;            // first CTA (grid x) of this sequence
-  int32_t part0;           // first partial-state index of this sequence
-  int32_t out_row;         // position of the sequence in the call (rows of q and out)
+  int32_t row;      // table row (sequence id)
+  int32_t ctx;      // context length L (includes the q_len new tokens)
+  int32_t out_row;  // position of the sequence in the call (rows of q and out)
+  int32_t part0;    // first partial-state index of this sequence
+  int32_t n_parts;  // units of this sequence (partial states per KV head)
+  int32_t pad;
 };
-constexpr int kDecodeMaxSeqs = 480;
+struct UnitDesc {
+  int32_t first;  // logical pages [first, last)
+  int32_t last;
+  int16_t seq;    // index into DecodeParams::seq
+  int16_t fmt;    // 0 FP8, 1 TQ3
+  int32_t part;   // index of this unit's partial state within its sequence
+};
+constexpr int kDecodeMaxSeqs = 256;
+constexpr int kDecodeMaxUnits = 1536;
+constexpr int kMaxPagesPerUnit = 256;  // pages of the unit's format inside its range
 struct DecodeParams {
   const uint8_t* fp8_slab;
   const uint8_t* tq3_slab;
   const int32_t* tables;
-  int32_t* status;
+  int32_t* status;    // status word
   const uint16_t* q;  // bf16 bits [n][q_len][Hq][D]
   float* out;         // fp32 [n][q_len][Hq][D]
-  int2* lists;        // page lists: {slot, logical page}
   float* part_ml;     // [part][Hkv][NC][2]: running max (log2 units), denominator
   float* part_acc;    // [part][Hkv][NC][D]: unnormalised accumulator
   int64_t fp8_slot_bytes, tq3_slot_bytes;
   int32_t Hkv, D, g, q_len, NC, Hq;
   int32_t max_pages, fp8_slots, tq3_slots;
-  int32_t P8, P3;      // pages per CTA for each format
-  float logit_scale;   // sm_scale * log2(e)
-  int32_t n_seqs;      // sequences in this launch
-  int32_t total_ctas;  // partial CTAs per KV head in this launch
+  float logit_scale;  // sm_scale * log2(e)
+  int32_t n_seqs;     // sequences in this launch
+  int32_t n_units;    // units in this launch (grid = n_units * Hkv CTAs)
   SeqDesc seq[kDecodeMaxSeqs];
+  UnitDesc unit[kDecodeMaxUnits];
 };
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 cudaError_t launch_demote(const DemoteParams& p, cudaStream_t s);
 cudaError_t launch_copy(const CopyParams& p, cudaStream_t s);
-cudaError_t launch_plan(const DecodeParams& p, cudaStream_t s);
 cudaError_t launch_partial(const DecodeParams& p, cudaStream_t s);
 cudaError_t launch_merge(const DecodeParams& p, cudaStream_t s);
 bool partial_supported(int D, int NC);

@@ -99,7 +99,7 @@ inline int fmt_of(int32_t e) { return static_cast<int>(static_cast<uint32_t>(e) 
 inline int32_t slot_of(int32_t e) { return static_cast<int32_t>(static_cast<uint32_t>(e) & kSlotMask); }
 
 struct TimingRec {
-  cudaEvent_t ev[4];
+  cudaEvent_t ev[3];  // before the partial kernel, between partial and merge, after the merge
 };
 
 }  // namespace
@@ -151,75 +151,85 @@ int validate_config(const mkv_pool_config* c) {
 
 cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
-// Pages of work per partial-attention CTA: enough CTAs for about four waves of two CTAs per
-// SM, an FP8 page counting as two TQ3 pages of bytes.
-void choose_split(const mkv_pool_t p, int64_t pages8, int64_t pages3, int32_t* P8, int32_t* P3) {
-  const int64_t work = (2 * pages8 + pages3) * p->cfg.num_kv_heads;
-  const int64_t target_ctas = static_cast<int64_t>(p->sm_count) * 2 * 4;
-  int64_t per = (work + target_ctas - 1) / target_ctas;
-  per = std::max<int64_t>(4, std::min<int64_t>(256, per));
-  *P3 = static_cast<int32_t>(per);
-  *P8 = static_cast<int32_t>(std::max<int64_t>(2, per / 2));
-}
+// Device status buffer: the status word (padded to 256 bytes).
+size_t status_bytes(const mkv_pool_config&) { return 256; }
 
 struct DecodePlan {
-  int32_t NC = 0, g = 0, P8 = 0, P3 = 0;
-  std::vector<SeqDesc> seq;
-  int64_t list_entries = 0, parts = 0;
-  size_t off_lists = 0, off_ml = 0, off_acc = 0, bytes = 0;
+  int32_t NC = 0, g = 0;
+  std::vector<SeqDesc> seq;    // per call position
+  std::vector<UnitDesc> unit;  // per sequence, in order; UnitDesc::seq = call position
+  std::vector<int64_t> cost;   // bytes per KV head of each unit
+  int64_t parts = 0;
+  size_t off_ml = 0, off_acc = 0, bytes = 0;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Cut every sequence into work units: TQ3 units are logical ranges of R3 pages (FP8 pages inside
+// are left to FP8 units); FP8 units are runs of up to P8 consecutive FP8 pages.  R3 and P8 aim at
+// about three waves of three CTAs per SM, each CTA reading a similar number of bytes.
 int plan_decode(mkv_pool_t p, const int32_t* seq_ids, int32_t n, int32_t q_len, int32_t Hq,
                 DecodePlan* plan) {
   if (n < 0 || (n > 0 && !seq_ids)) return fail(MKV_ERR_INVALID_ARG, "bad sequence list");
+  if (n > p->cfg.max_seqs)
+    return fail(MKV_ERR_INVALID_ARG, "at most max_seqs (%d) sequences per decode call", p->cfg.max_seqs);
   if (q_len < 1) return fail(MKV_ERR_INVALID_ARG, "q_len must be >= 1");
-  const int Hkv = p->cfg.num_kv_heads;
+  const int Hkv = p->cfg.num_kv_heads, D = p->cfg.head_dim;
   if (Hq < Hkv || Hq % Hkv) return fail(MKV_ERR_INVALID_ARG, "num_q_heads %d not a multiple of Hkv %d", Hq, Hkv);
   plan->g = Hq / Hkv;
   plan->NC = q_len * plan->g;
-  if (!partial_supported(p->cfg.head_dim, plan->NC))
+  if (!partial_supported(D, plan->NC))
     return fail(MKV_ERR_UNSUPPORTED, "q_len * num_q_heads / Hkv = %d > 32 is not built", plan->NC);
-  int64_t n8 = 0, n3 = 0;
+  const int64_t b8 = fp8_head_bytes(D), b3 = tq3_head_bytes(D);
+  int64_t total = 0;
   for (int32_t i = 0; i < n; ++i) {
     if (int e = check_seq(p, seq_ids[i])) return e;
     const Seq& s = p->seqs[seq_ids[i]];
     if (s.ctx < q_len || s.ctx == 0)
       return fail(MKV_ERR_EMPTY_CONTEXT, "sequence %d has %d tokens < q_len %d", seq_ids[i], s.ctx, q_len);
-    n8 += static_cast<int64_t>(s.fp8_pages.size());
-    n3 += s.n3;
+    total += static_cast<int64_t>(s.fp8_pages.size()) * b8 + static_cast<int64_t>(s.n3) * b3;
   }
-  choose_split(p, n8, n3, &plan->P8, &plan->P3);
+  const int64_t target_ctas = static_cast<int64_t>(p->sm_count) * 3 * 3;
+  const int64_t per_cta = std::max<int64_t>(1, total * Hkv / target_ctas);
+  const int32_t R3 = static_cast<int32_t>(std::max<int64_t>(8, std::min<int64_t>(kMaxPagesPerUnit, per_cta / b3)));
+  const int32_t P8 = static_cast<int32_t>(std::max<int64_t>(4, std::min<int64_t>(kMaxPagesPerUnit, per_cta / b8)));
   plan->seq.resize(n);
-  int64_t lists = 0, parts = 0;
+  plan->unit.clear();
+  plan->cost.clear();
+  int64_t parts = 0;
   for (int32_t i = 0; i < n; ++i) {
     const Seq& s = p->seqs[seq_ids[i]];
     SeqDesc& d = plan->seq[i];
     d.row = seq_ids[i];
     d.ctx = s.ctx;
-    d.n_pages = static_cast<int32_t>(s.table.size());
-    d.n8 = static_cast<int32_t>(s.fp8_pages.size());
-    d.n3 = s.n3;
-    d.list8 = static_cast<int32_t>(lists);
-    d.list3 = static_cast<int32_t>(lists + d.n8);
-    lists += d.n8 + d.n3;
-    d.split8 = (d.n8 + plan->P8 - 1) / plan->P8;
-    d.split3 = (d.n3 + plan->P3 - 1) / plan->P3;
-    d.part0 = static_cast<int32_t>(parts);
-    parts += d.split8 + d.split3;
     d.out_row = i;
-    d.cta0 = 0;  // per launch
+    d.part0 = static_cast<int32_t>(parts);
+    d.pad = 0;
+    int32_t np = 0;
+    const auto& f8 = s.fp8_pages;
+    for (size_t j = 0; j < f8.size(); j += P8) {
+      const size_t k = std::min(f8.size(), j + static_cast<size_t>(P8));
+      plan->unit.push_back({f8[j], f8[k - 1] + 1, static_cast<int16_t>(i), 0, np++});
+      plan->cost.push_back(static_cast<int64_t>(k - j) * b8);
+    }
+    const int32_t pages = static_cast<int32_t>(s.table.size());
+    for (int32_t a = 0; a < pages; a += R3) {
+      const int32_t b = std::min(pages, a + R3);
+      const int64_t in8 = std::lower_bound(f8.begin(), f8.end(), b) - std::lower_bound(f8.begin(), f8.end(), a);
+      const int64_t in3 = (b - a) - in8;
+      if (in3 <= 0) continue;
+      plan->unit.push_back({a, b, static_cast<int16_t>(i), 1, np++});
+      plan->cost.push_back(in3 * b3);
+    }
+    d.n_parts = np;
+    parts += np;
   }
-  if (lists > INT32_MAX || parts > INT32_MAX) return fail(MKV_ERR_INVALID_ARG, "call too large");
-  plan->list_entries = lists;
+  if (parts > INT32_MAX / 2) return fail(MKV_ERR_INVALID_ARG, "call too large");
   plan->parts = parts;
-  const int64_t cols = static_cast<int64_t>(parts) * Hkv * plan->NC;
-  plan->off_lists = 0;
-  plan->off_ml = align256(static_cast<size_t>(lists) * 8);
-  plan->off_acc = plan->off_ml + align256(static_cast<size_t>(cols) * 2 * 4);
-  plan->bytes = plan->off_acc + align256(static_cast<size_t>(cols) * p->cfg.head_dim * 4);
-  if (plan->bytes == 0) plan->bytes = 256;
+  const size_t cols = static_cast<size_t>(parts) * Hkv * plan->NC;
+  plan->off_ml = 0;
+  plan->off_acc = align256(cols * 2 * 4);
+  plan->bytes = std::max<size_t>(256, plan->off_acc + align256(cols * D * 4));
   return MKV_OK;
 }
 
@@ -248,7 +258,7 @@ int mkv_pool_required_bytes(const mkv_pool_config* cfg, size_t* fp8_slab, size_t
   if (fp8_slab) *fp8_slab = static_cast<size_t>(cfg->fp8_slots) * Hkv * fp8_head_bytes(D);
   if (tq3_slab) *tq3_slab = static_cast<size_t>(cfg->tq3_slots) * Hkv * tq3_head_bytes(D);
   if (tables) *tables = static_cast<size_t>(cfg->max_seqs) * cfg->max_pages_per_seq * 4;
-  if (status) *status = 16;
+  if (status) *status = status_bytes(*cfg);
   return ok();
 }
 
@@ -285,7 +295,7 @@ int mkv_pool_create(const mkv_pool_config* cfg, void* fp8_slab, void* tq3_slab,
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&p->sm_count, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess)
       e = cudaMemsetAsync(d_tables, 0xFF, static_cast<size_t>(cfg->max_seqs) * cfg->max_pages_per_seq * 4, 0);
-    if (e == cudaSuccess) e = cudaMemsetAsync(d_status, 0, 16, 0);
+    if (e == cudaSuccess) e = cudaMemsetAsync(d_status, 0, status_bytes(*cfg), 0);
     if (e == cudaSuccess) e = cudaStreamSynchronize(0);
     if (e != cudaSuccess) {
       delete p;
@@ -514,7 +524,6 @@ int mkv_decode_attention(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, i
   prm->status = p->d_status;
   prm->q = static_cast<const uint16_t*>(q_bf16);
   prm->out = out;
-  prm->lists = reinterpret_cast<int2*>(ws + plan.off_lists);
   prm->part_ml = reinterpret_cast<float*>(ws + plan.off_ml);
   prm->part_acc = reinterpret_cast<float*>(ws + plan.off_acc);
   prm->fp8_slot_bytes = p->fp8_slot_bytes;
@@ -528,40 +537,55 @@ int mkv_decode_attention(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, i
   prm->max_pages = p->cfg.max_pages_per_seq;
   prm->fp8_slots = p->cfg.fp8_slots;
   prm->tq3_slots = p->cfg.tq3_slots;
-  prm->P8 = plan.P8;
-  prm->P3 = plan.P3;
   prm->logit_scale = sm_scale * 1.4426950408889634f;
   TimingRec rec{};
   bool timed = p->timing;
-  if (timed) {
-    for (auto& e : rec.ev) {
-      e = get_event(p);
-      if (!e) timed = false;
+  if (timed)
+    for (auto& e : rec.ev)
+      if (!(e = get_event(p))) timed = false;
+  cudaError_t err = timed ? cudaEventRecord(rec.ev[0], st) : cudaSuccess;
+  // launches over groups of whole sequences, each within the parameter-block limits
+  size_t u0 = 0;
+  int32_t s0 = 0;
+  std::vector<size_t> order;
+  while (s0 < n_seqs && err == cudaSuccess) {
+    int32_t s1 = s0;
+    size_t u1 = u0;
+    while (s1 < n_seqs && s1 - s0 < kDecodeMaxSeqs) {
+      size_t ue = u1;
+      while (ue < plan.unit.size() && plan.unit[ue].seq == s1) ++ue;
+      if (ue - u0 > static_cast<size_t>(kDecodeMaxUnits) && s1 > s0) break;
+      if (ue - u0 > static_cast<size_t>(kDecodeMaxUnits)) {
+        err = cudaErrorInvalidValue;
+        break;
+      }
+      u1 = ue;
+      ++s1;
     }
-  }
-  cudaError_t err = cudaSuccess;
-  for (int32_t b = 0; b < n_seqs && err == cudaSuccess; b += kDecodeMaxSeqs) {
-    const int32_t m = std::min<int32_t>(kDecodeMaxSeqs, n_seqs - b);
-    int32_t ctas = 0;
-    for (int32_t i = 0; i < m; ++i) {
-      prm->seq[i] = plan.seq[b + i];
-      prm->seq[i].cta0 = ctas;
-      ctas += prm->seq[i].split8 + prm->seq[i].split3;
+    if (err != cudaSuccess) break;
+    for (int32_t i = s0; i < s1; ++i) prm->seq[i - s0] = plan.seq[i];
+    order.resize(u1 - u0);
+    for (size_t k = 0; k < order.size(); ++k) order[k] = u0 + k;
+    std::stable_sort(order.begin(), order.end(),
+                     [&](size_t x, size_t y) { return plan.cost[x] > plan.cost[y]; });
+    for (size_t k = 0; k < order.size(); ++k) {
+      prm->unit[k] = plan.unit[order[k]];
+      prm->unit[k].seq = static_cast<int16_t>(plan.unit[order[k]].seq - s0);
     }
-    prm->n_seqs = m;
-    prm->total_ctas = ctas;
-    const bool first = b == 0, last = b + m >= n_seqs;
-    if (timed && first) err = cudaEventRecord(rec.ev[0], st);
-    if (err == cudaSuccess) err = launch_plan(*prm, st), ++p->launches;
-    if (timed && first && err == cudaSuccess) err = cudaEventRecord(rec.ev[1], st);
-    if (err == cudaSuccess) err = launch_partial(*prm, st), ++p->launches;
-    if (timed && last && err == cudaSuccess) err = cudaEventRecord(rec.ev[2], st);
+    prm->n_seqs = s1 - s0;
+    prm->n_units = static_cast<int32_t>(order.size());
+    const bool last = s1 >= n_seqs;
+    err = launch_partial(*prm, st);
+    ++p->launches;
+    if (timed && last && err == cudaSuccess) err = cudaEventRecord(rec.ev[1], st);
     if (err == cudaSuccess) err = launch_merge(*prm, st), ++p->launches;
-    if (timed && last && err == cudaSuccess) err = cudaEventRecord(rec.ev[3], st);
+    s0 = s1;
+    u0 = u1;
   }
+  if (timed && err == cudaSuccess) err = cudaEventRecord(rec.ev[2], st);
   delete prm;
   if (timed) {
-    if (err == cudaSuccess && n_seqs <= kDecodeMaxSeqs) p->timing_recs.push_back(rec);
+    if (err == cudaSuccess) p->timing_recs.push_back(rec);
     else for (auto e : rec.ev) p->spare_events.push_back(e);
   }
   if (err != cudaSuccess) return cuda_fail(err, "decode launch");
@@ -703,20 +727,17 @@ int mkv_timing_enable(mkv_pool_t p, int32_t enable) {
   return ok();
 }
 
-int mkv_timing_read(mkv_pool_t p, double* ms_partial, double* ms_merge, double* ms_plan,
-                    int64_t* calls) {
+int mkv_timing_read(mkv_pool_t p, double* ms_partial, double* ms_merge, int64_t* calls) {
   if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
-  double a = 0, b = 0, c = 0;
+  double a = 0, b = 0;
   cudaError_t err = cudaSuccess;
   for (auto& r : p->timing_recs) {
-    float t0 = 0, t1 = 0, t2 = 0;
-    if (err == cudaSuccess) err = cudaEventSynchronize(r.ev[3]);
+    float t0 = 0, t1 = 0;
+    if (err == cudaSuccess) err = cudaEventSynchronize(r.ev[2]);
     if (err == cudaSuccess) err = cudaEventElapsedTime(&t0, r.ev[0], r.ev[1]);
     if (err == cudaSuccess) err = cudaEventElapsedTime(&t1, r.ev[1], r.ev[2]);
-    if (err == cudaSuccess) err = cudaEventElapsedTime(&t2, r.ev[2], r.ev[3]);
-    c += t0;
-    a += t1;
-    b += t2;
+    a += t0;
+    b += t1;
   }
   const int64_t n = static_cast<int64_t>(p->timing_recs.size());
   for (auto& r : p->timing_recs)
@@ -725,7 +746,6 @@ int mkv_timing_read(mkv_pool_t p, double* ms_partial, double* ms_merge, double* 
   if (err != cudaSuccess) return cuda_fail(err, "timing read");
   if (ms_partial) *ms_partial = a;
   if (ms_merge) *ms_merge = b;
-  if (ms_plan) *ms_plan = c;
   if (calls) *calls = n;
   return ok();
 }

@@ -8,7 +8,7 @@ library's tests/bench and the CPU oracle, so both see bit-identical inputs.
 Recipe (all values bf16 from fp32 N(0,1) draws rounded to nearest even):
   RNG      numpy PCG64, seed = 1000*cfg + stream, with a spawn key per (layer, sequence);
            streams: 0 Q, 1 K, 2 V, 3 slot order, 4 outlier channels, 5 protected pages,
-           6 context lengths.
+           6 context lengths, 7 per-step decode inputs.
   K        N(0,1); with ``outliers`` 4 distinct channels per (layer, KV head) are scaled x8
            before rounding (the same channels for every token and sequence).
   V, Q     N(0,1).
@@ -34,7 +34,7 @@ from dataclasses import dataclass
 import numpy as np
 
 PAGE = 16
-S_Q, S_K, S_V, S_SLOT, S_OUTLIER, S_PROTECT, S_CTX = range(7)
+S_Q, S_K, S_V, S_SLOT, S_OUTLIER, S_PROTECT, S_CTX, S_STEP = range(8)
 
 
 def bf16_bits(x) -> np.ndarray:
@@ -119,6 +119,20 @@ class Workload:
         """bf16 bits of the queries of a sequence: uint16 [q_len, Hq, D]."""
         r = self.rng(S_Q, layer, seq)
         return bf16_bits(r.standard_normal((self.q_len, self.Hq, self.D), dtype=np.float32))
+
+    def step_inputs(self, step: int, layer: int = 0):
+        """Inputs of one decode step of one layer: the new token's K and V for every sequence
+        (uint16 bf16 bits [B, Hkv, D] each, outlier channels as in ``kv``) and the queries
+        (uint16 [B, q_len, Hq, D])."""
+        r = self.rng(S_STEP, layer, step)
+        k = r.standard_normal((self.B, self.Hkv, self.D), dtype=np.float32)
+        v = r.standard_normal((self.B, self.Hkv, self.D), dtype=np.float32)
+        q = r.standard_normal((self.B, self.q_len, self.Hq, self.D), dtype=np.float32)
+        if self.outliers:
+            oc = self.outlier_channels(layer)
+            for h in range(self.Hkv):
+                k[:, h, oc[h]] *= np.float32(8.0)
+        return bf16_bits(k), bf16_bits(v), bf16_bits(q)
 
     def protected(self, seq: int) -> list:
         """Logical pages the caller marks protected (sorted).  Candidates are the full pages

@@ -103,8 +103,9 @@ def test_steady_state_append_demote_decode():
 
 def test_repeated_sequence_rows_and_order():
     w = WORKLOADS[2].scaled(B=3, ctx=(500, 900, 130))
-    lp = lib_pool(w)
-    op = oracle_pool(w)
+    shape = dict(w.pool_shape(), max_seqs=6)     # a call may list at most max_seqs rows
+    lp = lib_pool(w, shape=shape)
+    op = oracle_pool(w, shape=shape)
     order = [2, 0, 2, 1]
     q = to_bf16_tensor(np.stack([w.q(s) for s in order]))
     out = lp.decode(order, q).cpu().numpy()
