@@ -170,6 +170,28 @@ MKV_API int mkv_decode_attention(mkv_pool_t pool, const int32_t* seq_ids, int32_
                                  float sm_scale, float* out, void* workspace, size_t ws_bytes,
                                  void* stream);
 
+/* Decode attention like mkv_decode_attention, for callers that cannot allocate device memory
+ * (e.g. code running under stream capture where allocation is not allowed, or a host runtime
+ * that owns the whole device-memory budget and hands out no scratch).  The partial states go
+ * to a static device array inside this library instead of a caller workspace; nothing here has
+ * a counterpart in the method's description.  The caller still passes q (device bf16
+ * [n_seqs][q_len][num_q_heads][D]) and out (device fp32, same shape).
+ *   - Limit: the static array holds 32 MiB; a call whose partial states need more returns
+ *     MKV_ERR_WORKSPACE_TOO_SMALL.  At most 256 sequences and 1536 work units per call
+ *     (MKV_ERR_UNSUPPORTED beyond).  Other errors as mkv_decode_attention.
+ *   - The array is allocated when the library's device code is loaded and is held by every
+ *     GPU that loads it until the process exits.
+ *   - The first call on a device resolves the array's device address (cudaGetSymbolAddress
+ *     with that device current); make that first call before any stream capture.
+ *   - All calls share the array and it keeps the last call's contents; nothing in it needs to
+ *     start at zero.  Calls that overlap on the GPU (other streams, other pools on the same
+ *     device) race on it: order them.
+ *   - Allocates no device memory and, when it succeeds, no host memory.
+ * Results are identical to mkv_decode_attention's for the same inputs. */
+MKV_API int mkv_decode_attention_noalloc(mkv_pool_t pool, const int32_t* seq_ids, int32_t n_seqs,
+                                         int32_t q_len, const void* q_bf16, int32_t num_q_heads,
+                                         float sm_scale, float* out, void* stream);
+
 /* Free every page of a sequence and clear its table row and flags. */
 MKV_API int mkv_seq_reset(mkv_pool_t pool, int32_t seq, void* stream);
 

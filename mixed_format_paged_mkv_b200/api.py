@@ -48,6 +48,8 @@ SIGNATURES = {
     "mkv_decode_workspace_bytes": (ctypes.c_int, [_P, _I32P, _I32, _I32, _I32, _SZP]),
     "mkv_decode_attention": (ctypes.c_int, [_P, _I32P, _I32, _I32, _P, _I32, ctypes.c_float,
                                             _P, _P, ctypes.c_size_t, _P]),
+    "mkv_decode_attention_noalloc": (ctypes.c_int, [_P, _I32P, _I32, _I32, _P, _I32,
+                                                    ctypes.c_float, _P, _P]),
     "mkv_seq_reset": (ctypes.c_int, [_P, _I32, _P]),
     "mkv_seq_copy": (ctypes.c_int, [_P, _I32, _I32, _P]),
     "mkv_get_block_table": (ctypes.c_int, [_P, _I32, _I32P, _I32, _I32P, _I32P]),

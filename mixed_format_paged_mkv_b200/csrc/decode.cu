@@ -666,4 +666,33 @@ cudaError_t launch_partial(const DecodeParams& p, cudaStream_t s) {
   }
 }
 
+
+// ------------------------------------------------------------------ static decode scratch
+// Partial-state scratch for mkv_decode_attention_noalloc: a file-scope device array, so that
+// callers that cannot allocate device memory can still decode.  Every device that loads the
+// library holds it until exit; all calls share it.
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;
+static __device__ __align__(256) uint8_t g_decode_scratch[kStaticScratchBytes];
+
+// Device address of g_decode_scratch on the current device.  The first call on a device
+// resolves it with cudaGetSymbolAddress (with that device current) and caches it; later calls
+// only read the cache.
+cudaError_t static_decode_scratch(void** ptr, size_t* bytes) {
+  constexpr int kMaxDevices = 64;
+  static void* cache[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  void* p = __atomic_load_n(&cache[dev], __ATOMIC_ACQUIRE);
+  if (!p) {
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return e;
+    __atomic_store_n(&cache[dev], p, __ATOMIC_RELEASE);
+  }
+  *ptr = p;
+  *bytes = kStaticScratchBytes;
+  return cudaSuccess;
+}
+
 }  // namespace mkv

@@ -123,5 +123,6 @@ cudaError_t launch_copy(const CopyParams& p, cudaStream_t s);
 cudaError_t launch_partial(const DecodeParams& p, cudaStream_t s);
 cudaError_t launch_merge(const DecodeParams& p, cudaStream_t s);
 bool partial_supported(int D, int NC);
+cudaError_t static_decode_scratch(void** ptr, size_t* bytes);
 
 }  // namespace mkv

@@ -592,6 +592,129 @@ int mkv_decode_attention(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, i
   return ok();
 }
 
+// Decode with the library's static partial-state scratch instead of a caller workspace.  Same
+// units, order and kernels as mkv_decode_attention (so the same results), planned into a
+// parameter block on the stack: no device allocation and, on success, no host allocation.
+namespace {
+struct NoAllocPlan {
+  DecodeParams prm;
+  int64_t cost[kDecodeMaxUnits];
+  UnitDesc unit[kDecodeMaxUnits];
+  int32_t order[kDecodeMaxUnits];
+};
+}  // namespace
+
+int mkv_decode_attention_noalloc(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs,
+                                 int32_t q_len, const void* q_bf16, int32_t Hq, float sm_scale,
+                                 float* out, void* stream) {
+  if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
+  if (p->host_only) return fail(MKV_ERR_INVALID_ARG, "host-only pool cannot decode");
+  if (n_seqs < 0 || (n_seqs > 0 && !seq_ids)) return fail(MKV_ERR_INVALID_ARG, "bad sequence list");
+  if (n_seqs > p->cfg.max_seqs)
+    return fail(MKV_ERR_INVALID_ARG, "at most max_seqs (%d) sequences per decode call", p->cfg.max_seqs);
+  if (n_seqs > kDecodeMaxSeqs)
+    return fail(MKV_ERR_UNSUPPORTED, "the no-allocation decode takes at most %d sequences per call", kDecodeMaxSeqs);
+  if (q_len < 1) return fail(MKV_ERR_INVALID_ARG, "q_len must be >= 1");
+  if (!std::isfinite(sm_scale)) return fail(MKV_ERR_INVALID_ARG, "sm_scale is not finite");
+  const int Hkv = p->cfg.num_kv_heads, D = p->cfg.head_dim;
+  if (Hq < Hkv || Hq % Hkv) return fail(MKV_ERR_INVALID_ARG, "num_q_heads %d not a multiple of Hkv %d", Hq, Hkv);
+  const int32_t g = Hq / Hkv, NC = q_len * g;
+  if (!partial_supported(D, NC))
+    return fail(MKV_ERR_UNSUPPORTED, "q_len * num_q_heads / Hkv = %d > 32 is not built", NC);
+  const int64_t b8 = fp8_head_bytes(D), b3 = tq3_head_bytes(D);
+  int64_t total = 0;
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    if (int e = check_seq(p, seq_ids[i])) return e;
+    const Seq& s = p->seqs[seq_ids[i]];
+    if (s.ctx < q_len || s.ctx == 0)
+      return fail(MKV_ERR_EMPTY_CONTEXT, "sequence %d has %d tokens < q_len %d", seq_ids[i], s.ctx, q_len);
+    total += static_cast<int64_t>(s.fp8_pages.size()) * b8 + static_cast<int64_t>(s.n3) * b3;
+  }
+  if (n_seqs == 0) return ok();
+  if (!q_bf16 || !out) return fail(MKV_ERR_INVALID_ARG, "q/out is NULL");
+  // the same unit cut as plan_decode
+  const int64_t target_ctas = static_cast<int64_t>(p->sm_count) * 3 * 3;
+  const int64_t per_cta = std::max<int64_t>(1, total * Hkv / target_ctas);
+  const int32_t R3 = static_cast<int32_t>(std::max<int64_t>(8, std::min<int64_t>(kMaxPagesPerUnit, per_cta / b3)));
+  const int32_t P8 = static_cast<int32_t>(std::max<int64_t>(4, std::min<int64_t>(kMaxPagesPerUnit, per_cta / b8)));
+  NoAllocPlan t;  // about 75 KB of stack
+  DecodeParams& prm = t.prm;
+  int32_t nu = 0, parts = 0;
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    const Seq& s = p->seqs[seq_ids[i]];
+    SeqDesc& d = prm.seq[i];
+    d.row = seq_ids[i];
+    d.ctx = s.ctx;
+    d.out_row = i;
+    d.part0 = parts;
+    d.pad = 0;
+    int32_t np = 0;
+    const auto& f8 = s.fp8_pages;
+    const int32_t pages = static_cast<int32_t>(s.table.size());
+    const int64_t need = static_cast<int64_t>((f8.size() + P8 - 1) / P8) + (pages + R3 - 1) / R3;
+    if (nu + need > kDecodeMaxUnits)
+      return fail(MKV_ERR_UNSUPPORTED, "the no-allocation decode takes at most %d work units per call", kDecodeMaxUnits);
+    for (size_t j = 0; j < f8.size(); j += P8) {
+      const size_t k = std::min(f8.size(), j + static_cast<size_t>(P8));
+      t.unit[nu] = {f8[j], f8[k - 1] + 1, static_cast<int16_t>(i), 0, np++};
+      t.cost[nu++] = static_cast<int64_t>(k - j) * b8;
+    }
+    for (int32_t a = 0; a < pages; a += R3) {
+      const int32_t b = std::min(pages, a + R3);
+      const int64_t in8 = std::lower_bound(f8.begin(), f8.end(), b) - std::lower_bound(f8.begin(), f8.end(), a);
+      if ((b - a) - in8 <= 0) continue;
+      t.unit[nu] = {a, b, static_cast<int16_t>(i), 1, np++};
+      t.cost[nu++] = ((b - a) - in8) * b3;
+    }
+    d.n_parts = np;
+    parts += np;
+  }
+  const size_t cols = static_cast<size_t>(parts) * Hkv * NC;
+  const size_t off_acc = align256(cols * 2 * 4);
+  const size_t bytes = off_acc + align256(cols * D * 4);
+  void* scratch = nullptr;
+  size_t cap = 0;
+  cudaError_t err = static_decode_scratch(&scratch, &cap);
+  if (err != cudaSuccess) return cuda_fail(err, "static scratch address");
+  if (bytes > cap)
+    return fail(MKV_ERR_WORKSPACE_TOO_SMALL,
+                "call needs %zu bytes of partial-state scratch; the static scratch holds %zu", bytes, cap);
+  for (int32_t k = 0; k < nu; ++k) t.order[k] = k;
+  std::sort(t.order, t.order + nu, [&](int32_t x, int32_t y) {
+    return t.cost[x] != t.cost[y] ? t.cost[x] > t.cost[y] : x < y;
+  });
+  for (int32_t k = 0; k < nu; ++k) prm.unit[k] = t.unit[t.order[k]];
+  uint8_t* ws = static_cast<uint8_t*>(scratch);
+  prm.fp8_slab = p->fp8_slab;
+  prm.tq3_slab = p->tq3_slab;
+  prm.tables = p->d_tables;
+  prm.status = p->d_status;
+  prm.q = static_cast<const uint16_t*>(q_bf16);
+  prm.out = out;
+  prm.part_ml = reinterpret_cast<float*>(ws);
+  prm.part_acc = reinterpret_cast<float*>(ws + off_acc);
+  prm.fp8_slot_bytes = p->fp8_slot_bytes;
+  prm.tq3_slot_bytes = p->tq3_slot_bytes;
+  prm.Hkv = Hkv;
+  prm.D = D;
+  prm.g = g;
+  prm.q_len = q_len;
+  prm.NC = NC;
+  prm.Hq = Hq;
+  prm.max_pages = p->cfg.max_pages_per_seq;
+  prm.fp8_slots = p->cfg.fp8_slots;
+  prm.tq3_slots = p->cfg.tq3_slots;
+  prm.logit_scale = sm_scale * 1.4426950408889634f;
+  prm.n_seqs = n_seqs;
+  prm.n_units = nu;
+  cudaStream_t st = as_stream(stream);
+  err = launch_partial(prm, st);
+  ++p->launches;
+  if (err == cudaSuccess) err = launch_merge(prm, st), ++p->launches;
+  if (err != cudaSuccess) return cuda_fail(err, "decode launch");
+  return ok();
+}
+
 int mkv_seq_reset(mkv_pool_t p, int32_t seq, void* stream) {
   if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
   if (int e = check_seq(p, seq)) return e;
