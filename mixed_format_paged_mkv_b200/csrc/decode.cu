@@ -12,8 +12,10 @@
 //      unit's format (FP8 units run fp8_page, TQ3 units tq3_page: separate per-format code and
 //      separate partial states);
 //   2. the producer streams those pages through a shared-memory ring with bulk async copies
-//      completing on mbarriers; consumer warps compute (m, l, acc) per query column;
-//   3. the CTA writes its partial state.
+//      completing on mbarriers;
+//   3. consumer warps (pages round-robin) compute per page the logits, the online softmax
+//      (running max m and denominator l per query column) and P.V;
+//   4. the CTA combines its warps and writes its partial state (m, l, acc) per query column.
 // A second kernel merges, per (sequence, KV head, query column), all partial states of both
 // formats: M = max m, L = sum l 2^(m-M), O = sum acc 2^(m-M) / L.
 //
@@ -21,8 +23,9 @@
 // dimension, the q_len*g query columns of one KV head the N dimension) and P.V is a
 // (16 channels x 16 tokens) x (16 tokens x 8 columns) tile, both mma.sync m16n8k16 with f16
 // operands that are exact images of the stored codes.  Dequantisation happens in registers:
-//   TQ3 K: codes -> (c - 3.5) exactly; the per-(token, group) scale multiplies the group's
-//          MMA result (logits are summed over groups in fp32).
+//   TQ3 K: codes -> exact f16 images (base + c); each group's MMA starts from the correction
+//          -(base + 3.5) * (sum of the matching query values), so it yields sum q (c - 3.5);
+//          the per-(token, group) scale multiplies the group's result (summed in fp32).
 //   TQ3 V: codes -> (c - 3.5) exactly; the per-(token, group) scale multiplies P in f16.
 //   FP8:   e4m3x2 -> f16x2 conversions; the per-page scales multiply logits / the page's P.V.
 // Softmax runs in log2 units with a lazily raised reference maximum (raised only when a
@@ -43,31 +46,37 @@ struct Cfg {
   static constexpr int PW = NT == 1 ? 4 : (NT == 2 ? 2 : 1);  // page-parallel warps
   static constexpr int NWC = NT * PW;                          // consumer warps
   static constexpr int THREADS = 32 * (NWC + 1);               // + 1 producer warp
+  static constexpr int PRODUCER = NWC;
   static constexpr int FP8_STAGE = 32 * D + 16;
   static constexpr int TQ3_STAGE = 14 * D;
   static constexpr int FP8_NST = 6;
   static constexpr int TQ3_NST = 16;
   static constexpr int RING_FP8 = FP8_NST * FP8_STAGE;
   static constexpr int RING_TQ3 = TQ3_NST * TQ3_STAGE;
+  // end-of-unit combine: (m, l) and acc of the consumer warps with pw > 0
   static constexpr int COMBINE = (PW - 1) * NT * 8 * (D + 2) * 4;
   static constexpr int RING = RING_FP8 > RING_TQ3 ? (RING_FP8 > COMBINE ? RING_FP8 : COMBINE)
                                                   : (RING_TQ3 > COMBINE ? RING_TQ3 : COMBINE);
-  // Q fragments: per n-tile, D/32 x 32 lanes x 16 bytes
+  // header: full[16] | empty[16] mbarriers | stage tags | misc | page list | Q fragments |
+  //         TQ3 K corrections | ring
+  static constexpr int OFF_TAG = 256;
+  static constexpr int OFF_MISC = OFF_TAG + 64;
+  static constexpr int OFF_LIST = OFF_MISC + 64;
+  static constexpr int OFF_QF = (OFF_LIST + kMaxPagesPerUnit * 8 + 127) / 128 * 128;
   static constexpr int QF = NT * D * 16;
-  // header: 2 x 16 mbarriers | 16 stage tags | misc ints | page list | Q fragments | ring
-  static constexpr int OFF_TAG = 256, OFF_MISC = 320, OFF_LIST = 384;
-  static constexpr int OFF_QF = OFF_LIST + kMaxPagesPerUnit * 8;
-  static constexpr int OFF_RING = OFF_QF + QF;
+  static constexpr int OFF_CORR = OFF_QF + QF;
+  static constexpr int OFF_RING = (OFF_CORR + NT * (D / 32) * 64 + 127) / 128 * 128;
   static constexpr int SMEM = OFF_RING + RING;
 };
 
 struct Smem {
-  uint64_t* full;
-  uint64_t* empty;
-  int32_t* tag;    // logical page of each stage (-1: invalid entry)
-  int32_t* misc;   // [0] page count, [1] abort flag, [4..7] logit scales
-  int2* list;      // {slot, logical page} of the unit's pages
-  uint4* qf;       // Q fragments [NT][D/32][32 lanes]
+  uint64_t* full;   // [stage]: page landed (producer arrive + bulk-copy bytes)
+  uint64_t* empty;  // [stage]: the page's consumer warps are done with it
+  int32_t* tag;     // logical page of each stage
+  int32_t* misc;    // [0] page count, [1] abort flag, [4..7] logit scales per n-tile
+  int2* list;       // {slot, logical page} of the unit's pages
+  uint4* qf;        // Q fragments [NT][D/32][32 lanes]
+  float4* corr;     // TQ3 K corrections [NT][D/32][4 column pairs] as {c0, c1, c0, c1}
   uint8_t* ring;
 };
 
@@ -81,29 +90,37 @@ __device__ __forceinline__ Smem carve(uint8_t* base) {
   s.misc = reinterpret_cast<int32_t*>(base + C::OFF_MISC);
   s.list = reinterpret_cast<int2*>(base + C::OFF_LIST);
   s.qf = reinterpret_cast<uint4*>(base + C::OFF_QF);
+  s.corr = reinterpret_cast<float4*>(base + C::OFF_CORR);
   s.ring = base + C::OFF_RING;
   return s;
 }
 
 __device__ __forceinline__ uint32_t f16x2_const(float lo, float hi) { return pack_f16x2(lo, hi); }
 
-// Per-warp online-softmax state for the thread's two columns (2c, 2c+1) and its share of the
-// P.V accumulator: acc[mt][0..3] = (channel row r, col 2c), (r, 2c+1), (r+8, 2c), (r+8, 2c+1)
-// of channel tile mt; tile 2G+j row r holds channel 32G + 4r + 2j, row r+8 channel 32G+4r+2j+1.
-template <int D>
-struct WarpState {
+// K-warp softmax state for the thread's two columns (2c, 2c+1): reference maximum (log2 units)
+// and this thread's share of the denominator.
+struct KState {
   float m[2];
   float l[2];
+};
+
+// V-warp accumulator: acc[mt][0..3] = (channel row r, col 2c), (r, 2c+1), (r+8, 2c),
+// (r+8, 2c+1) of channel tile mt; tile 2G+j row r holds channel 32G+4r+2j, row r+8 channel
+// 32G+4r+2j+1.
+template <int D>
+struct VState {
   float acc[D / 16][4];
 };
 
 // Logits -> probabilities for one page (thread holds logits x[0..3] for tokens (r, r+8) x
-// columns (2c, 2c+1), in log2 units).  Returns P^T as two B fragments (tokens 0-7, 8-15).
-template <int D>
-__device__ __forceinline__ void softmax_page(WarpState<D>& st, float (&x)[4], uint32_t& pb0,
-                                             uint32_t& pb1) {
+// columns (2c, 2c+1), in log2 units).  Gives P^T as two B fragments (tokens 0-7, 8-15) and the
+// factors (a0, a1) by which earlier accumulations of the two columns must be rescaled (1 when
+// the reference maximum did not move).
+__device__ __forceinline__ void softmax_k(KState& st, float (&x)[4], uint32_t& pb0,
+                                          uint32_t& pb1, float& a0, float& a1) {
   float mx0 = fmaxf(x[0], x[2]);
   float mx1 = fmaxf(x[1], x[3]);
+  a0 = a1 = 1.f;
   const bool need = (mx0 > st.m[0] + kLazyRescale) || (mx1 > st.m[1] + kLazyRescale);
   if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
@@ -112,26 +129,17 @@ __device__ __forceinline__ void softmax_page(WarpState<D>& st, float (&x)[4], ui
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
     }
     const float n0 = fmaxf(st.m[0], mx0), n1 = fmaxf(st.m[1], mx1);
-    const float a0 = (n0 == -INFINITY) ? 1.f : exp2f(st.m[0] - n0);
-    const float a1 = (n1 == -INFINITY) ? 1.f : exp2f(st.m[1] - n1);
-    if (a0 != 1.f || a1 != 1.f) {
-#pragma unroll
-      for (int mt = 0; mt < D / 16; ++mt) {
-        st.acc[mt][0] *= a0;
-        st.acc[mt][2] *= a0;
-        st.acc[mt][1] *= a1;
-        st.acc[mt][3] *= a1;
-      }
-      st.l[0] *= a0;
-      st.l[1] *= a1;
-    }
+    a0 = (n0 == -INFINITY) ? 1.f : fast_exp2(st.m[0] - n0);
+    a1 = (n1 == -INFINITY) ? 1.f : fast_exp2(st.m[1] - n1);
+    st.l[0] *= a0;
+    st.l[1] *= a1;
     st.m[0] = n0;
     st.m[1] = n1;
   }
   const float r0 = st.m[0] == -INFINITY ? 0.f : st.m[0];
   const float r1 = st.m[1] == -INFINITY ? 0.f : st.m[1];
-  const float p0 = exp2f(x[0] - r0), p1 = exp2f(x[1] - r1);
-  const float p2 = exp2f(x[2] - r0), p3 = exp2f(x[3] - r1);
+  const float p0 = fast_exp2(x[0] - r0), p1 = fast_exp2(x[1] - r1);
+  const float p2 = fast_exp2(x[2] - r0), p3 = fast_exp2(x[3] - r1);
   st.l[0] += p0 + p2;
   st.l[1] += p1 + p3;
   pb0 = movmatrix_trans(pack_f16x2(p0, p1));
@@ -151,36 +159,33 @@ __device__ __forceinline__ void mask_page(float (&x)[4], int tok0, int r, int li
 // un-permuted when stored): TQ3 K, group G, lane quad column c: MMA k 2c,2c+1 <- channels
 // 8c+0, 8c+4 (k-block 0), 8c+1, 8c+5 (k-block 0, upper k), 8c+2, 8c+6 / 8c+3, 8c+7 (k-block 1).
 template <int D>
-__device__ __forceinline__ void tq3_page(WarpState<D>& st, const uint8_t* pg,
-                                         const uint4* qf, int lane,
-                                         float ls, int tok0, bool masked, int lim0, int lim1,
-                                         int kw, int ks5, int vw, int vs1) {
+__device__ __forceinline__ void tq3_logits(const uint8_t* pg, const uint4* qf, const float4* corr,
+                                           int lane, int kw, int ks5, float (&x)[4]) {
   constexpr int G = D / 32;
   const int r = lane >> 2, c = lane & 3;
   const uint8_t* krec = pg;
   const __half* kscale = reinterpret_cast<const __half*>(pg + G * 16 * 12);
-  const uint8_t* vrec = pg + G * 16 * 14;
-  const __half* vscale = reinterpret_cast<const __half*>(vrec + G * 16 * 12);
-  const uint32_t kMask = 0x000E00E0u, kMagic = 0x60005000u;
-  const uint32_t kSub = f16x2_const(35.5f, 515.5f);
-
-  float x[4] = {0.f, 0.f, 0.f, 0.f};
+  // K images: code k of a pair lands in mantissa bits 7-9 of the low half (value 8 + c) and
+  // code k+4 in bits 3-5 of the high half (value 128 + c); both exact.  The offsets 11.5 and
+  // 131.5 (base + 3.5) times the query sums are the group's starting accumulator (corr).
+  uint32_t kMask = 0x00380380u, kMagic = 0x58004800u;
+  opaque(kMask, kMagic);
+  x[0] = x[1] = x[2] = x[3] = 0.f;
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     const uint32_t* ra = reinterpret_cast<const uint32_t*>(krec + 12 * (16 * g + r));
     const uint32_t* rb = ra + 24;  // token r + 8
-    const uint32_t xa = __funnelshift_r(ra[kw], ra[kw + 1], ks5);
+    const uint32_t xa = __funnelshift_r(ra[kw], ra[kw + 1], ks5);  // code j at bit 3j+5
     const uint32_t xb = __funnelshift_r(rb[kw], rb[kw + 1], ks5);
-    uint32_t a[4], b[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      a[j] = hsub2_u32(((xa >> (3 * j)) & kMask) | kMagic, kSub);
-      b[j] = hsub2_u32(((xb >> (3 * j)) & kMask) | kMagic, kSub);
-    }
+    const uint32_t a0 = ((xa << 2) & kMask) | kMagic, b0 = ((xb << 2) & kMask) | kMagic;
+    const uint32_t a1 = ((xa >> 1) & kMask) | kMagic, b1 = ((xb >> 1) & kMask) | kMagic;
+    const uint32_t a2 = ((xa >> 4) & kMask) | kMagic, b2 = ((xb >> 4) & kMask) | kMagic;
+    const uint32_t a3 = ((xa >> 7) & kMask) | kMagic, b3 = ((xb >> 7) & kMask) | kMagic;
     const uint4 qb = qf[32 * g + lane];
-    float cg[4] = {0.f, 0.f, 0.f, 0.f};
-    mma_f16_16816(cg, a[0], b[0], a[1], b[1], qb.x, qb.y, cg);
-    mma_f16_16816(cg, a[2], b[2], a[3], b[3], qb.z, qb.w, cg);
+    const float4 cr = corr[4 * g + c];
+    float cg[4] = {cr.x, cr.y, cr.z, cr.w};
+    mma_f16_16816(cg, a0, b0, a1, b1, qb.x, qb.y, cg);
+    mma_f16_16816(cg, a2, b2, a3, b3, qb.z, qb.w, cg);
     const float sa = __half2float(kscale[16 * g + r]);
     const float sb = __half2float(kscale[16 * g + r + 8]);
     x[0] = fmaf(sa, cg[0], x[0]);
@@ -188,17 +193,23 @@ __device__ __forceinline__ void tq3_page(WarpState<D>& st, const uint8_t* pg,
     x[2] = fmaf(sb, cg[2], x[2]);
     x[3] = fmaf(sb, cg[3], x[3]);
   }
-#pragma unroll
-  for (int j = 0; j < 4; ++j) x[j] *= ls;
-  if (masked) mask_page(x, tok0, r, lim0, lim1);
-  uint32_t pb0, pb1;
-  softmax_page<D>(st, x, pb0, pb1);
+}
 
-  // V: A = V^T tile (channels x tokens); lane row r holds channels 32G+4r+{0,1} (tile 2G)
-  // and 32G+4r+{2,3} (tile 2G+1) for tokens (2c, 2c+1) and (2c+8, 2c+9).
-  const uint32_t m0 = 0x000E000Eu, g0 = 0x60006000u, s0 = f16x2_const(515.5f, 515.5f);
-  const uint32_t m1 = 0x00700070u, g1 = 0x54005400u, s1 = f16x2_const(67.5f, 67.5f);
-  const uint32_t m2 = 0x03800380u, g2 = 0x48004800u, s2 = f16x2_const(11.5f, 11.5f);
+// V: A = V^T tile (channels x tokens); lane row r holds channels 32G+4r+{0,1} (tile 2G) and
+// 32G+4r+{2,3} (tile 2G+1) for tokens (2c, 2c+1) and (2c+8, 2c+9); codes -> exact (c - 3.5);
+// the per-(token, group) scale multiplies P in f16.
+template <int D>
+__device__ __forceinline__ void tq3_pv(VState<D>& st, const uint8_t* pg, int lane, int vw,
+                                       int vs1, uint32_t pb0, uint32_t pb1) {
+  constexpr int G = D / 32;
+  const int c = lane & 3;
+  const uint8_t* vrec = pg + G * 16 * 14;
+  const __half* vscale = reinterpret_cast<const __half*>(vrec + G * 16 * 12);
+  uint32_t m0 = 0x000E000Eu, g0 = 0x60006000u, m1 = 0x00700070u, g1 = 0x54005400u;
+  uint32_t m2 = 0x03800380u, g2 = 0x48004800u;
+  opaque(m0, g0, m1, g1, m2, g2);
+  const uint32_t s0 = f16x2_const(515.5f, 515.5f), s1 = f16x2_const(67.5f, 67.5f);
+  const uint32_t s2 = f16x2_const(11.5f, 11.5f);
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     const uint32_t* rc = reinterpret_cast<const uint32_t*>(vrec + 12 * (16 * g + 2 * c));
@@ -226,12 +237,10 @@ __device__ __forceinline__ void tq3_page(WarpState<D>& st, const uint8_t* pg,
 // K channel order: k-block kb = 4j + i, lane quad column c: k 2c,2c+1 <- channels
 // 64j+16c+4i+{0,1}, k 2c+8,2c+9 <- 64j+16c+4i+{2,3}.
 template <int D>
-__device__ __forceinline__ void fp8_page(WarpState<D>& st, const uint8_t* pg,
-                                         const uint4* qf, int lane, float ls,
-                                         int tok0, bool masked, int lim0, int lim1) {
+__device__ __forceinline__ void fp8_logits(const uint8_t* pg, const uint4* qf, int lane,
+                                           float (&x)[4]) {
   const int r = lane >> 2, c = lane & 3;
   const float sk = *reinterpret_cast<const float*>(pg + 32 * D);
-  const float sv = *reinterpret_cast<const float*>(pg + 32 * D + 4);
   float cg[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int j = 0; j < D / 64; ++j) {
@@ -248,14 +257,17 @@ __device__ __forceinline__ void fp8_page(WarpState<D>& st, const uint8_t* pg,
                     qq[2 * i], qq[2 * i + 1], cg);
     }
   }
-  float x[4];
-  const float lsk = ls * sk;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) x[j] = cg[j] * lsk;
-  if (masked) mask_page(x, tok0, r, lim0, lim1);
-  uint32_t pb0, pb1;
-  softmax_page<D>(st, x, pb0, pb1);
+  for (int j = 0; j < 4; ++j) x[j] = cg[j] * sk;
+}
 
+// V channel order as for TQ3 (lane row r: channels 32g+4r+{0..3}); the page's V scale
+// multiplies the page's P.V result per channel tile.
+template <int D>
+__device__ __forceinline__ void fp8_pv(VState<D>& st, const uint8_t* pg, int lane, uint32_t pb0,
+                                       uint32_t pb1) {
+  const int r = lane >> 2, c = lane & 3;
+  const float sv = *reinterpret_cast<const float*>(pg + 32 * D + 4);
   const uint8_t* vrows = pg + 16 * D;
 #pragma unroll
   for (int g = 0; g < D / 32; ++g) {
@@ -293,7 +305,7 @@ __device__ __forceinline__ const uint16_t* q_row(const DecodeParams& p, const Se
 // with the power of two undone.
 template <int D, bool FP8>
 __device__ __forceinline__ float build_q(const DecodeParams& p, const SeqDesc& sd, int h, int nt,
-                                         int lane, uint4* qf) {
+                                         int lane, uint4* qf, float* corr) {
   const int r = lane >> 2, c = lane & 3;
   const uint16_t* qr = q_row(p, sd, h, 8 * nt + r);
   float qv[D / 4];
@@ -330,6 +342,22 @@ __device__ __forceinline__ float build_q(const DecodeParams& p, const SeqDesc& s
       f.y = pack_f16x2(v[1] * qs, v[5] * qs);
       f.z = pack_f16x2(v[2] * qs, v[6] * qs);
       f.w = pack_f16x2(v[3] * qs, v[7] * qs);
+      // correction of this column and group: -(11.5 * sum of the f16 q that meet codes 0-3
+      // of a chunk + 131.5 * sum of those that meet codes 4-7), over the 4 chunks
+      float lo = 0.f, hi = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        lo += __half2float(__float2half_rn(v[e] * qs));
+        hi += __half2float(__float2half_rn(v[e + 4] * qs));
+      }
+      float part = -(11.5f * lo + 131.5f * hi);
+      part += __shfl_xor_sync(0xffffffffu, part, 1);
+      part += __shfl_xor_sync(0xffffffffu, part, 2);
+      if (c == 0) {  // stored twice per column pair: {col 2k, col 2k+1, col 2k, col 2k+1}
+        float* c4 = corr + 16 * w + 4 * (r >> 1) + (r & 1);
+        c4[0] = part;
+        c4[2] = part;
+      }
     }
     qf[32 * w + lane] = f;
   }
@@ -390,19 +418,23 @@ __device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDes
     sm.misc[1] = 0;
     mbar_fence_init();
   }
-  if (warp == C::NWC) {
+  if (warp == C::PRODUCER) {
     const int32_t* row = p.tables + static_cast<int64_t>(sd.row) * p.max_pages;
     const int n = scan_range(p, row, u.first, u.last, FP8 ? 0 : 1, lane, sm.list);
     if (lane == 0) sm.misc[0] = n;
   } else if (pw == 0) {
-    const float ls = build_q<D, FP8>(p, sd, h, nt, lane, sm.qf + nt * (D / 32) * 32);
+    const float ls = build_q<D, FP8>(p, sd, h, nt, lane, sm.qf + nt * (D / 32) * 32,
+                                     reinterpret_cast<float*>(sm.corr + nt * (D / 32) * 4));
     if (lane == 0) reinterpret_cast<float*>(sm.misc)[4 + nt] = ls;
   }
   __syncthreads();
   const int count = sm.misc[0];
 
-  WarpState<D> st;
-  if (warp == C::NWC) {
+  KState ks;
+  VState<D> vs;
+  ks.m[0] = ks.m[1] = -INFINITY;
+  ks.l[0] = ks.l[1] = 0.f;
+  if (warp == C::PRODUCER) {
     // ---------------- producer: one lane streams the unit's pages into the ring
     if (lane == 0) {
       const uint8_t* slab = FP8 ? p.fp8_slab : p.tq3_slab;
@@ -430,47 +462,66 @@ __device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDes
       }
     }
   } else {
-    // ---------------- consumers
+    // ---------------- consumers: logits, online softmax, P.V per page
     const int n0 = 8 * nt + 2 * c, n1 = n0 + 1;
     const int lim0 = n0 < p.NC ? sd.ctx - p.q_len + n0 / p.g : sd.ctx - 1;
     const int lim1 = n1 < p.NC ? sd.ctx - p.q_len + n1 / p.g : sd.ctx - 1;
     const int min_lim = sd.ctx - p.q_len;
     const float ls = reinterpret_cast<const float*>(sm.misc)[4 + nt];
     const uint4* qf = sm.qf + nt * (D / 32) * 32;
-    // TQ3 lane constants: K chunk c of a record starts at bit 24c; we read bits from 24c-5
-    // (codes land at 5+3k); V field of row r starts at bit 12r; we read from 12r-1.
+    const float4* corr = sm.corr + nt * (D / 32) * 4;
+    // TQ3 K chunk c of a record starts at bit 24c; read from bit 24c-5 (codes at 5+3k).
+    // TQ3 V field of row r starts at bit 12r; read from bit 12r-1 (codes at 1+3k).
     const int kbit = 24 * c - 5, vbit = 12 * r - 1;
     const int kw = kbit >= 0 ? kbit >> 5 : -1, ks5 = kbit & 31;
     const int vw = vbit >= 0 ? vbit >> 5 : -1, vs1 = vbit & 31;
-
-    st.m[0] = st.m[1] = -INFINITY;
-    st.l[0] = st.l[1] = 0.f;
 #pragma unroll
     for (int mt = 0; mt < D / 16; ++mt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) st.acc[mt][e] = 0.f;
+      for (int e = 0; e < 4; ++e) vs.acc[mt][e] = 0.f;
 
     for (int i = pw; i < count; i += C::PW) {
       const int s = i % NST;
-      if (!mbar_wait(&sm.full[s], (i / NST) & 1)) {
-        flag_status(p.status, kStatusTimeout);
-        atomicExch(&sm.misc[1], 1);
+      if (!mbar_wait_warp(&sm.full[s], (i / NST) & 1)) {
+        if (lane == 0) {
+          flag_status(p.status, kStatusTimeout);
+          atomicExch(&sm.misc[1], 1);
+        }
         break;
       }
       const int tok0 = 16 * sm.tag[s];
-      const bool masked = tok0 + 15 > min_lim;
       const uint8_t* pg = sm.ring + s * STAGE;
+      float x[4];
       if constexpr (FP8)
-        fp8_page<D>(st, pg, qf, lane, ls, tok0, masked, lim0, lim1);
+        fp8_logits<D>(pg, qf, lane, x);
       else
-        tq3_page<D>(st, pg, qf, lane, ls, tok0, masked, lim0, lim1, kw, ks5, vw, vs1);
+        tq3_logits<D>(pg, qf, corr, lane, kw, ks5, x);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) x[j] *= ls;
+      if (tok0 + 15 > min_lim) mask_page(x, tok0, r, lim0, lim1);
+      uint32_t pb0, pb1;
+      float a0, a1;
+      softmax_k(ks, x, pb0, pb1, a0, a1);
+      if (__any_sync(0xffffffffu, a0 != 1.f || a1 != 1.f)) {
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+          vs.acc[mt][0] *= a0;
+          vs.acc[mt][2] *= a0;
+          vs.acc[mt][1] *= a1;
+          vs.acc[mt][3] *= a1;
+        }
+      }
+      if constexpr (FP8)
+        fp8_pv<D>(vs, pg, lane, pb0, pb1);
+      else
+        tq3_pv<D>(vs, pg, lane, vw, vs1, pb0, pb1);
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.empty[s]);
     }
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
-      st.l[0] += __shfl_xor_sync(0xffffffffu, st.l[0], o);
-      st.l[1] += __shfl_xor_sync(0xffffffffu, st.l[1], o);
+      ks.l[0] += __shfl_xor_sync(0xffffffffu, ks.l[0], o);
+      ks.l[1] += __shfl_xor_sync(0xffffffffu, ks.l[1], o);
     }
   }
   __syncthreads();  // ring no longer needed: reuse it for the cross-warp combine
@@ -480,23 +531,24 @@ __device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDes
   if (warp < C::NWC && pw > 0) {
     float* reg = cmb + ((pw - 1) * NT + nt) * REGION;
     if (r == 0) {
-      reg[2 * (2 * c)] = st.m[0];
-      reg[2 * (2 * c) + 1] = st.l[0];
-      reg[2 * (2 * c + 1)] = st.m[1];
-      reg[2 * (2 * c + 1) + 1] = st.l[1];
+      reg[2 * (2 * c)] = ks.m[0];
+      reg[2 * (2 * c) + 1] = ks.l[0];
+      reg[2 * (2 * c + 1)] = ks.m[1];
+      reg[2 * (2 * c + 1) + 1] = ks.l[1];
     }
     float* ra = reg + 16;
 #pragma unroll
     for (int mt = 0; mt < D / 16; ++mt) {
       const int ch = 32 * (mt >> 1) + 4 * r + 2 * (mt & 1);
-      ra[(2 * c) * D + ch] = st.acc[mt][0];
-      ra[(2 * c + 1) * D + ch] = st.acc[mt][1];
-      ra[(2 * c) * D + ch + 1] = st.acc[mt][2];
-      ra[(2 * c + 1) * D + ch + 1] = st.acc[mt][3];
+      ra[(2 * c) * D + ch] = vs.acc[mt][0];
+      ra[(2 * c + 1) * D + ch] = vs.acc[mt][1];
+      ra[(2 * c) * D + ch + 1] = vs.acc[mt][2];
+      ra[(2 * c + 1) * D + ch + 1] = vs.acc[mt][3];
     }
   }
   __syncthreads();
   if (warp < C::NWC && pw == 0) {
+    float m[2] = {ks.m[0], ks.m[1]}, l[2] = {ks.l[0], ks.l[1]};
     for (int o = 1; o < C::PW; ++o) {
       const float* reg = cmb + ((o - 1) * NT + nt) * REGION;
       const float* ra = reg + 16;
@@ -504,21 +556,20 @@ __device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDes
       for (int k = 0; k < 2; ++k) {
         const int col = 2 * c + k;
         const float mo = reg[2 * col], lo = reg[2 * col + 1];
-        const float M = fmaxf(st.m[k], mo);
+        const float M = fmaxf(m[k], mo);
         if (M == -INFINITY) continue;
-        const float as = st.m[k] == -INFINITY ? 0.f : exp2f(st.m[k] - M);
+        const float as = m[k] == -INFINITY ? 0.f : exp2f(m[k] - M);
         const float ao = mo == -INFINITY ? 0.f : exp2f(mo - M);
-        st.l[k] = st.l[k] * as + lo * ao;
+        l[k] = l[k] * as + lo * ao;
 #pragma unroll
         for (int mt = 0; mt < D / 16; ++mt) {
           const int ch = 32 * (mt >> 1) + 4 * r + 2 * (mt & 1);
-          st.acc[mt][k] = st.acc[mt][k] * as + ra[col * D + ch] * ao;
-          st.acc[mt][k + 2] = st.acc[mt][k + 2] * as + ra[col * D + ch + 1] * ao;
+          vs.acc[mt][k] = vs.acc[mt][k] * as + ra[col * D + ch] * ao;
+          vs.acc[mt][k + 2] = vs.acc[mt][k + 2] * as + ra[col * D + ch + 1] * ao;
         }
-        st.m[k] = M;
+        m[k] = M;
       }
     }
-    // write the partial state of columns 8nt + 2c + k
     const int part = sd.part0 + u.part;
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
@@ -526,14 +577,14 @@ __device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDes
       if (n >= p.NC) continue;
       const int64_t base = (static_cast<int64_t>(part) * p.Hkv + h) * p.NC + n;
       if (r == 0) {
-        p.part_ml[2 * base] = st.m[k];
-        p.part_ml[2 * base + 1] = st.l[k];
+        p.part_ml[2 * base] = m[k];
+        p.part_ml[2 * base + 1] = l[k];
       }
       float* dst = p.part_acc + base * D;
 #pragma unroll
       for (int g = 0; g < D / 32; ++g) {
-        const float4 v = make_float4(st.acc[2 * g][k], st.acc[2 * g][k + 2],
-                                     st.acc[2 * g + 1][k], st.acc[2 * g + 1][k + 2]);
+        const float4 v = make_float4(vs.acc[2 * g][k], vs.acc[2 * g][k + 2],
+                                     vs.acc[2 * g + 1][k], vs.acc[2 * g + 1][k + 2]);
         *reinterpret_cast<float4*>(dst + 32 * g + 4 * r) = v;
       }
     }

@@ -66,6 +66,30 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   }
 }
 
+// Warp-collective form: every lane polls (each acquires the barrier's phase), then the warp
+// reconverges, so warp-synchronous instructions that follow (mma.sync.aligned, movmatrix) run
+// converged.  Returns false on every lane if any lane gave up.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity) {
+  const bool ok = mbar_wait(bar, parity);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Hide the values of bit-mask constants from the compiler so that it keeps them in registers
+// instead of re-materialising an immediate at every use (a LOP3 has one immediate slot, so
+// `(x & mask) | magic` with two literal constants costs an extra move per use).
+__device__ __forceinline__ void opaque1(uint32_t& v) { asm volatile("" : "+r"(v)); }
+template <typename... T>
+__device__ __forceinline__ void opaque(T&... v) {
+  (opaque1(v), ...);
+}
+
+// 2^x with the MUFU approximation (ftz); x = -inf gives 0.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ------------------------------------------------------------------ bulk copy global -> smem
 // One contiguous async copy completing on an mbarrier (no multicast).  dst, src and bytes
 // must be multiples of 16.
@@ -83,7 +107,7 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
 __device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
                                               uint32_t a2, uint32_t a3, uint32_t b0,
                                               uint32_t b1, const float (&c)[4]) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
       "{%8,%9}, {%10,%11,%12,%13};"
       : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
@@ -95,7 +119,7 @@ __device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32
 // (lane = 4*row + col/2) into the same layout.
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   uint32_t y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
   return y;
 }
 
