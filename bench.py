@@ -36,7 +36,10 @@ METRIC = "decode-attention µs/step and KV GB/s read (fraction of B200 HBM roofl
 FALLBACK_HBM_GBS = 6650.0
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the partial-attention kernel, from
 # the ncu capture summarised in profiles/, keyed by the hash of the kernel sources it measured.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # profiles/decode_kernel_long_ctx128k_1layer.md: 494,559,744 B read + 9,681,408 B written
+    "b9ec8f134d6dc117": 504241152,
+}
 
 
 def kernel_hash() -> str:

@@ -49,8 +49,12 @@ struct Cfg {
   static constexpr int PRODUCER = NWC;
   static constexpr int FP8_STAGE = 32 * D + 16;
   static constexpr int TQ3_STAGE = 14 * D;
-  static constexpr int FP8_NST = 6;
+  // Every stage must always be consumed by the same warp(s): a warp waits on a stage's fill f
+  // with parity f & 1, which is only unambiguous if fill f-1 of that stage was its own (and so
+  // already completed).  Hence ring depths are multiples of PW.
+  static constexpr int FP8_NST = 8;
   static constexpr int TQ3_NST = 16;
+  static_assert(FP8_NST % PW == 0 && TQ3_NST % PW == 0, "stage ownership");
   static constexpr int RING_FP8 = FP8_NST * FP8_STAGE;
   static constexpr int RING_TQ3 = TQ3_NST * TQ3_STAGE;
   // end-of-unit combine: (m, l) and acc of the consumer warps with pw > 0
