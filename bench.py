@@ -80,6 +80,23 @@ def decode_bytes(tables, ctxs, Hkv, D, Hq, q_len):
     return kv + 4 * ent + q + out, kv + q
 
 
+# ---------------------------------------------------------------------------- ranks
+def rank_max(x: float, world: int, device=None) -> float:
+    """Maximum of a per-rank float over all ranks (the job's time is its slowest rank)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_rank: float, world: int, elapsed_max_ms: float) -> float:
+    """Whole-job GB/s of independent replicas: every rank's bytes over the slowest rank's time."""
+    return bytes_per_rank * world / (elapsed_max_ms * 1e-3) / 1e9
+
+
 # ---------------------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -273,11 +290,7 @@ def run_gpu(args, rank, world, local_rank):
         torch.cuda.synchronize()
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return rank_max(x, world, device)
 
     # ---------------- device-resident run (value)
     for s in range(args.warmup):
@@ -305,8 +318,7 @@ def run_gpu(args, rank, world, local_rank):
     pool.device_status()
     per_call_total = 0.5 * (b0[0] + b1[0])
     per_call_partial = 0.5 * (b0[1] + b1[1])
-    bytes_all = per_call_total * layers * args.steps * world
-    value_gbs = bytes_all / (elapsed_ms * 1e-3) / 1e9
+    value_gbs = job_throughput(per_call_total * layers * args.steps, world, elapsed_ms)
     partial_ms = tm["partial_ms"] / max(tm["calls"], 1)
     achieved = per_call_partial / (partial_ms * 1e-3) / 1e9
     peak, peak_src = hbm_peak()
@@ -344,8 +356,8 @@ def run_gpu(args, rank, world, local_rank):
         barrier()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1))
         b2 = tables_now()
-        e2e_bytes = 0.5 * (b1[0] + b2[0]) * layers * args.steps * world
-        e2e = {"value": round(e2e_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+        e2e_gbs = job_throughput(0.5 * (b1[0] + b2[0]) * layers * args.steps, world, e2e_ms)
+        e2e = {"value": round(e2e_gbs, 2), "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": round(e2e_ms / args.steps, 4)}
         pool.device_status()
