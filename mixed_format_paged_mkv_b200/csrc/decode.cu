@@ -181,10 +181,10 @@ __device__ __forceinline__ void tq3_logits(const uint8_t* pg, const uint4* qf, c
     const uint32_t* rb = ra + 24;  // token r + 8
     const uint32_t xa = __funnelshift_r(ra[kw], ra[kw + 1], ks5);  // code j at bit 3j+5
     const uint32_t xb = __funnelshift_r(rb[kw], rb[kw + 1], ks5);
-    const uint32_t a0 = ((xa << 2) & kMask) | kMagic, b0 = ((xb << 2) & kMask) | kMagic;
-    const uint32_t a1 = ((xa >> 1) & kMask) | kMagic, b1 = ((xb >> 1) & kMask) | kMagic;
-    const uint32_t a2 = ((xa >> 4) & kMask) | kMagic, b2 = ((xb >> 4) & kMask) | kMagic;
-    const uint32_t a3 = ((xa >> 7) & kMask) | kMagic, b3 = ((xb >> 7) & kMask) | kMagic;
+    const uint32_t a0 = and_or(xa << 2, kMask, kMagic), b0 = and_or(xb << 2, kMask, kMagic);
+    const uint32_t a1 = and_or(xa >> 1, kMask, kMagic), b1 = and_or(xb >> 1, kMask, kMagic);
+    const uint32_t a2 = and_or(xa >> 4, kMask, kMagic), b2 = and_or(xb >> 4, kMask, kMagic);
+    const uint32_t a3 = and_or(xa >> 7, kMask, kMagic), b3 = and_or(xb >> 7, kMask, kMagic);
     const uint4 qb = qf[32 * g + lane];
     const float4 cr = corr[4 * g + c];
     float cg[4] = {cr.x, cr.y, cr.z, cr.w};
@@ -223,11 +223,11 @@ __device__ __forceinline__ void tq3_pv(VState<D>& st, const uint8_t* pg, int lan
     const uint32_t f9 = __funnelshift_r(rc[vw + 27], rc[vw + 28], vs1);  // token 2c+9
     const uint32_t z01 = __byte_perm(f0, f1, 0x5410);
     const uint32_t z89 = __byte_perm(f8, f9, 0x5410);
-    const uint32_t a0 = hsub2_u32((z01 & m0) | g0, s0), b0 = hsub2_u32((z89 & m0) | g0, s0);
-    const uint32_t a1 = hsub2_u32((z01 & m1) | g1, s1), b1 = hsub2_u32((z89 & m1) | g1, s1);
-    const uint32_t a2 = hsub2_u32((z01 & m2) | g2, s2), b2 = hsub2_u32((z89 & m2) | g2, s2);
-    const uint32_t a3 = hsub2_u32(((z01 >> 3) & m2) | g2, s2);
-    const uint32_t b3 = hsub2_u32(((z89 >> 3) & m2) | g2, s2);
+    const uint32_t a0 = hsub2_u32(and_or(z01, m0, g0), s0), b0 = hsub2_u32(and_or(z89, m0, g0), s0);
+    const uint32_t a1 = hsub2_u32(and_or(z01, m1, g1), s1), b1 = hsub2_u32(and_or(z89, m1, g1), s1);
+    const uint32_t a2 = hsub2_u32(and_or(z01, m2, g2), s2), b2 = hsub2_u32(and_or(z89, m2, g2), s2);
+    const uint32_t a3 = hsub2_u32(and_or(z01 >> 3, m2, g2), s2);
+    const uint32_t b3 = hsub2_u32(and_or(z89 >> 3, m2, g2), s2);
     const uint32_t sv0 = *reinterpret_cast<const uint32_t*>(vscale + 16 * g + 2 * c);
     const uint32_t sv8 = *reinterpret_cast<const uint32_t*>(vscale + 16 * g + 2 * c + 8);
     const uint32_t q0 = hmul2_u32(pb0, sv0), q1 = hmul2_u32(pb1, sv8);

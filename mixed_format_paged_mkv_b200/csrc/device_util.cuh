@@ -98,6 +98,14 @@ __device__ __forceinline__ void opaque(T&... v) {
   (opaque1(v), ...);
 }
 
+// (a & mask) | bits as one three-input logic instruction.  Written out because the compiler
+// splits the expression into two instructions when mask and bits live in registers.
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t mask, uint32_t bits) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "r"(bits));
+  return d;
+}
+
 // 2^x with the MUFU approximation (ftz); x = -inf gives 0.
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
