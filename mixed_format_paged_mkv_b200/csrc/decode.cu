@@ -674,18 +674,45 @@ __global__ void __launch_bounds__(Cfg<D, NT>::THREADS, 3)
     run_unit<D, NT, false>(p, sd, u, h, sm);
 }
 
+// Per-instantiation launch set-up, done once: the dynamic shared-memory opt-in and the number of
+// CTAs the SM keeps resident (the planner sizes work units from it).
+template <int D, int NT>
+struct KernelInfo {
+  cudaError_t err = cudaSuccess;
+  int ctas_per_sm = 1;
+  KernelInfo() {
+    using C = Cfg<D, NT>;
+    err = cudaFuncSetAttribute(decode_kernel<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               C::SMEM);
+    int n = 0;
+    if (err == cudaSuccess)
+      err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<D, NT>, C::THREADS,
+                                                          C::SMEM);
+    ctas_per_sm = n > 0 ? n : 1;
+  }
+  static const KernelInfo& get() {
+    static const KernelInfo info;
+    return info;
+  }
+};
+
 template <int D, int NT>
 cudaError_t launch_t(const DecodeParams& p, cudaStream_t s) {
   using C = Cfg<D, NT>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, NT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  const KernelInfo<D, NT>& info = KernelInfo<D, NT>::get();
+  if (info.err != cudaSuccess) return info.err;
   decode_kernel<D, NT><<<p.n_units * p.Hkv, C::THREADS, C::SMEM, s>>>(p);
   return cudaGetLastError();
+}
+
+template <int D>
+int ctas_per_sm_d(int nt) {
+  switch (nt) {
+    case 1: return KernelInfo<D, 1>::get().ctas_per_sm;
+    case 2: return KernelInfo<D, 2>::get().ctas_per_sm;
+    case 3: return KernelInfo<D, 3>::get().ctas_per_sm;
+    default: return KernelInfo<D, 4>::get().ctas_per_sm;
+  }
 }
 
 template <int D>
@@ -700,6 +727,15 @@ cudaError_t launch_d(const DecodeParams& p, cudaStream_t s) {
 }
 
 }  // namespace
+
+int partial_ctas_per_sm(int D, int NC) {
+  const int nt = (NC + 7) / 8;
+  switch (D) {
+    case 64: return ctas_per_sm_d<64>(nt);
+    case 128: return ctas_per_sm_d<128>(nt);
+    default: return ctas_per_sm_d<256>(nt);
+  }
+}
 
 bool partial_supported(int D, int NC) {
   return (D == 64 || D == 128 || D == 256) && NC >= 1 && NC <= 32;

@@ -97,7 +97,7 @@ struct UnitDesc {
 };
 constexpr int kDecodeMaxSeqs = 256;
 constexpr int kDecodeMaxUnits = 1536;
-constexpr int kMaxPagesPerUnit = 256;  // pages of the unit's format inside its range
+constexpr int kMaxPagesPerUnit = 512;  // pages of the unit's format inside its range
 struct DecodeParams {
   const uint8_t* fp8_slab;
   const uint8_t* tq3_slab;
@@ -123,6 +123,8 @@ cudaError_t launch_copy(const CopyParams& p, cudaStream_t s);
 cudaError_t launch_partial(const DecodeParams& p, cudaStream_t s);
 cudaError_t launch_merge(const DecodeParams& p, cudaStream_t s);
 bool partial_supported(int D, int NC);
+// CTAs of the partial kernel for (D, NC) that one SM keeps resident (queried once).
+int partial_ctas_per_sm(int D, int NC);
 cudaError_t static_decode_scratch(void** ptr, size_t* bytes);
 
 }  // namespace mkv

@@ -158,16 +158,121 @@ struct DecodePlan {
   int32_t NC = 0, g = 0;
   std::vector<SeqDesc> seq;    // per call position
   std::vector<UnitDesc> unit;  // per sequence, in order; UnitDesc::seq = call position
-  std::vector<int64_t> cost;   // bytes per KV head of each unit
+  std::vector<int64_t> cost;   // relative time of each unit (per KV head)
   int64_t parts = 0;
   size_t off_ml = 0, off_acc = 0, bytes = 0;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Cut every sequence into work units: TQ3 units are logical ranges of R3 pages (FP8 pages inside
-// are left to FP8 units); FP8 units are runs of up to P8 consecutive FP8 pages.  R3 and P8 aim at
-// about three waves of three CTAs per SM, each CTA reading a similar number of bytes.
+// Work-unit cut shared by both decode entry points (no allocation).  A unit is one format's
+// pages inside a logical page range of one sequence; the partial kernel runs one CTA per (unit,
+// KV head).  Units are cut for a single wave: at most SMs x resident CTAs per SM CTAs, each
+// (sequence, format) group split into equal parts, and the unit cost chosen as the smallest that
+// fits that budget, so the longest CTA, which ends the wave, is as short as the groups allow.
+// A single balanced wave measured faster than several smaller ones: each CTA sets up and
+// combines its warps once and no partial last wave is left.  Units hold at most
+// kMaxPagesPerUnit and at least a few pages.  `emit(unit, cost)` is called in sequence order;
+// UnitDesc::part numbers the units of a sequence.  Returns the unit count, or -1 as soon as
+// `emit` returns false.
+constexpr int kMinTq3PagesPerUnit = 8;
+constexpr int kMinFp8PagesPerUnit = 4;
+// Relative time of one page of each format in a CTA (measured with device timestamps on the
+// long-context workload: 0.45 us per TQ3 page and 0.48-0.53 us per FP8 page per CTA).  Units are
+// balanced by time, not bytes: an FP8 page carries 2.3x the bytes of a TQ3 page but costs less
+// arithmetic per byte.
+constexpr int64_t kFp8PageCost = 11;
+constexpr int64_t kTq3PageCost = 10;
+
+template <class Emit>
+int64_t cut_units(const mkv_pool* p, const int32_t* seq_ids, int32_t n, int32_t NC,
+                  int32_t* n_parts, Emit&& emit) {
+  const int64_t b8 = kFp8PageCost, b3 = kTq3PageCost;
+  const int Hkv = p->cfg.num_kv_heads;
+  int64_t total = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    const Seq& s = p->seqs[seq_ids[i]];
+    total += static_cast<int64_t>(s.fp8_pages.size()) * b8 + static_cast<int64_t>(s.n3) * b3;
+  }
+  const int64_t slots =
+      static_cast<int64_t>(p->sm_count) * partial_ctas_per_sm(p->cfg.head_dim, NC);
+  const int64_t U = std::max<int64_t>(1, slots / Hkv);
+  // units of a group at unit cost c: as many as its cost needs, clamped to the page limits
+  auto units_at = [](double c, int64_t cost, int64_t pages, int min_pages) -> int64_t {
+    const int64_t lo = (pages + kMaxPagesPerUnit - 1) / kMaxPagesPerUnit;
+    const int64_t hi = std::max<int64_t>(lo, std::max<int64_t>(1, pages / min_pages));
+    const int64_t u = static_cast<int64_t>(std::ceil(static_cast<double>(cost) / c - 1e-9));
+    return std::max(lo, std::min(std::max<int64_t>(u, 1), hi));
+  };
+  auto count_at = [&](double c) -> int64_t {
+    int64_t sum = 0;
+    for (int32_t i = 0; i < n; ++i) {
+      const Seq& s = p->seqs[seq_ids[i]];
+      const int64_t n8 = static_cast<int64_t>(s.fp8_pages.size()), n3 = s.n3;
+      if (n8 > 0) sum += units_at(c, n8 * b8, n8, kMinFp8PagesPerUnit);
+      if (n3 > 0) sum += units_at(c, n3 * b3, n3, kMinTq3PagesPerUnit);
+    }
+    return sum;
+  };
+  // smallest unit cost whose cut needs at most U units (the largest unit bounds the wave)
+  double lo_c = std::max(1.0, static_cast<double>(total) / U), hi_c = lo_c;
+  while (count_at(hi_c) > U && hi_c < 4.0 * total) hi_c *= 2.0;
+  for (int it = 0; it < 40 && hi_c - lo_c > 0.5; ++it) {
+    const double mid = 0.5 * (lo_c + hi_c);
+    (count_at(mid) <= U ? hi_c : lo_c) = mid;
+  }
+  const double unit_cost = hi_c;
+  int64_t nu = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    const Seq& s = p->seqs[seq_ids[i]];
+    int32_t np = 0;
+    const auto& f8 = s.fp8_pages;
+    const int64_t n8 = static_cast<int64_t>(f8.size());
+    if (n8 > 0) {
+      const int64_t u = units_at(unit_cost, n8 * b8, n8, kMinFp8PagesPerUnit);
+      for (int64_t k = 0; k < u; ++k) {
+        const int64_t j0 = k * n8 / u, j1 = (k + 1) * n8 / u;
+        if (j1 <= j0) continue;
+        if (!emit(UnitDesc{f8[j0], f8[j1 - 1] + 1, static_cast<int16_t>(i), 0, np++}, (j1 - j0) * b8))
+          return -1;
+        ++nu;
+      }
+    }
+    const int64_t n3 = s.n3;
+    if (n3 > 0) {
+      const int64_t u = units_at(unit_cost, n3 * b3, n3, kMinTq3PagesPerUnit);
+      // unit k takes TQ3 pages number [k n3 / u, (k+1) n3 / u) in logical order; its range
+      // starts at the logical page of its first TQ3 page (the first unit at page 0) and ends
+      // where the next one starts (the last at the end of the table)
+      const int32_t pages = static_cast<int32_t>(s.table.size());
+      int32_t start = 0;
+      int64_t seen = 0, k = 0, next = (k + 1) * n3 / u;
+      for (int32_t lp = 0; lp < pages && k < u; ++lp) {
+        const int32_t e = s.table[lp];
+        if (e < 0 || fmt_of(e) != 1) continue;
+        if (seen == next) {  // lp is the first TQ3 page of unit k + 1
+          const int64_t cnt = next - k * n3 / u;
+          if (cnt > 0) {
+            if (!emit(UnitDesc{start, lp, static_cast<int16_t>(i), 1, np++}, cnt * b3)) return -1;
+            ++nu;
+          }
+          start = lp;
+          ++k;
+          next = (k + 1) * n3 / u;
+        }
+        ++seen;
+      }
+      const int64_t cnt = n3 - k * n3 / u;
+      if (cnt > 0) {
+        if (!emit(UnitDesc{start, pages, static_cast<int16_t>(i), 1, np++}, cnt * b3)) return -1;
+        ++nu;
+      }
+    }
+    n_parts[i] = np;
+  }
+  return nu;
+}
+
 int plan_decode(mkv_pool_t p, const int32_t* seq_ids, int32_t n, int32_t q_len, int32_t Hq,
                 DecodePlan* plan) {
   if (n < 0 || (n > 0 && !seq_ids)) return fail(MKV_ERR_INVALID_ARG, "bad sequence list");
@@ -180,49 +285,31 @@ int plan_decode(mkv_pool_t p, const int32_t* seq_ids, int32_t n, int32_t q_len, 
   plan->NC = q_len * plan->g;
   if (!partial_supported(D, plan->NC))
     return fail(MKV_ERR_UNSUPPORTED, "q_len * num_q_heads / Hkv = %d > 32 is not built", plan->NC);
-  const int64_t b8 = fp8_head_bytes(D), b3 = tq3_head_bytes(D);
-  int64_t total = 0;
   for (int32_t i = 0; i < n; ++i) {
     if (int e = check_seq(p, seq_ids[i])) return e;
     const Seq& s = p->seqs[seq_ids[i]];
     if (s.ctx < q_len || s.ctx == 0)
       return fail(MKV_ERR_EMPTY_CONTEXT, "sequence %d has %d tokens < q_len %d", seq_ids[i], s.ctx, q_len);
-    total += static_cast<int64_t>(s.fp8_pages.size()) * b8 + static_cast<int64_t>(s.n3) * b3;
   }
-  const int64_t target_ctas = static_cast<int64_t>(p->sm_count) * 3 * 3;
-  const int64_t per_cta = std::max<int64_t>(1, total * Hkv / target_ctas);
-  const int32_t R3 = static_cast<int32_t>(std::max<int64_t>(8, std::min<int64_t>(kMaxPagesPerUnit, per_cta / b3)));
-  const int32_t P8 = static_cast<int32_t>(std::max<int64_t>(4, std::min<int64_t>(kMaxPagesPerUnit, per_cta / b8)));
   plan->seq.resize(n);
   plan->unit.clear();
   plan->cost.clear();
+  std::vector<int32_t> np(n);
+  cut_units(p, seq_ids, n, plan->NC, np.data(), [&](const UnitDesc& u, int64_t cost) {
+    plan->unit.push_back(u);
+    plan->cost.push_back(cost);
+    return true;
+  });
   int64_t parts = 0;
   for (int32_t i = 0; i < n; ++i) {
-    const Seq& s = p->seqs[seq_ids[i]];
     SeqDesc& d = plan->seq[i];
     d.row = seq_ids[i];
-    d.ctx = s.ctx;
+    d.ctx = p->seqs[seq_ids[i]].ctx;
     d.out_row = i;
     d.part0 = static_cast<int32_t>(parts);
+    d.n_parts = np[i];
     d.pad = 0;
-    int32_t np = 0;
-    const auto& f8 = s.fp8_pages;
-    for (size_t j = 0; j < f8.size(); j += P8) {
-      const size_t k = std::min(f8.size(), j + static_cast<size_t>(P8));
-      plan->unit.push_back({f8[j], f8[k - 1] + 1, static_cast<int16_t>(i), 0, np++});
-      plan->cost.push_back(static_cast<int64_t>(k - j) * b8);
-    }
-    const int32_t pages = static_cast<int32_t>(s.table.size());
-    for (int32_t a = 0; a < pages; a += R3) {
-      const int32_t b = std::min(pages, a + R3);
-      const int64_t in8 = std::lower_bound(f8.begin(), f8.end(), b) - std::lower_bound(f8.begin(), f8.end(), a);
-      const int64_t in3 = (b - a) - in8;
-      if (in3 <= 0) continue;
-      plan->unit.push_back({a, b, static_cast<int16_t>(i), 1, np++});
-      plan->cost.push_back(in3 * b3);
-    }
-    d.n_parts = np;
-    parts += np;
+    parts += np[i];
   }
   if (parts > INT32_MAX / 2) return fail(MKV_ERR_INVALID_ARG, "call too large");
   plan->parts = parts;
@@ -621,53 +708,36 @@ int mkv_decode_attention_noalloc(mkv_pool_t p, const int32_t* seq_ids, int32_t n
   const int32_t g = Hq / Hkv, NC = q_len * g;
   if (!partial_supported(D, NC))
     return fail(MKV_ERR_UNSUPPORTED, "q_len * num_q_heads / Hkv = %d > 32 is not built", NC);
-  const int64_t b8 = fp8_head_bytes(D), b3 = tq3_head_bytes(D);
-  int64_t total = 0;
   for (int32_t i = 0; i < n_seqs; ++i) {
     if (int e = check_seq(p, seq_ids[i])) return e;
     const Seq& s = p->seqs[seq_ids[i]];
     if (s.ctx < q_len || s.ctx == 0)
       return fail(MKV_ERR_EMPTY_CONTEXT, "sequence %d has %d tokens < q_len %d", seq_ids[i], s.ctx, q_len);
-    total += static_cast<int64_t>(s.fp8_pages.size()) * b8 + static_cast<int64_t>(s.n3) * b3;
   }
   if (n_seqs == 0) return ok();
   if (!q_bf16 || !out) return fail(MKV_ERR_INVALID_ARG, "q/out is NULL");
-  // the same unit cut as plan_decode
-  const int64_t target_ctas = static_cast<int64_t>(p->sm_count) * 3 * 3;
-  const int64_t per_cta = std::max<int64_t>(1, total * Hkv / target_ctas);
-  const int32_t R3 = static_cast<int32_t>(std::max<int64_t>(8, std::min<int64_t>(kMaxPagesPerUnit, per_cta / b3)));
-  const int32_t P8 = static_cast<int32_t>(std::max<int64_t>(4, std::min<int64_t>(kMaxPagesPerUnit, per_cta / b8)));
   NoAllocPlan t;  // about 75 KB of stack
   DecodeParams& prm = t.prm;
-  int32_t nu = 0, parts = 0;
+  int32_t np[kDecodeMaxSeqs];
+  int32_t nu = 0;
+  const int64_t cut = cut_units(p, seq_ids, n_seqs, NC, np, [&](const UnitDesc& u, int64_t cost) {
+    if (nu >= kDecodeMaxUnits) return false;
+    t.unit[nu] = u;
+    t.cost[nu++] = cost;
+    return true;
+  });
+  if (cut < 0)
+    return fail(MKV_ERR_UNSUPPORTED, "the no-allocation decode takes at most %d work units per call", kDecodeMaxUnits);
+  int32_t parts = 0;
   for (int32_t i = 0; i < n_seqs; ++i) {
-    const Seq& s = p->seqs[seq_ids[i]];
     SeqDesc& d = prm.seq[i];
     d.row = seq_ids[i];
-    d.ctx = s.ctx;
+    d.ctx = p->seqs[seq_ids[i]].ctx;
     d.out_row = i;
     d.part0 = parts;
+    d.n_parts = np[i];
     d.pad = 0;
-    int32_t np = 0;
-    const auto& f8 = s.fp8_pages;
-    const int32_t pages = static_cast<int32_t>(s.table.size());
-    const int64_t need = static_cast<int64_t>((f8.size() + P8 - 1) / P8) + (pages + R3 - 1) / R3;
-    if (nu + need > kDecodeMaxUnits)
-      return fail(MKV_ERR_UNSUPPORTED, "the no-allocation decode takes at most %d work units per call", kDecodeMaxUnits);
-    for (size_t j = 0; j < f8.size(); j += P8) {
-      const size_t k = std::min(f8.size(), j + static_cast<size_t>(P8));
-      t.unit[nu] = {f8[j], f8[k - 1] + 1, static_cast<int16_t>(i), 0, np++};
-      t.cost[nu++] = static_cast<int64_t>(k - j) * b8;
-    }
-    for (int32_t a = 0; a < pages; a += R3) {
-      const int32_t b = std::min(pages, a + R3);
-      const int64_t in8 = std::lower_bound(f8.begin(), f8.end(), b) - std::lower_bound(f8.begin(), f8.end(), a);
-      if ((b - a) - in8 <= 0) continue;
-      t.unit[nu] = {a, b, static_cast<int16_t>(i), 1, np++};
-      t.cost[nu++] = ((b - a) - in8) * b3;
-    }
-    d.n_parts = np;
-    parts += np;
+    parts += np[i];
   }
   const size_t cols = static_cast<size_t>(parts) * Hkv * NC;
   const size_t off_acc = align256(cols * 2 * 4);

@@ -53,8 +53,10 @@ def test_noalloc_matches_workspace_decode_twice():
 
 
 def test_noalloc_rejects_calls_beyond_the_static_scratch():
-    Hkv, D, B, L = 8, 256, 8, 16384
-    pool = Pool(Hkv, D, B, L // 16 + 1, L // 16 + 64, B * (L // 16) + 8)
+    # many short sequences: at least two partial states each (FP8 page 0 and the TQ3 rest), so
+    # the call needs more than the 32 MiB static scratch whatever the unit cut
+    Hkv, D, B, L = 8, 256, 80, 512
+    pool = Pool(Hkv, D, B, L // 16 + 1, L // 16 + B + 64, B * (L // 16) + 8)
     z = torch.zeros((L, Hkv, D), dtype=torch.bfloat16, device="cuda")
     for s in range(B):
         pool.append([s], [L], z, z)
