@@ -37,8 +37,8 @@ FALLBACK_HBM_GBS = 6650.0
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the partial-attention kernel, from
 # the ncu capture summarised in profiles/, keyed by the hash of the kernel sources it measured.
 NCU_TRAFFIC = {
-    # profiles/decode_kernel_long_ctx128k_1layer.md: 494,559,744 B read + 9,681,408 B written
-    "b9ec8f134d6dc117": 504241152,
+    # profiles/decode_kernel_long_ctx128k_1layer.md: 494,523,392 B read + 3,909,120 B written
+    "071b028e215214ab": 498432512,
 }
 
 
