@@ -433,6 +433,123 @@ def run_reference(args, rank, world):
     }
 
 
+# ---------------------------------------------------------------------------- extra studies
+# Measurements beyond the headline line, one JSON line per point (not part of the driver's
+# contract): --mode sweep (FP8 page share from page 0 + window only up to all pages FP8, on one
+# layer of the long-context workload), --mode canary (two 59,008-token sequences at the long
+# workload's head shape, mixed cache against an all-FP8 control: decode time and KV bytes per
+# token), --mode pack (bulk FP8 -> TQ3 demotion of an all-FP8 pool shaped like the batch-8
+# workload, in GB/s).
+def _bf16_tensor(bits, device):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def _time_decode(pool, w, device, reps=20, warm=3):
+    """Partial and merge time (µs) and algorithmic bytes of one decode call over all sequences
+    of one layer, averaged over `reps` calls after `warm` untimed ones."""
+    import torch
+    seqs = list(range(w.B))
+    q = _bf16_tensor(np.stack([w.q(s) for s in seqs]), device)
+    out = torch.empty((w.B, w.q_len, w.Hq, w.D), dtype=torch.float32, device=device)
+    ws = torch.empty(pool.workspace_bytes(seqs, w.q_len, w.Hq) + (1 << 20), dtype=torch.uint8,
+                     device=device)
+    for _ in range(warm):
+        pool.decode(seqs, q, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    pool.timing(True)
+    pool.timing_read()
+    for _ in range(reps):
+        pool.decode(seqs, q, out=out, workspace=ws)
+    tm = pool.timing_read()
+    pool.timing(False)
+    pool.device_status()
+    tabs, ctxs = zip(*(pool.block_table(s) for s in seqs))
+    total, partial = decode_bytes(tabs, ctxs, w.Hkv, w.D, w.Hq, w.q_len)
+    n8 = sum(1 for t in tabs for e in t if (e >> 30) == 0)
+    return dict(partial_us=1000 * tm["partial_ms"] / tm["calls"],
+                merge_us=1000 * tm["merge_ms"] / tm["calls"], bytes=partial,
+                fp8_page_share=n8 / sum(len(t) for t in tabs), out=out)
+
+
+def run_extra(args):
+    import torch
+    from mixed_format_paged_mkv_b200 import Pool
+    from mixed_format_paged_mkv_b200.workloads import WORKLOADS
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    peak, peak_src = hbm_peak()
+    lines = []
+    if args.mode == "sweep":
+        for frac in (0.0, 0.04, 0.25, 0.5, 1.0):
+            w = WORKLOADS[4].scaled(fp8_page_frac=frac, layers=1)
+            pool = build_pool(w, 1, 3, device)
+            r = _time_decode(pool, w, device)
+            gbs = r["bytes"] / (r["partial_us"] * 1e-6) / 1e9
+            lines.append(dict(mode="sweep", workload=w.name, fp8_page_share=round(r["fp8_page_share"], 4),
+                              partial_us=round(r["partial_us"], 2), merge_us=round(r["merge_us"], 2),
+                              bytes_per_call=int(r["bytes"]), gbs=round(gbs, 1),
+                              frac=round(gbs / peak, 4), peak_source=peak_src,
+                              kv_bytes_per_token=round(pool.stats()[3], 1)))
+            del pool
+            torch.cuda.empty_cache()
+    elif args.mode == "canary":
+        res = {}
+        for name, frac in (("mixed", 0.0), ("fp8_control", 1.0)):
+            w = WORKLOADS[4].scaled(B=2, ctx=(59008, 59008), fp8_page_frac=frac, layers=1)
+            pool = build_pool(w, 1, 3, device)
+            r = _time_decode(pool, w, device)
+            res[name] = dict(r, bpt=pool.stats()[3])
+            del pool
+            torch.cuda.empty_cache()
+        m, c = res["mixed"], res["fp8_control"]
+        diff = (m["out"] - c["out"]).abs().max().item()
+        tm, tc = m["partial_us"] + m["merge_us"], c["partial_us"] + c["merge_us"]
+        lines.append(dict(mode="canary", sequences=2, context=59008, q_heads=24, kv_heads=4, head_dim=256,
+                          mixed_us=round(tm, 2), control_us=round(tc, 2),
+                          throughput_vs_control=round(tc / tm, 4),
+                          kv_bytes_per_token_mixed=round(m["bpt"], 1),
+                          kv_bytes_per_token_control=round(c["bpt"], 1),
+                          active_kv_ratio=round(c["bpt"] / m["bpt"], 4),
+                          fp8_page_share_mixed=round(m["fp8_page_share"], 4),
+                          max_abs_output_difference=diff))
+    elif args.mode == "pack":
+        w = WORKLOADS[2]
+        pages = w.pages()
+        n = sum(pages)
+        pool = Pool(w.Hkv, w.D, 2 * w.B, max(pages) + 2, 2 * n + 64, n + 64, device=device)
+        for s in range(w.B):  # templates: every page FP8
+            k, v = w.kv(s, 0)
+            pool.append([s], [w.lengths()[s]], _bf16_tensor(k, device), _bf16_tensor(v, device))
+        torch.cuda.synchronize()
+        work = list(range(w.B, 2 * w.B))
+        stream = torch.cuda.current_stream()
+        times, demoted = [], 0
+        for rep in range(8):
+            for s in range(w.B):
+                pool.copy(s, w.B + s)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            demoted = pool.demote(work, w.window)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if rep >= 2:
+                times.append(e0.elapsed_time(e1))
+            for s in work:
+                pool.reset(s)
+        pool.device_status()
+        per_page = w.Hkv * ((32 * w.D + 8) + 14 * w.D)
+        ms = statistics.median(times)
+        gbs = demoted * per_page / (ms * 1e-3) / 1e9
+        lines.append(dict(mode="pack", workload=w.name, pages_demoted=demoted, bytes=demoted * per_page,
+                          ms=round(ms, 4), gbs=round(gbs, 1), frac=round(gbs / peak, 4),
+                          peak_source=peak_src,
+                          note="one mkv_demote_pages call, host planning included in the span"))
+    for l in lines:
+        print(json.dumps(l), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -443,7 +560,12 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--mode", choices=["bench", "sweep", "canary", "pack"], default="bench",
+                    help="extra studies on one GPU (one JSON line per point); default: the bench")
     args = ap.parse_args()
+    if args.mode != "bench":
+        run_extra(args)
+        return
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -213,6 +213,17 @@ MKV_API int mkv_slot_bytes(mkv_pool_t pool, int32_t fmt, size_t* bytes);
 MKV_API int mkv_read_slot(mkv_pool_t pool, int32_t entry, void* host_out, size_t cap,
                           void* stream);
 
+/* Materialising profile (pt page, section "Qualidade em contexto longo": the profile in which
+ * the hybrid pages really are expanded into tensors).  A debugging and quality-control path,
+ * never part of decode: writes the sequence's dequantised K and V as dense fp32
+ * [ctx][Hkv][D] rows into the caller's device buffers k_out and v_out (each at least
+ * ctx * Hkv * D floats; max_tokens states their capacity in tokens).  FP8 values are
+ * fp32(dec(code) * page scale) (the fp32 product, rounded to nearest even); TQ3 values are
+ * (q - 3.5) * s (exact).  Asynchronous on the stream.  Errors: BAD_SEQ, INVALID_ARG (NULL
+ * output, capacity below the context), CUDA; a bad table entry is a device check. */
+MKV_API int mkv_materialise_kv(mkv_pool_t pool, int32_t seq, float* k_out, float* v_out,
+                               int64_t max_tokens, void* stream);
+
 /* Footprint (section "Memória e compressão"): live tokens, pages per format and KV slab bytes
  * held by live pages per live token. */
 MKV_API int mkv_pool_stats(mkv_pool_t pool, int64_t* live_tokens, int32_t* fp8_pages,

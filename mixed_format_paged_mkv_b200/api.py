@@ -52,6 +52,7 @@ SIGNATURES = {
                                                     ctypes.c_float, _P, _P]),
     "mkv_seq_reset": (ctypes.c_int, [_P, _I32, _P]),
     "mkv_seq_copy": (ctypes.c_int, [_P, _I32, _I32, _P]),
+    "mkv_materialise_kv": (ctypes.c_int, [_P, _I32, _P, _P, ctypes.c_int64, _P]),
     "mkv_get_block_table": (ctypes.c_int, [_P, _I32, _I32P, _I32, _I32P, _I32P]),
     "mkv_slot_bytes": (ctypes.c_int, [_P, _I32, _SZP]),
     "mkv_read_slot": (ctypes.c_int, [_P, _I32, _P, ctypes.c_size_t, _P]),
@@ -226,6 +227,22 @@ class Pool:
     def copy(self, src, dst, stream=None):
         st = None if self.host_only else _stream_ptr(stream)
         _check(lib().mkv_seq_copy(self.handle, src, dst, st), "mkv_seq_copy")
+
+    def materialise(self, seq, k_out=None, v_out=None, stream=None):
+        """Dense fp32 dequantised K and V of a sequence, [ctx, Hkv, D] each (a debugging and
+        quality-control path; decode never uses it)."""
+        import torch
+        _, ctx = self.block_table(seq)
+        dev = self.buffers[0].device if self.buffers else torch.device("cuda")
+        shape = (ctx, self.Hkv, self.D)
+        k_out = torch.empty(shape, dtype=torch.float32, device=dev) if k_out is None else k_out
+        v_out = torch.empty(shape, dtype=torch.float32, device=dev) if v_out is None else v_out
+        kp = _dev_ptr(k_out, torch.float32, "k_out")
+        vp = _dev_ptr(v_out, torch.float32, "v_out")
+        cap = min(k_out.numel(), v_out.numel()) // (self.Hkv * self.D)
+        _check(lib().mkv_materialise_kv(self.handle, seq, kp, vp, cap, _stream_ptr(stream)),
+               "mkv_materialise_kv")
+        return k_out, v_out
 
     def block_table(self, seq):
         n = ctypes.c_int32()

@@ -141,7 +141,52 @@ __global__ void __launch_bounds__(256) copy_kernel(const __grid_constant__ CopyP
         static_cast<int32_t>((static_cast<uint32_t>(d.fmt) << kFmtShift) | static_cast<uint32_t>(d.dst_slot));
 }
 
+// Materialising profile ("Minima-KV ..." pt page, section "Qualidade em contexto longo": the
+// profile in which the hybrid pages really are expanded into tensors).  A debugging and
+// quality-control path: one CTA per (page, KV head, K/V) writes the page's dequantised values
+// as dense fp32 rows -- FP8: fp32(dec(code) * scale); TQ3: (q - 3.5) * s, exact.  Decode never
+// calls it.
+__global__ void __launch_bounds__(256) materialise_kernel(const __grid_constant__ MaterialiseParams p) {
+  const int page = blockIdx.x, h = blockIdx.y, kv = blockIdx.z;
+  const int D = p.D, n = min(kPageTokens, p.ctx - kPageTokens * page);
+  const int32_t e = p.table[page];
+  const int fmt = static_cast<int>(static_cast<uint32_t>(e) >> kFmtShift);
+  const int64_t slot = static_cast<int64_t>(static_cast<uint32_t>(e) & kSlotMask);
+  if (e < 0 || fmt > 1 || slot >= (fmt == 0 ? p.fp8_slots : p.tq3_slots)) {
+    if (threadIdx.x == 0) flag_status(p.status, kStatusCheck);
+    return;
+  }
+  float* out = (kv ? p.v_out : p.k_out) + (static_cast<int64_t>(kPageTokens) * page * p.Hkv + h) * D;
+  const int64_t row_stride = static_cast<int64_t>(p.Hkv) * D;
+  if (fmt == 0) {
+    const uint8_t* base = p.fp8_slab + slot * p.fp8_slot_bytes + h * (32LL * D + 16);
+    const uint8_t* codes = base + kv * kPageTokens * D;
+    const float scale = reinterpret_cast<const float*>(base + 2 * kPageTokens * D)[kv];
+    for (int i = threadIdx.x; i < n * D; i += blockDim.x)
+      out[(i / D) * row_stride + i % D] = e4m3_to_float(codes[i]) * scale;
+  } else {
+    const int G = D / 32;
+    const uint8_t* base = p.tq3_slab + slot * p.tq3_slot_bytes + h * (14LL * D) + kv * (7LL * D);
+    const __half* scales = reinterpret_cast<const __half*>(base + G * kPageTokens * 12);
+    for (int i = threadIdx.x; i < n * D; i += blockDim.x) {
+      const int t = i / D, d = i % D, g = d / 32, j = d % 32;
+      const uint8_t* rec = base + 12 * (kPageTokens * g + t);
+      const int bit = 3 * j;  // LSB-first stream bit of code j
+      const uint32_t two = rec[bit >> 3] | (static_cast<uint32_t>(rec[min((bit >> 3) + 1, 11)]) << 8);
+      const float q = static_cast<float>((two >> (bit & 7)) & 7u);
+      out[t * row_stride + d] = (q - 3.5f) * __half2float(scales[kPageTokens * g + t]);
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_materialise(const MaterialiseParams& p, cudaStream_t s) {
+  if (p.ctx <= 0) return cudaSuccess;
+  const int pages = (p.ctx + kPageTokens - 1) / kPageTokens;
+  materialise_kernel<<<dim3(pages, p.Hkv, 2), 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
   if (p.n_desc <= 0) return cudaSuccess;

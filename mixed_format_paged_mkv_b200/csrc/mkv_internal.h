@@ -74,6 +74,19 @@ struct CopyParams {
   CopyDesc desc[kCopyMaxDesc];
 };
 
+// ------------------------------------------------------------------ materialise (debug / QC)
+// Dense fp32 copy of one sequence's dequantised K and V; never used by decode.
+struct MaterialiseParams {
+  const uint8_t* fp8_slab;
+  const uint8_t* tq3_slab;
+  const int32_t* table;  // the sequence's block-table row
+  int32_t* status;
+  float* k_out;  // [ctx][Hkv][D]
+  float* v_out;
+  int64_t fp8_slot_bytes, tq3_slot_bytes;
+  int32_t Hkv, D, ctx, fp8_slots, tq3_slots;
+};
+
 // ------------------------------------------------------------------ decode
 // Decode = partial kernel + merge kernel.  Work unit = (sequence, format, logical page range);
 // a partial CTA takes one (unit, KV head): it scans the block-table entries of its range,
@@ -120,6 +133,7 @@ struct DecodeParams {
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 cudaError_t launch_demote(const DemoteParams& p, cudaStream_t s);
 cudaError_t launch_copy(const CopyParams& p, cudaStream_t s);
+cudaError_t launch_materialise(const MaterialiseParams& p, cudaStream_t s);
 cudaError_t launch_partial(const DecodeParams& p, cudaStream_t s);
 cudaError_t launch_merge(const DecodeParams& p, cudaStream_t s);
 bool partial_supported(int D, int NC);

@@ -800,6 +800,37 @@ int mkv_seq_reset(mkv_pool_t p, int32_t seq, void* stream) {
   return ok();
 }
 
+int mkv_materialise_kv(mkv_pool_t p, int32_t seq, float* k_out, float* v_out,
+                       int64_t max_tokens, void* stream) {
+  if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
+  if (p->host_only) return fail(MKV_ERR_INVALID_ARG, "host-only pool has no device pages");
+  if (int e = check_seq(p, seq)) return e;
+  const Seq& s = p->seqs[seq];
+  if (s.ctx == 0) return ok();
+  if (!k_out || !v_out) return fail(MKV_ERR_INVALID_ARG, "output is NULL");
+  if (max_tokens < s.ctx)
+    return fail(MKV_ERR_INVALID_ARG, "outputs hold %lld tokens < context %d",
+                static_cast<long long>(max_tokens), s.ctx);
+  MaterialiseParams prm{};
+  prm.fp8_slab = p->fp8_slab;
+  prm.tq3_slab = p->tq3_slab;
+  prm.table = p->d_tables + static_cast<int64_t>(seq) * p->cfg.max_pages_per_seq;
+  prm.status = p->d_status;
+  prm.k_out = k_out;
+  prm.v_out = v_out;
+  prm.fp8_slot_bytes = p->fp8_slot_bytes;
+  prm.tq3_slot_bytes = p->tq3_slot_bytes;
+  prm.Hkv = p->cfg.num_kv_heads;
+  prm.D = p->cfg.head_dim;
+  prm.ctx = s.ctx;
+  prm.fp8_slots = p->cfg.fp8_slots;
+  prm.tq3_slots = p->cfg.tq3_slots;
+  cudaError_t e = launch_materialise(prm, as_stream(stream));
+  ++p->launches;
+  if (e != cudaSuccess) return cuda_fail(e, "materialise launch");
+  return ok();
+}
+
 int mkv_seq_copy(mkv_pool_t p, int32_t src, int32_t dst, void* stream) {
   if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
   if (int e = check_seq(p, src)) return e;
