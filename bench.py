@@ -38,7 +38,8 @@ FALLBACK_HBM_GBS = 6650.0
 # the ncu capture summarised in profiles/, keyed by the hash of the kernel sources it measured.
 NCU_TRAFFIC = {
     # profiles/decode_kernel_long_ctx128k_1layer.md: 494,523,392 B read + 3,909,120 B written
-    "071b028e215214ab": 498432512,
+    # (re-keyed after mkv_internal.h gained the materialise parameters; decode code unchanged)
+    "e2d4b1461b2c1aa8": 498432512,
 }
 
 
