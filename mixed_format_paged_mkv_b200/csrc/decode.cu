@@ -57,8 +57,8 @@ struct Cfg {
   static_assert(FP8_NST % PW == 0 && TQ3_NST % PW == 0, "stage ownership");
   static constexpr int RING_FP8 = FP8_NST * FP8_STAGE;
   static constexpr int RING_TQ3 = TQ3_NST * TQ3_STAGE;
-  // end-of-unit combine: (m, l) and acc of the consumer warps with pw > 0
-  static constexpr int COMBINE = (PW - 1) * NT * 8 * (D + 2) * 4;
+  // end-of-unit combine: (m, l) and acc of every consumer warp
+  static constexpr int COMBINE = PW * NT * 8 * (D + 2) * 4;
   static constexpr int RING = RING_FP8 > RING_TQ3 ? (RING_FP8 > COMBINE ? RING_FP8 : COMBINE)
                                                   : (RING_TQ3 > COMBINE ? RING_TQ3 : COMBINE);
   // header: full[16] | empty[16] mbarriers | stage tags | misc | page list | Q fragments |
@@ -414,18 +414,33 @@ __device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDes
   const int r = lane >> 2, c = lane & 3;
   const int nt = warp % NT, pw = warp / NT;
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < NST; ++s) {
-      mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], NT);
-    }
-    sm.misc[1] = 0;
-    mbar_fence_init();
-  }
+  const uint8_t* slab = FP8 ? p.fp8_slab : p.tq3_slab;
+  const int64_t slot_bytes = FP8 ? p.fp8_slot_bytes : p.tq3_slot_bytes;
   if (warp == C::PRODUCER) {
+    // the producer owns the ring set-up, so its first fills (which need no free stage) are in
+    // flight while the consumers build their Q fragments
+    if (lane == 0) {
+      for (int s = 0; s < NST; ++s) {
+        mbar_init(&sm.full[s], 1);
+        mbar_init(&sm.empty[s], NT);
+      }
+      sm.misc[1] = 0;
+      mbar_fence_init();
+    }
     const int32_t* row = p.tables + static_cast<int64_t>(sd.row) * p.max_pages;
     const int n = scan_range(p, row, u.first, u.last, FP8 ? 0 : 1, lane, sm.list);
-    if (lane == 0) sm.misc[0] = n;
+    __syncwarp();
+    if (lane == 0) {
+      sm.misc[0] = n;
+      for (int i = 0; i < min(n, NST); ++i) {
+        const int2 e = sm.list[i];
+        sm.tag[i] = e.y;
+        mbar_arrive_expect_tx(&sm.full[i], STAGE);
+        bulk_g2s(sm.ring + i * STAGE,
+                 slab + static_cast<int64_t>(e.x) * slot_bytes + static_cast<int64_t>(h) * STAGE,
+                 STAGE, &sm.full[i]);
+      }
+    }
   } else if (pw == 0) {
     const float ls = build_q<D, FP8>(p, sd, h, nt, lane, sm.qf + nt * (D / 32) * 32,
                                      reinterpret_cast<float*>(sm.corr + nt * (D / 32) * 4));
@@ -441,10 +456,8 @@ __device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDes
   if (warp == C::PRODUCER) {
     // ---------------- producer: one lane streams the unit's pages into the ring
     if (lane == 0) {
-      const uint8_t* slab = FP8 ? p.fp8_slab : p.tq3_slab;
-      const int64_t slot_bytes = FP8 ? p.fp8_slot_bytes : p.tq3_slot_bytes;
-      int issued = 0;
-      for (int i = 0; i < count; ++i) {
+      int issued = min(count, NST);
+      for (int i = issued; i < count; ++i) {
         const int s = i % NST;
         if (i >= NST && !mbar_wait(&sm.empty[s], ((i / NST) - 1) & 1)) {
           flag_status(p.status, kStatusTimeout);
@@ -530,10 +543,12 @@ __device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDes
   }
   __syncthreads();  // ring no longer needed: reuse it for the cross-warp combine
 
+  // every page-parallel warp stores its state; then all of them combine a share of the
+  // columns' channels: M = max m, l = sum l 2^(m-M), acc = sum acc 2^(m-M)
   float* cmb = reinterpret_cast<float*>(sm.ring);
-  constexpr int REGION = 8 * (D + 2);
-  if (warp < C::NWC && pw > 0) {
-    float* reg = cmb + ((pw - 1) * NT + nt) * REGION;
+  constexpr int REGION = 8 * (D + 2);  // per (warp, n-tile): (m, l) of 8 columns, then acc [8][D]
+  if (warp < C::NWC) {
+    float* reg = cmb + (pw * NT + nt) * REGION;
     if (r == 0) {
       reg[2 * (2 * c)] = ks.m[0];
       reg[2 * (2 * c) + 1] = ks.l[0];
@@ -551,46 +566,39 @@ __device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDes
     }
   }
   __syncthreads();
-  if (warp < C::NWC && pw == 0) {
-    float m[2] = {ks.m[0], ks.m[1]}, l[2] = {ks.l[0], ks.l[1]};
-    for (int o = 1; o < C::PW; ++o) {
-      const float* reg = cmb + ((o - 1) * NT + nt) * REGION;
-      const float* ra = reg + 16;
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const int col = 2 * c + k;
-        const float mo = reg[2 * col], lo = reg[2 * col + 1];
-        const float M = fmaxf(m[k], mo);
-        if (M == -INFINITY) continue;
-        const float as = m[k] == -INFINITY ? 0.f : exp2f(m[k] - M);
-        const float ao = mo == -INFINITY ? 0.f : exp2f(mo - M);
-        l[k] = l[k] * as + lo * ao;
-#pragma unroll
-        for (int mt = 0; mt < D / 16; ++mt) {
-          const int ch = 32 * (mt >> 1) + 4 * r + 2 * (mt & 1);
-          vs.acc[mt][k] = vs.acc[mt][k] * as + ra[col * D + ch] * ao;
-          vs.acc[mt][k + 2] = vs.acc[mt][k + 2] * as + ra[col * D + ch + 1] * ao;
-        }
-        m[k] = M;
-      }
-    }
+  if (warp < C::NWC) {
     const int part = sd.part0 + u.part;
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int n = 8 * nt + 2 * c + k;
+    const float* regs = cmb + nt * REGION;  // warp w's region: regs + w * NT * REGION
+    for (int q = pw * 32 + lane; q < 8 * (D / 4); q += 32 * C::PW) {
+      const int col = q / (D / 4), ch = 4 * (q % (D / 4));
+      const int n = 8 * nt + col;
       if (n >= p.NC) continue;
-      const int64_t base = (static_cast<int64_t>(part) * p.Hkv + h) * p.NC + n;
-      if (r == 0) {
-        p.part_ml[2 * base] = m[k];
-        p.part_ml[2 * base + 1] = l[k];
-      }
-      float* dst = p.part_acc + base * D;
+      float M = -INFINITY;
 #pragma unroll
-      for (int g = 0; g < D / 32; ++g) {
-        const float4 v = make_float4(vs.acc[2 * g][k], vs.acc[2 * g][k + 2],
-                                     vs.acc[2 * g + 1][k], vs.acc[2 * g + 1][k + 2]);
-        *reinterpret_cast<float4*>(dst + 32 * g + 4 * r) = v;
+      for (int w = 0; w < C::PW; ++w) M = fmaxf(M, regs[w * NT * REGION + 2 * col]);
+      float L = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int w = 0; w < C::PW; ++w) {
+          const float* rw = regs + w * NT * REGION;
+          const float mw = rw[2 * col];
+          if (mw == -INFINITY) continue;
+          const float a = exp2f(mw - M);
+          L += rw[2 * col + 1] * a;
+          const float4 v = *reinterpret_cast<const float4*>(rw + 16 + col * D + ch);
+          acc.x += a * v.x;
+          acc.y += a * v.y;
+          acc.z += a * v.z;
+          acc.w += a * v.w;
+        }
       }
+      const int64_t base = (static_cast<int64_t>(part) * p.Hkv + h) * p.NC + n;
+      if (ch == 0) {
+        p.part_ml[2 * base] = M;
+        p.part_ml[2 * base + 1] = L;
+      }
+      *reinterpret_cast<float4*>(p.part_acc + base * D + ch) = acc;
     }
   }
 }
