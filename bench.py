@@ -37,9 +37,8 @@ FALLBACK_HBM_GBS = 6650.0
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the partial-attention kernel, from
 # the ncu capture summarised in profiles/, keyed by the hash of the kernel sources it measured.
 NCU_TRAFFIC = {
-    # profiles/decode_kernel_long_ctx128k_1layer.md: 494,523,392 B read + 3,909,120 B written
-    # (re-keyed after mkv_internal.h gained the materialise parameters; decode code unchanged)
-    "e2d4b1461b2c1aa8": 498432512,
+    # profiles/decode_kernel_long_ctx128k_1layer.md: 494,519,552 B read + 4,348,928 B written
+    "be67ba50c62aa9f1": 498868480,
 }
 
 
@@ -440,7 +439,8 @@ def run_reference(args, rank, world):
 # layer of the long-context workload), --mode canary (two 59,008-token sequences at the long
 # workload's head shape, mixed cache against an all-FP8 control: decode time and KV bytes per
 # token), --mode pack (bulk FP8 -> TQ3 demotion of an all-FP8 pool shaped like the batch-8
-# workload, in GB/s).
+# workload, in GB/s), --mode prefill (direct bf16 -> TQ3 packing of that workload's prompts) and
+# --mode materialise (dense fp32 K and V of that workload's sequences).
 def _bf16_tensor(bits, device):
     import torch
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
@@ -547,6 +547,66 @@ def run_extra(args):
                           ms=round(ms, 4), gbs=round(gbs, 1), frac=round(gbs / peak, 4),
                           peak_source=peak_src,
                           note="one mkv_demote_pages call, host planning included in the span"))
+    elif args.mode == "prefill":
+        # direct bf16 -> TQ3 packing of the batch-8 workload's prompts (256-token window FP8)
+        w = WORKLOADS[2]
+        pages = w.pages()
+        n = sum(pages)
+        pool = Pool(w.Hkv, w.D, w.B, max(pages) + 2, n + 64, n + 64, device=device)
+        ks, vs = zip(*(w.kv(s, 0) for s in range(w.B)))
+        kd, vd = _bf16_tensor(np.concatenate(ks), device), _bf16_tensor(np.concatenate(vs), device)
+        seqs, lens = list(range(w.B)), w.lengths()
+        stream = torch.cuda.current_stream()
+        times = []
+        for rep in range(8):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            pool.prefill(seqs, lens, kd, vd, window=w.window)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if rep >= 2:
+                times.append(e0.elapsed_time(e1))
+            if rep < 7:
+                for s in seqs:
+                    pool.reset(s)
+        pool.device_status()
+        tabs = [pool.block_table(s)[0] for s in seqs]
+        n3 = sum(1 for t in tabs for e in t if (e >> 30) == 1)
+        n8 = sum(len(t) for t in tabs) - n3
+        rd = sum(lens) * w.Hkv * w.D * 2 * 2
+        wr = n3 * w.Hkv * 14 * w.D + n8 * w.Hkv * (32 * w.D + 16)
+        ms = statistics.median(times)
+        gbs = (rd + wr) / (ms * 1e-3) / 1e9
+        lines.append(dict(mode="prefill", workload=w.name, tokens=sum(lens), tq3_pages=n3, fp8_pages=n8,
+                          bytes=rd + wr, ms=round(ms, 4), gbs=round(gbs, 1), frac=round(gbs / peak, 4),
+                          peak_source=peak_src,
+                          note="one mkv_prefill_kv call (bf16 read, TQ3/FP8 pages written), host planning included"))
+    elif args.mode == "materialise":
+        w = WORKLOADS[2]
+        pool = build_pool(w, 1, 3, device)
+        L = max(w.lengths())
+        k = torch.empty((L, w.Hkv, w.D), dtype=torch.float32, device=device)
+        v = torch.empty_like(k)
+        stream = torch.cuda.current_stream()
+        for s in range(w.B):
+            pool.materialise(s, k, v)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for rep in range(4):
+            for s in range(w.B):
+                pool.materialise(s, k, v)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        pool.device_status()
+        tabs, ctxs = zip(*(pool.block_table(s) for s in range(w.B)))
+        kv_bytes = decode_bytes(tabs, ctxs, w.Hkv, w.D, 0, 0)[1]
+        out_bytes = sum(ctxs) * w.Hkv * w.D * 4 * 2
+        ms = e0.elapsed_time(e1) / 4
+        gbs = (kv_bytes + out_bytes) / (ms * 1e-3) / 1e9
+        lines.append(dict(mode="materialise", workload=w.name, tokens=sum(ctxs), bytes=int(kv_bytes + out_bytes),
+                          ms=round(ms, 4), gbs=round(gbs, 1), frac=round(gbs / peak, 4),
+                          peak_source=peak_src, note="mkv_materialise_kv of every sequence (dense fp32 K and V)"))
     for l in lines:
         print(json.dumps(l), flush=True)
 
@@ -561,7 +621,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--mode", choices=["bench", "sweep", "canary", "pack"], default="bench",
+    ap.add_argument("--mode", choices=["bench", "sweep", "canary", "pack", "prefill", "materialise"],
+                    default="bench",
                     help="extra studies on one GPU (one JSON line per point); default: the bench")
     args = ap.parse_args()
     if args.mode != "bench":

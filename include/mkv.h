@@ -213,6 +213,21 @@ MKV_API int mkv_slot_bytes(mkv_pool_t pool, int32_t fmt, size_t* bytes);
 MKV_API int mkv_read_slot(mkv_pool_t pool, int32_t entry, void* host_out, size_t cap,
                           void* stream);
 
+/* Prefill-time compression: write the first n_tokens[i] tokens of each listed sequence, which
+ * must be empty (k, v as for mkv_append_kv).  Every full page that the anchor policy would
+ * demote at once -- page p >= sink_pages with 16p + 16 <= n - anchor_window_tokens (new pages
+ * are not protected) -- is packed to TQ3 straight from the bf16 values, with the same
+ * per-group scale and thresholds as demotion (sections "Âncoras em FP8, arquivo em TQ3" /
+ * "Des ancres en FP8, une archive en TQ3" describe TQ3 as the archive format of older pages);
+ * every other page is written as a fresh FP8 page, as by mkv_append_kv.  Pages take slots of
+ * their own format, ascending, sequences in list order.  Values differ from append-then-demote
+ * only through the FP8 rounding that the direct path skips.  Errors: BAD_SEQ, INVALID_ARG
+ * (non-empty or repeated sequence, negative count or window, NULL k/v), OUT_OF_PAGES (nothing
+ * changed), CUDA. */
+MKV_API int mkv_prefill_kv(mkv_pool_t pool, const int32_t* seq_ids, const int32_t* n_tokens,
+                           int32_t n_seqs, const void* k_bf16, const void* v_bf16,
+                           int32_t anchor_window_tokens, void* stream);
+
 /* Materialising profile (pt page, section "Qualidade em contexto longo": the profile in which
  * the hybrid pages really are expanded into tensors).  A debugging and quality-control path,
  * never part of decode: writes the sequence's dequantised K and V as dense fp32

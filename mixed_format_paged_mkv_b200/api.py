@@ -53,6 +53,7 @@ SIGNATURES = {
     "mkv_seq_reset": (ctypes.c_int, [_P, _I32, _P]),
     "mkv_seq_copy": (ctypes.c_int, [_P, _I32, _I32, _P]),
     "mkv_materialise_kv": (ctypes.c_int, [_P, _I32, _P, _P, ctypes.c_int64, _P]),
+    "mkv_prefill_kv": (ctypes.c_int, [_P, _I32P, _I32P, _I32, _P, _P, _I32, _P]),
     "mkv_get_block_table": (ctypes.c_int, [_P, _I32, _I32P, _I32, _I32P, _I32P]),
     "mkv_slot_bytes": (ctypes.c_int, [_P, _I32, _SZP]),
     "mkv_read_slot": (ctypes.c_int, [_P, _I32, _P, ctypes.c_size_t, _P]),
@@ -180,6 +181,25 @@ class Pool:
                 raise ValueError(f"k, v must be [{rows}, {self.Hkv}, {self.D}]")
             st = _stream_ptr(stream)
         _check(lib().mkv_append_kv(self.handle, sp, np_, s.size, kp, vp, st), "mkv_append_kv")
+
+    def prefill(self, seq_ids, n_tokens, k=None, v=None, window=0, stream=None):
+        """First tokens of empty sequences; full pages the anchor policy would demote at once
+        are packed to TQ3 straight from bf16 (mkv_prefill_kv)."""
+        import torch
+        s, sp = _i32_array(seq_ids)
+        n, np_ = _i32_array(n_tokens)
+        if self.host_only:
+            kp = vp = None
+            st = None
+        else:
+            kp = _dev_ptr(k, torch.bfloat16, "k")
+            vp = _dev_ptr(v, torch.bfloat16, "v")
+            rows = int(n.sum())
+            if tuple(k.shape) != (rows, self.Hkv, self.D) or tuple(v.shape) != (rows, self.Hkv, self.D):
+                raise ValueError(f"k, v must be [{rows}, {self.Hkv}, {self.D}]")
+            st = _stream_ptr(stream)
+        _check(lib().mkv_prefill_kv(self.handle, sp, np_, s.size, kp, vp, int(window), st),
+               "mkv_prefill_kv")
 
     def set_protected(self, seq, page, flag=True):
         _check(lib().mkv_set_protected(self.handle, seq, page, 1 if flag else 0), "mkv_set_protected")

@@ -79,9 +79,38 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ App
   }
 }
 
+// TQ3 record of one (token, KV head, K-or-V, group of 32 channels), one channel per lane:
+// s = fp16(min(fp32(amax/3.5), 65504)); q = #{k in -3..3 : x >= k*s}; the 32 codes packed
+// LSB-first into the 12-byte record, the scale into the area's scale array.
+__device__ __forceinline__ void pack_group(float x, int lane, uint8_t* area, int G, int grp, int t) {
+  float amax = fabsf(x);
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const __half sh = __float2half_rn(fminf(__fdiv_rn(amax, 3.5f), 65504.f));
+  const float s = __half2float(sh);
+  uint32_t q = 0;
+#pragma unroll
+  for (int k = -3; k <= 3; ++k) q += (x >= __fmul_rn(static_cast<float>(k), s)) ? 1u : 0u;
+  // bit 3*lane + i of the 96-bit record holds bit i of q
+  const int bit = 3 * lane;
+  uint32_t w0 = 0, w1 = 0, w2 = 0;
+  if (bit < 32) w0 = q << bit;
+  if (bit + 2 >= 32 && bit < 64) w1 = (bit >= 32) ? (q << (bit - 32)) : (q >> (32 - bit));
+  if (bit + 2 >= 64) w2 = (bit >= 64) ? (q << (bit - 64)) : (q >> (64 - bit));
+  w0 = __reduce_or_sync(0xffffffffu, w0);
+  w1 = __reduce_or_sync(0xffffffffu, w1);
+  w2 = __reduce_or_sync(0xffffffffu, w2);
+  uint32_t* rec = reinterpret_cast<uint32_t*>(area + 12 * (grp * kPageTokens + t));
+  if (lane == 0) rec[0] = w0;
+  if (lane == 1) rec[1] = w1;
+  if (lane == 2) rec[2] = w2;
+  if (lane == 3) {
+    __half* sc = reinterpret_cast<__half*>(area + G * kPageTokens * 12);
+    sc[grp * kPageTokens + t] = sh;
+  }
+}
+
 // One block per (page, KV head); one warp per (K-or-V, group of 32 channels, token), lane =
-// channel.  x = fp32(dec(code) * page scale); s = fp16(min(fp32(amax/3.5), 65504));
-// q = #{k in -3..3 : x >= k*s}; 32 codes packed LSB-first into 12 bytes.
+// channel.  x = fp32(dec(code) * page scale), packed by pack_group.
 __global__ void __launch_bounds__(256) demote_kernel(const __grid_constant__ DemoteParams p) {
   const DemoteDesc d = p.desc[blockIdx.x];
   const int h = blockIdx.y, D = p.D, G = D / 32;
@@ -98,31 +127,29 @@ __global__ void __launch_bounds__(256) demote_kernel(const __grid_constant__ Dem
     const int t = u % kPageTokens;
     const uint8_t code = src[which * kPageTokens * D + t * D + grp * 32 + lane];
     const float x = __fmul_rn(e4m3_to_float(code), scales[which]);
-    float amax = fabsf(x);
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const __half sh = __float2half_rn(fminf(__fdiv_rn(amax, 3.5f), 65504.f));
-    const float s = __half2float(sh);
-    uint32_t q = 0;
-#pragma unroll
-    for (int k = -3; k <= 3; ++k) q += (x >= __fmul_rn(static_cast<float>(k), s)) ? 1u : 0u;
-    // bit 3*lane + i of the 96-bit record holds bit i of q
-    const int bit = 3 * lane;
-    uint32_t w0 = 0, w1 = 0, w2 = 0;
-    if (bit < 32) w0 = q << bit;
-    if (bit + 2 >= 32 && bit < 64) w1 = (bit >= 32) ? (q << (bit - 32)) : (q >> (32 - bit));
-    if (bit + 2 >= 64) w2 = (bit >= 64) ? (q << (bit - 64)) : (q >> (64 - bit));
-    w0 = __reduce_or_sync(0xffffffffu, w0);
-    w1 = __reduce_or_sync(0xffffffffu, w1);
-    w2 = __reduce_or_sync(0xffffffffu, w2);
-    uint8_t* area = dst + which * (G * kPageTokens * 14);
-    uint32_t* rec = reinterpret_cast<uint32_t*>(area + 12 * (grp * kPageTokens + t));
-    if (lane == 0) rec[0] = w0;
-    if (lane == 1) rec[1] = w1;
-    if (lane == 2) rec[2] = w2;
-    if (lane == 3) {
-      __half* sc = reinterpret_cast<__half*>(area + G * kPageTokens * 12);
-      sc[grp * kPageTokens + t] = sh;
-    }
+    pack_group(x, lane, dst + which * (G * kPageTokens * 14), G, grp, t);
+  }
+  if (h == 0 && threadIdx.x == 0)
+    p.tables[d.table_index] = static_cast<int32_t>((1u << kFmtShift) | static_cast<uint32_t>(d.dst_slot));
+}
+
+// Prefill: a full page packed to TQ3 straight from the bf16 input rows (the values are exact in
+// fp32), with the same per-group packing as demotion.  One block per (page, KV head).
+__global__ void __launch_bounds__(256) pack_kernel(const __grid_constant__ PackParams p) {
+  const PackDesc d = p.desc[blockIdx.x];
+  const int h = blockIdx.y, D = p.D, G = D / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* dst = p.tq3_slab + static_cast<int64_t>(d.dst_slot) * p.tq3_slot_bytes +
+                 static_cast<int64_t>(h) * (14 * D);
+  const int units = 2 * G * kPageTokens;
+  for (int u = warp; u < units; u += blockDim.x >> 5) {
+    const int which = u / (G * kPageTokens);
+    const int grp = (u / kPageTokens) % G;
+    const int t = u % kPageTokens;
+    const uint16_t* src = which ? p.v : p.k;
+    const float x = bf16_bits_to_float(
+        src[(static_cast<int64_t>(d.first_row + t) * p.Hkv + h) * D + grp * 32 + lane]);
+    pack_group(x, lane, dst + which * (G * kPageTokens * 14), G, grp, t);
   }
   if (h == 0 && threadIdx.x == 0)
     p.tables[d.table_index] = static_cast<int32_t>((1u << kFmtShift) | static_cast<uint32_t>(d.dst_slot));
@@ -180,6 +207,12 @@ __global__ void __launch_bounds__(256) materialise_kernel(const __grid_constant_
 }
 
 }  // namespace
+
+cudaError_t launch_pack(const PackParams& p, cudaStream_t s) {
+  if (p.n_desc <= 0) return cudaSuccess;
+  pack_kernel<<<dim3(p.n_desc, p.Hkv), 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_materialise(const MaterialiseParams& p, cudaStream_t s) {
   if (p.ctx <= 0) return cudaSuccess;

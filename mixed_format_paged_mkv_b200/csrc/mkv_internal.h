@@ -60,6 +60,24 @@ struct DemoteParams {
   DemoteDesc desc[kDemoteMaxDesc];
 };
 
+// ------------------------------------------------------------------ prefill (bf16 -> TQ3)
+struct PackDesc {
+  int32_t dst_slot;     // TQ3 slot
+  int32_t table_index;  // entry set to TQ3
+  int32_t first_row;    // input row of the page's first token
+};
+constexpr int kPackMaxDesc = 2560;
+struct PackParams {
+  const uint16_t* k;  // bf16 bits [rows][Hkv][D]
+  const uint16_t* v;
+  uint8_t* tq3_slab;
+  int32_t* tables;
+  int64_t tq3_slot_bytes;
+  int32_t Hkv, D;
+  int32_t n_desc;
+  PackDesc desc[kPackMaxDesc];
+};
+
 // ------------------------------------------------------------------ slot copy
 struct CopyDesc {
   int32_t src_slot, dst_slot, fmt, table_index;
@@ -134,6 +152,7 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 cudaError_t launch_demote(const DemoteParams& p, cudaStream_t s);
 cudaError_t launch_copy(const CopyParams& p, cudaStream_t s);
 cudaError_t launch_materialise(const MaterialiseParams& p, cudaStream_t s);
+cudaError_t launch_pack(const PackParams& p, cudaStream_t s);
 cudaError_t launch_partial(const DecodeParams& p, cudaStream_t s);
 cudaError_t launch_merge(const DecodeParams& p, cudaStream_t s);
 bool partial_supported(int D, int NC);

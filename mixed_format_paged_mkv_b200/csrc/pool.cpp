@@ -800,6 +800,116 @@ int mkv_seq_reset(mkv_pool_t p, int32_t seq, void* stream) {
   return ok();
 }
 
+int mkv_prefill_kv(mkv_pool_t p, const int32_t* seq_ids, const int32_t* n_tokens, int32_t n_seqs,
+                   const void* k_bf16, const void* v_bf16, int32_t anchor_window_tokens,
+                   void* stream) {
+  if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
+  if (n_seqs < 0 || (n_seqs > 0 && (!seq_ids || !n_tokens)))
+    return fail(MKV_ERR_INVALID_ARG, "bad sequence list");
+  if (anchor_window_tokens < 0) return fail(MKV_ERR_INVALID_ARG, "negative anchor window");
+  const int32_t MP = p->cfg.max_pages_per_seq, sink = p->cfg.sink_pages;
+  // page p of a prefill of n tokens is packed to TQ3 at once iff the anchor policy would demote
+  // it: p >= sink and 16p + 16 <= n - W (new pages carry no protection)
+  auto direct = [&](int64_t pg, int64_t n) {
+    return pg >= sink && kPageTokens * pg + kPageTokens <= n - anchor_window_tokens;
+  };
+  int64_t need[2] = {0, 0}, rows = 0;
+  std::vector<uint8_t> seen(p->cfg.max_seqs, 0);
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    if (int e = check_seq(p, seq_ids[i])) return e;
+    if (seen[seq_ids[i]]) return fail(MKV_ERR_INVALID_ARG, "sequence %d listed twice", seq_ids[i]);
+    seen[seq_ids[i]] = 1;
+    if (n_tokens[i] < 0) return fail(MKV_ERR_INVALID_ARG, "negative token count");
+    const Seq& s = p->seqs[seq_ids[i]];
+    if (s.ctx || !s.table.empty())
+      return fail(MKV_ERR_INVALID_ARG, "prefill needs an empty sequence (%d is not)", seq_ids[i]);
+    const int64_t pages = (static_cast<int64_t>(n_tokens[i]) + kPageTokens - 1) / kPageTokens;
+    if (pages > MP)
+      return fail(MKV_ERR_OUT_OF_PAGES, "sequence %d would need %lld pages > %d", seq_ids[i],
+                  static_cast<long long>(pages), MP);
+    for (int64_t pg = 0; pg < pages; ++pg) ++need[direct(pg, n_tokens[i]) ? 1 : 0];
+    rows += n_tokens[i];
+  }
+  for (int f = 0; f < 2; ++f)
+    if (need[f] > p->alloc[f].n_free)
+      return fail(MKV_ERR_OUT_OF_PAGES, "%s slab has %d free slots, %lld needed", f ? "TQ3" : "FP8",
+                  p->alloc[f].n_free, static_cast<long long>(need[f]));
+  if (rows > 0 && !p->host_only && (!k_bf16 || !v_bf16))
+    return fail(MKV_ERR_INVALID_ARG, "k/v are NULL");
+  if (rows > INT32_MAX) return fail(MKV_ERR_INVALID_ARG, "too many tokens");
+
+  // ---- commit host state: pages ascending, each taking a slot of its own format
+  std::vector<AppendDesc> fp8_descs;
+  std::vector<PackDesc> tq3_descs;
+  int32_t row = 0;
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    Seq& s = p->seqs[seq_ids[i]];
+    const int32_t n = n_tokens[i], pages = (n + kPageTokens - 1) / kPageTokens;
+    s.prot.assign(pages, 0);
+    for (int32_t pg = 0; pg < pages; ++pg) {
+      const int32_t first_row = row + kPageTokens * pg;
+      const int32_t table_index = seq_ids[i] * MP + pg;
+      if (direct(pg, n)) {
+        const int32_t slot = p->alloc[1].take();
+        s.table.push_back(entry_of(MKV_FMT_TQ3, slot));
+        ++s.n3;
+        tq3_descs.push_back({slot, table_index, first_row});
+      } else {
+        const int32_t slot = p->alloc[0].take();
+        s.fp8_pages.push_back(pg);
+        s.table.push_back(entry_of(MKV_FMT_FP8, slot));
+        AppendDesc d;
+        d.slot = slot;
+        d.table_index = table_index;
+        d.first_row = first_row;
+        d.n_old = 0;
+        d.n_new = static_cast<int16_t>(std::min(kPageTokens, n - kPageTokens * pg));
+        fp8_descs.push_back(d);
+      }
+    }
+    s.ctx = n;
+    row += n;
+  }
+  if (p->host_only) return ok();
+  cudaStream_t st = as_stream(stream);
+  AppendParams* ap = new AppendParams;
+  ap->fp8_slab = p->fp8_slab;
+  ap->tables = p->d_tables;
+  ap->status = p->d_status;
+  ap->k = static_cast<const uint16_t*>(k_bf16);
+  ap->v = static_cast<const uint16_t*>(v_bf16);
+  ap->slot_bytes = p->fp8_slot_bytes;
+  ap->Hkv = p->cfg.num_kv_heads;
+  ap->D = p->cfg.head_dim;
+  cudaError_t e = cudaSuccess;
+  for (size_t b = 0; b < fp8_descs.size() && e == cudaSuccess; b += kAppendMaxDesc) {
+    const size_t m = std::min<size_t>(kAppendMaxDesc, fp8_descs.size() - b);
+    ap->n_desc = static_cast<int32_t>(m);
+    std::memcpy(ap->desc, fp8_descs.data() + b, m * sizeof(AppendDesc));
+    e = launch_append(*ap, st);
+    ++p->launches;
+  }
+  delete ap;
+  PackParams* pp = new PackParams;
+  pp->k = static_cast<const uint16_t*>(k_bf16);
+  pp->v = static_cast<const uint16_t*>(v_bf16);
+  pp->tq3_slab = p->tq3_slab;
+  pp->tables = p->d_tables;
+  pp->tq3_slot_bytes = p->tq3_slot_bytes;
+  pp->Hkv = p->cfg.num_kv_heads;
+  pp->D = p->cfg.head_dim;
+  for (size_t b = 0; b < tq3_descs.size() && e == cudaSuccess; b += kPackMaxDesc) {
+    const size_t m = std::min<size_t>(kPackMaxDesc, tq3_descs.size() - b);
+    pp->n_desc = static_cast<int32_t>(m);
+    std::memcpy(pp->desc, tq3_descs.data() + b, m * sizeof(PackDesc));
+    e = launch_pack(*pp, st);
+    ++p->launches;
+  }
+  delete pp;
+  if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+  return ok();
+}
+
 int mkv_materialise_kv(mkv_pool_t p, int32_t seq, float* k_out, float* v_out,
                        int64_t max_tokens, void* stream) {
   if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");

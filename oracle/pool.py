@@ -143,6 +143,66 @@ class RefPool:
             self.ctx[s] = L0 + n
             row += n
 
+    # ------------------------------------------------------------------ prefill (direct pack)
+    def prefill(self, seq_ids, n_tokens, k, v, window_tokens):
+        """Write the first tokens of empty sequences: k, v float64 [sum(n_tokens), Hkv, D]
+        (bf16 values), rows grouped by sequence in ``seq_ids`` order.  A full page that the
+        anchor policy would demote at once (p >= sink_pages and 16p + 16 <= L - W, with L the
+        sequence's new length; new pages carry no protection) is packed to TQ3 straight from
+        the bf16 values, as ``convert`` packs an FP8 page's values; every other page is written
+        as a fresh FP8 page, as by ``append``.  Pages take slots of their own format, in
+        ascending page order, sequences in list order."""
+        seq_ids = [int(s) for s in seq_ids]
+        n_tokens = [int(n) for n in n_tokens]
+        for s in seq_ids:
+            self._check_seq(s)
+        if (len(set(seq_ids)) != len(seq_ids) or any(n < 0 for n in n_tokens)
+                or window_tokens < 0):
+            raise PoolError("INVALID_ARG", "repeated sequence, negative count or window")
+        if any(self.table[s] or self.ctx[s] for s in seq_ids):
+            raise PoolError("INVALID_ARG", "prefill needs empty sequences")
+        direct = []
+        need = [0, 0]
+        for s, n in zip(seq_ids, n_tokens):
+            pages = -(-n // PAGE)
+            if pages > self.max_pages:
+                raise PoolError("OUT_OF_PAGES", f"sequence {s} exceeds max pages")
+            d = [p >= self.sink_pages and PAGE * p + PAGE <= n - window_tokens
+                 for p in range(pages)]
+            direct.append(d)
+            need[TQ3] += sum(d)
+            need[FP8] += pages - sum(d)
+        for fmt in (FP8, TQ3):
+            if need[fmt] > len(self.alloc[fmt].free):
+                raise PoolError("OUT_OF_PAGES", "pool exhausted")
+        row = 0
+        for s, n, d in zip(seq_ids, n_tokens, direct):
+            for p, is_tq3 in enumerate(d):
+                r0, cnt = row + PAGE * p, min(PAGE, n - PAGE * p)
+                if is_tq3:
+                    slot = self.alloc[TQ3].take()
+                    res = []
+                    for src in (k, v):
+                        x = np.transpose(src[r0:r0 + PAGE], (1, 0, 2))          # [Hkv,16,D]
+                        q, sc = F.tq3_quantize(x.reshape(self.Hkv, PAGE, self.G, F.TQ3_GROUP))
+                        res += [q.reshape(self.Hkv, PAGE, self.D), sc]
+                    self.tq3[slot] = res
+                    self.table[s].append((TQ3, slot))
+                else:
+                    slot = self.alloc[FP8].take()
+                    z = np.zeros((self.Hkv, PAGE, self.D), np.uint8)
+                    st = [z, z.copy(), np.zeros(self.Hkv), np.zeros(self.Hkv)]
+                    for h in range(self.Hkv):
+                        for which, src in ((0, k), (1, v)):
+                            codes, sc = F.fp8_write(st[which][h], st[2 + which][h], 0,
+                                                    src[r0:r0 + cnt, h, :])
+                            st[which][h] = codes
+                            st[2 + which][h] = sc
+                    self.fp8[slot] = st
+                    self.table[s].append((FP8, slot))
+            self.ctx[s] = n
+            row += n
+
     # ------------------------------------------------------------------ policy
     def is_anchor(self, seq, page, window_tokens) -> bool:
         L = self.ctx[seq]

@@ -168,3 +168,30 @@ def test_stats_footprint_formula():
     live, n8, n3, bpt = lp.stats()
     assert (live, n8, n3) == (1600, 1 + 32, 67)
     assert bpt == pytest.approx((33 * 4 * (32 * 256 + 16) + 67 * 4 * 14 * 256) / 1600)
+
+
+@pytest.mark.parametrize("window,sink", [(0, 1), (48, 1), (1000, 1), (16, 0), (32, 3)])
+def test_host_only_prefill_tables_match_oracle(window, sink):
+    """Slot allocation of the direct prefill pack (pages ascending, each from its format's
+    slab, sequences in list order) matches the oracle's block tables."""
+    rng = np.random.default_rng(window + sink)
+    lens = [0, 1, 15, 16, 17, 200, 333]
+    Hkv, D = 2, 64
+    lp = Pool(Hkv, D, len(lens) + 1, 32, 80, 80, sink_pages=sink, host_only=True)
+    op = P.RefPool(Hkv, D, len(lens) + 1, 32, 80, 80, sink_pages=sink)
+    for fmt in (0, 1):
+        order = rng.permutation(80).astype(np.int32)
+        lp.set_slot_order(fmt, order)
+        op.set_slot_order(fmt, order)
+    lp.append([len(lens)], [5])
+    op.append([len(lens)], [5], np.zeros((5, Hkv, D)), np.zeros((5, Hkv, D)))
+    seqs = list(range(len(lens)))
+    lp.prefill(seqs, lens, window=window)
+    x = np.zeros((sum(lens), Hkv, D))
+    op.prefill(seqs, lens, x, x, window)
+    for s in seqs + [len(lens)]:
+        t, ctx = lp.block_table(s)
+        assert t == op.block_table(s) and ctx == op.ctx[s], s
+    with pytest.raises(MkvError) as e:
+        lp.prefill([len(lens)], [16], window=0)          # not empty
+    assert e.value.name == "INVALID_ARG"
