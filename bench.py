@@ -440,7 +440,9 @@ def run_reference(args, rank, world):
 # workload's head shape, mixed cache against an all-FP8 control: decode time and KV bytes per
 # token), --mode pack (bulk FP8 -> TQ3 demotion of an all-FP8 pool shaped like the batch-8
 # workload, in GB/s), --mode prefill (direct bf16 -> TQ3 packing of that workload's prompts) and
-# --mode materialise (dense fp32 K and V of that workload's sequences).
+# --mode materialise (dense fp32 K and V of that workload's sequences), --mode configs (decode
+# µs per call, algorithmic GB/s and roofline fractions of every workload configuration, L2
+# flushed before each call, and the steady-state append -> demote -> decode step).
 def _bf16_tensor(bits, device):
     import torch
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
@@ -607,6 +609,83 @@ def run_extra(args):
         lines.append(dict(mode="materialise", workload=w.name, tokens=sum(ctxs), bytes=int(kv_bytes + out_bytes),
                           ms=round(ms, 4), gbs=round(gbs, 1), frac=round(gbs / peak, 4),
                           peak_source=peak_src, note="mkv_materialise_kv of every sequence (dense fp32 K and V)"))
+    elif args.mode == "configs":
+        from mixed_format_paged_mkv_b200.workloads import long_qlen4
+        spec_tbs = 8.0  # the spec HBM figure, reported beside the measured peak
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)   # > 126 MB L2
+        stream = torch.cuda.current_stream()
+        for w in (WORKLOADS[1], WORKLOADS[2], WORKLOADS[3], WORKLOADS[4].scaled(layers=1),
+                  long_qlen4().scaled(layers=1)):
+            pool = build_pool(w, 1, 3, device)
+            seqs = list(range(w.B))
+            q = _bf16_tensor(np.stack([w.q(s) for s in seqs]), device)
+            out = torch.empty((w.B, w.q_len, w.Hq, w.D), dtype=torch.float32, device=device)
+            ws = torch.empty(pool.workspace_bytes(seqs, w.q_len, w.Hq) + (1 << 20),
+                             dtype=torch.uint8, device=device)
+            for _ in range(3):
+                pool.decode(seqs, q, out=out, workspace=ws)
+            pool.timing(True)
+            pool.timing_read()
+            for _ in range(20):   # L2 flushed before every call
+                flush.zero_()
+                pool.decode(seqs, q, out=out, workspace=ws)
+            tm = pool.timing_read()
+            pool.timing(False)
+            pool.device_status()
+            tabs, ctxs = zip(*(pool.block_table(s) for s in seqs))
+            total, partial = decode_bytes(tabs, ctxs, w.Hkv, w.D, w.Hq, w.q_len)
+            pu, mu = 1000 * tm["partial_ms"] / tm["calls"], 1000 * tm["merge_ms"] / tm["calls"]
+            gbs = partial / (pu * 1e-6) / 1e9
+            lines.append(dict(mode="configs", workload=w.name, sequences=w.B, tokens=int(sum(ctxs)),
+                              q_len=w.q_len, partial_us=round(pu, 2), merge_us=round(mu, 2),
+                              call_us=round(pu + mu, 2), algorithmic_bytes=int(total),
+                              partial_gbs=round(gbs, 1), frac_of_measured=round(gbs / peak, 4),
+                              frac_of_8tbs=round(gbs / (spec_tbs * 1000), 4),
+                              call_gbs=round(total / ((pu + mu) * 1e-6) / 1e9, 1),
+                              l2="flushed (256 MB write) before every call"))
+            del pool, ws
+            torch.cuda.empty_cache()
+        # steady state: per step append 1 token per sequence, demote, decode
+        w = WORKLOADS[5]
+        warm, steps = 16, 64
+        pool = build_pool(w, 1, (warm + steps) // 16 + 3, device)
+        seqs = list(range(w.B))
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(warm + steps)]
+        out = torch.empty((w.B, 1, w.Hq, w.D), dtype=torch.float32, device=device)
+        ws = torch.empty(int(pool.workspace_bytes(seqs, 1, w.Hq) * 1.5) + (1 << 20),
+                         dtype=torch.uint8, device=device)
+        ones = [1] * w.B
+        demoted = 0
+        kvq = [w.step_inputs(st, 0) for st in range(warm + steps)]
+        kvq = [(_bf16_tensor(k, device), _bf16_tensor(v, device), _bf16_tensor(q, device))
+               for k, v, q in kvq]
+        for st in range(warm + steps):
+            k, v, q = kvq[st]
+            e = ev[st]
+            e[0].record(stream)
+            pool.append(seqs, ones, k, v)
+            e[1].record(stream)
+            n = pool.demote(seqs, w.window)
+            e[2].record(stream)
+            pool.decode(seqs, q, out=out, workspace=ws)
+            e[3].record(stream)
+            if st >= warm:
+                demoted += n
+        torch.cuda.synchronize()
+        pool.device_status()
+        ph = np.array([[ev[st][i].elapsed_time(ev[st][i + 1]) for i in range(3)]
+                       for st in range(warm, warm + steps)]) * 1000
+        tabs, ctxs = zip(*(pool.block_table(s) for s in seqs))
+        total, partial = decode_bytes(tabs, ctxs, w.Hkv, w.D, w.Hq, 1)
+        dec = float(np.median(ph[:, 2]))
+        lines.append(dict(mode="configs", workload=w.name, sequences=w.B, tokens=int(sum(ctxs)),
+                          steps=steps, append_us=round(float(np.median(ph[:, 0])), 2),
+                          demote_us=round(float(np.median(ph[:, 1])), 2), decode_us=round(dec, 2),
+                          step_us=round(float(np.median(ph.sum(1))), 2),
+                          pages_demoted_per_step=round(demoted / steps, 2),
+                          decode_call_gbs=round(total / (dec * 1e-6) / 1e9, 1),
+                          frac_of_measured=round(total / (dec * 1e-6) / 1e9 / peak, 4),
+                          note="medians over the timed steps; spans include host planning"))
     for l in lines:
         print(json.dumps(l), flush=True)
 
@@ -621,7 +700,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--mode", choices=["bench", "sweep", "canary", "pack", "prefill", "materialise"],
+    ap.add_argument("--mode", choices=["bench", "sweep", "canary", "pack", "prefill", "materialise",
+                                       "configs"],
                     default="bench",
                     help="extra studies on one GPU (one JSON line per point); default: the bench")
     args = ap.parse_args()

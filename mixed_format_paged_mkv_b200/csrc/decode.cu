@@ -669,7 +669,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
 }
 
 template <int D, int NT>
-__global__ void __launch_bounds__(Cfg<D, NT>::THREADS, 3)
+__global__ void __launch_bounds__(Cfg<D, NT>::THREADS, D == 256 ? 3 : 4)
     decode_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const Smem sm = carve<D, NT>(smem_raw);
