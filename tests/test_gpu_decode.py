@@ -127,3 +127,20 @@ def test_long_context_full_size_sampled():
         op = oracle_pool(w, seqs=[s], heads=[h], shape=dict(w.pool_shape(), num_kv_heads=1))
         ref = oracle_decode(op, w, s, heads=[h])
         assert_close(out[s][:, h * w.g:(h + 1) * w.g], ref, what=f"full-size seq {s} head {h}")
+
+
+def test_more_sequences_than_one_launch_holds():
+    """300 sequences (more than a launch's 256) are split into launch groups; every row must
+    still come out right, in call order."""
+    rng = np.random.default_rng(30)
+    n = 300
+    ctx = tuple(int(x) for x in rng.integers(1, 60, size=n))
+    w = Workload("many", 30, B=n, Hq=4, Hkv=2, D=64, q_len=1, window=16, ctx=ctx)
+    lp = lib_pool(w)
+    op = oracle_pool(w)
+    order = list(rng.permutation(n))
+    q = to_bf16_tensor(np.stack([w.q(s) for s in order]))
+    out = lp.decode(order, q).cpu().numpy()
+    lp.device_status()
+    for i, s in enumerate(order):
+        assert_close(out[i], oracle_decode(op, w, s), what=f"row {i} seq {s}")
