@@ -251,9 +251,12 @@ class Pool:
     def materialise(self, seq, k_out=None, v_out=None, stream=None):
         """Dense fp32 dequantised K and V of a sequence, [ctx, Hkv, D] each (a debugging and
         quality-control path; decode never uses it)."""
+        if self.host_only:  # the library rejects it (no device pages)
+            _check(lib().mkv_materialise_kv(self.handle, seq, None, None, 0, None),
+                   "mkv_materialise_kv")
         import torch
         _, ctx = self.block_table(seq)
-        dev = self.buffers[0].device if self.buffers else torch.device("cuda")
+        dev = self.buffers[0].device
         shape = (ctx, self.Hkv, self.D)
         k_out = torch.empty(shape, dtype=torch.float32, device=dev) if k_out is None else k_out
         v_out = torch.empty(shape, dtype=torch.float32, device=dev) if v_out is None else v_out

@@ -195,3 +195,29 @@ def test_host_only_prefill_tables_match_oracle(window, sink):
     with pytest.raises(MkvError) as e:
         lp.prefill([len(lens)], [16], window=0)          # not empty
     assert e.value.name == "INVALID_ARG"
+
+
+def test_prefill_and_materialise_errors_leave_the_pool_unchanged():
+    lp = Pool(1, 64, 3, 8, 3, 8, host_only=True)
+    op = P.RefPool(1, 64, 3, 8, 3, 8)
+    with pytest.raises(MkvError) as e:
+        lp.prefill([0], [16], window=-1)
+    assert e.value.name == "INVALID_ARG"
+    with pytest.raises(MkvError) as e:
+        lp.prefill([0, 0], [16, 16], window=0)
+    assert e.value.name == "INVALID_ARG"
+    # 100 tokens, window 100: all 7 pages stay FP8, 3 FP8 slots -> nothing may change
+    with pytest.raises(MkvError) as e:
+        lp.prefill([1], [100], window=100)
+    assert e.value.name == "OUT_OF_PAGES"
+    assert lp.block_table(1) == ([], 0)
+    # the same call with window 0 packs pages 1..5 to TQ3 and keeps page 0 and the partial
+    # page 6 as FP8
+    lp.prefill([1], [100], window=0)
+    x = np.zeros((100, 1, 64))
+    op.prefill([1], [100], x, x, 0)
+    assert lp.block_table(1) == (op.block_table(1), 100)
+    assert [e >> 30 for e in lp.block_table(1)[0]] == [0, 1, 1, 1, 1, 1, 0]
+    with pytest.raises(MkvError) as e:
+        lp.materialise(1)
+    assert e.value.name == "INVALID_ARG"
