@@ -213,6 +213,13 @@ MKV_API int mkv_slot_bytes(mkv_pool_t pool, int32_t fmt, size_t* bytes);
 MKV_API int mkv_read_slot(mkv_pool_t pool, int32_t entry, void* host_out, size_t cap,
                           void* stream);
 
+/* Self-test of failure detection (no counterpart in the pages): launch one kernel that waits on
+ * a device barrier nothing completes, with the library's bounded wait cut to limit_ns
+ * (0 .. 2e9).  The wait gives up and records a timeout in the status word, so the next
+ * mkv_get_device_status returns MKV_ERR_DEVICE_TIMEOUT; the context stays usable.  Errors:
+ * INVALID_ARG (host-only pool, limit out of range), CUDA. */
+MKV_API int mkv_selftest_wait(mkv_pool_t pool, int64_t limit_ns, void* stream);
+
 /* Prefill-time compression: write the first n_tokens[i] tokens of each listed sequence, which
  * must be empty (k, v as for mkv_append_kv).  Every full page that the anchor policy would
  * demote at once -- page p >= sink_pages with 16p + 16 <= n - anchor_window_tokens (new pages

@@ -54,6 +54,7 @@ SIGNATURES = {
     "mkv_seq_copy": (ctypes.c_int, [_P, _I32, _I32, _P]),
     "mkv_materialise_kv": (ctypes.c_int, [_P, _I32, _P, _P, ctypes.c_int64, _P]),
     "mkv_prefill_kv": (ctypes.c_int, [_P, _I32P, _I32P, _I32, _P, _P, _I32, _P]),
+    "mkv_selftest_wait": (ctypes.c_int, [_P, ctypes.c_int64, _P]),
     "mkv_get_block_table": (ctypes.c_int, [_P, _I32, _I32P, _I32, _I32P, _I32P]),
     "mkv_slot_bytes": (ctypes.c_int, [_P, _I32, _SZP]),
     "mkv_read_slot": (ctypes.c_int, [_P, _I32, _P, ctypes.c_size_t, _P]),
@@ -200,6 +201,11 @@ class Pool:
             st = _stream_ptr(stream)
         _check(lib().mkv_prefill_kv(self.handle, sp, np_, s.size, kp, vp, int(window), st),
                "mkv_prefill_kv")
+
+    def selftest_wait(self, limit_ns=1_000_000, stream=None):
+        """Launch the bounded-wait self-test; the next device_status() raises DEVICE_TIMEOUT."""
+        st = None if self.host_only else _stream_ptr(stream)
+        _check(lib().mkv_selftest_wait(self.handle, int(limit_ns), st), "mkv_selftest_wait")
 
     def set_protected(self, seq, page, flag=True):
         _check(lib().mkv_set_protected(self.handle, seq, page, 1 if flag else 0), "mkv_set_protected")

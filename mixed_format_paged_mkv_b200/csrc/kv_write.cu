@@ -206,7 +206,24 @@ __global__ void __launch_bounds__(256) materialise_kernel(const __grid_constant_
   }
 }
 
+// Self-test of the bounded waits: one thread waits on a barrier that nothing completes, gives
+// up after limit_ns and records a timeout in the status word, as every wait of the library
+// does; the context stays usable.
+__global__ void wait_selftest_kernel(int32_t* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    mbar_fence_init();
+    if (!mbar_wait(&bar, 0, limit_ns)) flag_status(status, kStatusTimeout);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_wait_selftest(int32_t* status, uint64_t limit_ns, cudaStream_t s) {
+  wait_selftest_kernel<<<1, 32, 0, s>>>(status, limit_ns);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_pack(const PackParams& p, cudaStream_t s) {
   if (p.n_desc <= 0) return cudaSuccess;

@@ -800,6 +800,17 @@ int mkv_seq_reset(mkv_pool_t p, int32_t seq, void* stream) {
   return ok();
 }
 
+int mkv_selftest_wait(mkv_pool_t p, int64_t limit_ns, void* stream) {
+  if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
+  if (p->host_only) return fail(MKV_ERR_INVALID_ARG, "host-only pool has no device");
+  if (limit_ns < 0 || limit_ns > 2000000000LL)
+    return fail(MKV_ERR_INVALID_ARG, "limit must be in [0, 2 s]");
+  cudaError_t e = launch_wait_selftest(p->d_status, static_cast<uint64_t>(limit_ns), as_stream(stream));
+  ++p->launches;
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  return ok();
+}
+
 int mkv_prefill_kv(mkv_pool_t p, const int32_t* seq_ids, const int32_t* n_tokens, int32_t n_seqs,
                    const void* k_bf16, const void* v_bf16, int32_t anchor_window_tokens,
                    void* stream) {

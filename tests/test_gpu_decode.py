@@ -144,3 +144,43 @@ def test_more_sequences_than_one_launch_holds():
     lp.device_status()
     for i, s in enumerate(order):
         assert_close(out[i], oracle_decode(op, w, s), what=f"row {i} seq {s}")
+
+
+def test_bounded_wait_reports_a_timeout_and_the_context_survives():
+    """Failure detection without a fault: a wait that nothing completes gives up after its limit
+    and is reported as DEVICE_TIMEOUT; the same context then decodes correctly."""
+    from mixed_format_paged_mkv_b200 import MkvError
+    w = Workload("wait", 31, B=1, Hq=4, Hkv=2, D=64, q_len=1, window=16, ctx=(100,))
+    lp = lib_pool(w)
+    lp.device_status()
+    lp.selftest_wait(1_000_000)
+    with pytest.raises(MkvError) as e:
+        lp.device_status()
+    assert e.value.name == "DEVICE_TIMEOUT"
+    lp.device_status()  # reading cleared it
+    run_and_check(w, lp=lp)
+
+
+def test_corrupted_device_table_entry_is_flagged():
+    """A table entry corrupted on the device (slot beyond the slab) is caught by the kernels'
+    checks (the page is skipped, not read) and reported as DEVICE_CHECK; restoring it restores
+    the result."""
+    from mixed_format_paged_mkv_b200 import MkvError
+    w = Workload("corrupt", 32, B=2, Hq=4, Hkv=2, D=64, q_len=1, window=16, ctx=(300, 90))
+    shape = w.pool_shape()
+    lp = lib_pool(w, shape=shape)
+    tables = lp.buffers[2].view(torch.int32)
+    idx = 0 * shape["max_pages_per_seq"] + 3          # sequence 0, page 3 (TQ3)
+    good = int(tables[idx].item())
+    assert good >> 30 == 1
+    tables[idx] = (1 << 30) | (shape["tq3_slots"] + 7)
+    lp.decode([0, 1], q_tensor(w))
+    with pytest.raises(MkvError) as e:
+        lp.device_status()
+    assert e.value.name == "DEVICE_CHECK"
+    lp.materialise(0)
+    with pytest.raises(MkvError) as e:
+        lp.device_status()
+    assert e.value.name == "DEVICE_CHECK"
+    tables[idx] = good
+    run_and_check(w, lp=lp)
