@@ -220,6 +220,15 @@ MKV_API int mkv_read_slot(mkv_pool_t pool, int32_t entry, void* host_out, size_t
  * INVALID_ARG (host-only pool, limit out of range), CUDA. */
 MKV_API int mkv_selftest_wait(mkv_pool_t pool, int64_t limit_ns, void* stream);
 
+/* Self-test of the Blackwell tensor-memory MMA path that a tcgen05 logits kernel would use
+ * (no counterpart in the pages; decode does not use it yet): one CTA computes
+ * d_out[128][8] (fp32) = a[128][256] . q[8][256]^T (f16, row-major device buffers).  Each
+ * thread writes one row of a into tensor memory, q is read by the tensor core from shared
+ * memory, one thread issues tcgen05.mma and the result is read back from tensor memory.  A
+ * bounded wait records MKV_ERR_DEVICE_TIMEOUT in the status word.  Errors: INVALID_ARG, CUDA. */
+MKV_API int mkv_selftest_tc_logits(mkv_pool_t pool, const void* a_f16, const void* q_f16,
+                                   float* d_out, void* stream);
+
 /* Prefill-time compression: write the first n_tokens[i] tokens of each listed sequence, which
  * must be empty (k, v as for mkv_append_kv).  Every full page that the anchor policy would
  * demote at once -- page p >= sink_pages with 16p + 16 <= n - anchor_window_tokens (new pages

@@ -55,6 +55,7 @@ SIGNATURES = {
     "mkv_materialise_kv": (ctypes.c_int, [_P, _I32, _P, _P, ctypes.c_int64, _P]),
     "mkv_prefill_kv": (ctypes.c_int, [_P, _I32P, _I32P, _I32, _P, _P, _I32, _P]),
     "mkv_selftest_wait": (ctypes.c_int, [_P, ctypes.c_int64, _P]),
+    "mkv_selftest_tc_logits": (ctypes.c_int, [_P, _P, _P, _P, _P]),
     "mkv_get_block_table": (ctypes.c_int, [_P, _I32, _I32P, _I32, _I32P, _I32P]),
     "mkv_slot_bytes": (ctypes.c_int, [_P, _I32, _SZP]),
     "mkv_read_slot": (ctypes.c_int, [_P, _I32, _P, ctypes.c_size_t, _P]),
@@ -206,6 +207,19 @@ class Pool:
         """Launch the bounded-wait self-test; the next device_status() raises DEVICE_TIMEOUT."""
         st = None if self.host_only else _stream_ptr(stream)
         _check(lib().mkv_selftest_wait(self.handle, int(limit_ns), st), "mkv_selftest_wait")
+
+    def selftest_tc_logits(self, a, q, stream=None):
+        """fp32 [128, 8] = a [128, 256] . q [8, 256]^T (f16 device tensors) through tensor memory
+        and tcgen05.mma (mkv_selftest_tc_logits)."""
+        import torch
+        if tuple(a.shape) != (128, 256) or tuple(q.shape) != (8, 256):
+            raise ValueError("a must be [128, 256] and q [8, 256]")
+        d = torch.empty((128, 8), dtype=torch.float32, device=a.device)
+        _check(lib().mkv_selftest_tc_logits(self.handle, _dev_ptr(a, torch.float16, "a"),
+                                            _dev_ptr(q, torch.float16, "q"),
+                                            _dev_ptr(d, torch.float32, "d"), _stream_ptr(stream)),
+               "mkv_selftest_tc_logits")
+        return d
 
     def set_protected(self, seq, page, flag=True):
         _check(lib().mkv_set_protected(self.handle, seq, page, 1 if flag else 0), "mkv_set_protected")

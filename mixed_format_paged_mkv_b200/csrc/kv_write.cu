@@ -7,6 +7,7 @@
 // host computation that applies the same roundings.
 #include "device_util.cuh"
 #include "mkv_internal.h"
+#include "selftest.h"
 
 namespace mkv {
 

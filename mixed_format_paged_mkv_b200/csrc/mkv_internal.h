@@ -153,7 +153,6 @@ cudaError_t launch_demote(const DemoteParams& p, cudaStream_t s);
 cudaError_t launch_copy(const CopyParams& p, cudaStream_t s);
 cudaError_t launch_materialise(const MaterialiseParams& p, cudaStream_t s);
 cudaError_t launch_pack(const PackParams& p, cudaStream_t s);
-cudaError_t launch_wait_selftest(int32_t* status, uint64_t limit_ns, cudaStream_t s);
 cudaError_t launch_partial(const DecodeParams& p, cudaStream_t s);
 cudaError_t launch_merge(const DecodeParams& p, cudaStream_t s);
 bool partial_supported(int D, int NC);

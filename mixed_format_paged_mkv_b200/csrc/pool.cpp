@@ -17,6 +17,7 @@
 
 #include "mkv.h"
 #include "mkv_internal.h"
+#include "selftest.h"
 
 using namespace mkv;
 
@@ -808,6 +809,17 @@ int mkv_selftest_wait(mkv_pool_t p, int64_t limit_ns, void* stream) {
   cudaError_t e = launch_wait_selftest(p->d_status, static_cast<uint64_t>(limit_ns), as_stream(stream));
   ++p->launches;
   if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  return ok();
+}
+
+int mkv_selftest_tc_logits(mkv_pool_t p, const void* a_f16, const void* q_f16, float* d_out,
+                           void* stream) {
+  if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
+  if (p->host_only) return fail(MKV_ERR_INVALID_ARG, "host-only pool has no device");
+  if (!a_f16 || !q_f16 || !d_out) return fail(MKV_ERR_INVALID_ARG, "a/q/d is NULL");
+  cudaError_t e = launch_tc_logits_selftest(a_f16, q_f16, d_out, p->d_status, as_stream(stream));
+  ++p->launches;
+  if (e != cudaSuccess) return cuda_fail(e, "tensor-memory self-test launch");
   return ok();
 }
 
