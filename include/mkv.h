@@ -149,6 +149,20 @@ MKV_API int mkv_decode_workspace_bytes(mkv_pool_t pool, const int32_t* seq_ids,
                                        int32_t n_seqs, int32_t q_len, int32_t num_q_heads,
                                        size_t* bytes);
 
+/* The work units mkv_decode_attention would cut for this call (host computation; also on
+ * host-only pools), for inspection and tests.  A unit is the pages of one format (0 FP8, 1 TQ3)
+ * inside a logical page range of one sequence; the partial kernel runs one CTA per (unit, KV
+ * head).  units_out (host int32 [cap][5]) receives, per unit in sequence order: {call position
+ * of the sequence, format, first logical page, end logical page (exclusive), pages of that
+ * format in the range}; with units_out NULL the call only counts.  *n_units receives the unit
+ * count, also when it exceeds cap (then INVALID_ARG and nothing is written); *ctas_per_wave
+ * (may be NULL) the CTA
+ * budget of one wave the cut aims at (SMs x resident partial CTAs per SM; 148 x 1 where no
+ * device is visible).  Errors: as mkv_decode_workspace_bytes, INVALID_ARG. */
+MKV_API int mkv_decode_plan(mkv_pool_t pool, const int32_t* seq_ids, int32_t n_seqs,
+                            int32_t q_len, int32_t num_q_heads, int32_t* units_out, int32_t cap,
+                            int32_t* n_units, int32_t* ctas_per_wave);
+
 /* Decode attention directly over the mixed-format cache (section "Como os resultados
  * parciais são combinados"): for sequence seq_ids[i] of length L, query j < q_len (the new
  * tokens are the last q_len positions), query head hq (KV head hq / (num_q_heads/Hkv)):

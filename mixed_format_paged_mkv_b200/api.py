@@ -46,6 +46,7 @@ SIGNATURES = {
     "mkv_set_protected": (ctypes.c_int, [_P, _I32, _I32, _I32]),
     "mkv_demote_pages": (ctypes.c_int, [_P, _I32P, _I32, _I32, _I32P, _P]),
     "mkv_decode_workspace_bytes": (ctypes.c_int, [_P, _I32P, _I32, _I32, _I32, _SZP]),
+    "mkv_decode_plan": (ctypes.c_int, [_P, _I32P, _I32, _I32, _I32, _I32P, _I32, _I32P, _I32P]),
     "mkv_decode_attention": (ctypes.c_int, [_P, _I32P, _I32, _I32, _P, _I32, ctypes.c_float,
                                             _P, _P, ctypes.c_size_t, _P]),
     "mkv_decode_attention_noalloc": (ctypes.c_int, [_P, _I32P, _I32, _I32, _P, _I32,
@@ -238,6 +239,20 @@ class Pool:
         _check(lib().mkv_decode_workspace_bytes(self.handle, sp, s.size, q_len, num_q_heads,
                                                 ctypes.byref(b)), "mkv_decode_workspace_bytes")
         return b.value
+
+    def decode_plan(self, seq_ids, q_len, num_q_heads):
+        """The work units a decode call would cut (mkv_decode_plan): int32 [units, 5] rows of
+        (call position, format, first logical page, end logical page, pages of that format), and
+        the CTA budget of one wave."""
+        s, sp = _i32_array(seq_ids)
+        n, wave = ctypes.c_int32(), ctypes.c_int32()
+        _check(lib().mkv_decode_plan(self.handle, sp, s.size, q_len, num_q_heads, None, 0,
+                                     ctypes.byref(n), ctypes.byref(wave)), "mkv_decode_plan")
+        u = np.zeros((max(n.value, 1), 5), dtype=np.int32)
+        _check(lib().mkv_decode_plan(self.handle, sp, s.size, q_len, num_q_heads,
+                                     u.ctypes.data_as(_I32P), n.value, ctypes.byref(n), None),
+               "mkv_decode_plan")
+        return u[:n.value], wave.value
 
     def decode(self, seq_ids, q, sm_scale=None, out=None, workspace=None, stream=None):
         """q: bf16 [n, q_len, Hq, D] on the device -> fp32 [n, q_len, Hq, D]."""

@@ -158,7 +158,8 @@ size_t status_bytes(const mkv_pool_config&) { return 256; }
 struct DecodePlan {
   int32_t NC = 0, g = 0;
   std::vector<SeqDesc> seq;    // per call position
-  std::vector<UnitDesc> unit;  // per sequence, in order; UnitDesc::seq = call position
+  std::vector<UnitDesc> unit;  // per sequence, in order
+  std::vector<int32_t> pos;    // call position of each unit's sequence
   std::vector<int64_t> cost;   // relative time of each unit (per KV head)
   int64_t parts = 0;
   size_t off_ml = 0, off_acc = 0, bytes = 0;
@@ -173,8 +174,9 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 // fits that budget, so the longest CTA, which ends the wave, is as short as the groups allow.
 // A single balanced wave measured faster than several smaller ones: each CTA sets up and
 // combines its warps once and no partial last wave is left.  Units hold at most
-// kMaxPagesPerUnit and at least a few pages.  `emit(unit, cost)` is called in sequence order;
-// UnitDesc::part numbers the units of a sequence.  Returns the unit count, or -1 as soon as
+// kMaxPagesPerUnit and at least a few pages.  `emit(unit, cost, pos)` is called in sequence
+// order, pos the sequence's call position (UnitDesc::seq is left 0: it is the position within
+// one launch, set when the units are grouped); UnitDesc::part numbers the units of a sequence.  Returns the unit count, or -1 as soon as
 // `emit` returns false.
 constexpr int kMinTq3PagesPerUnit = 8;
 constexpr int kMinFp8PagesPerUnit = 4;
@@ -234,8 +236,7 @@ int64_t cut_units(const mkv_pool* p, const int32_t* seq_ids, int32_t n, int32_t 
       for (int64_t k = 0; k < u; ++k) {
         const int64_t j0 = k * n8 / u, j1 = (k + 1) * n8 / u;
         if (j1 <= j0) continue;
-        if (!emit(UnitDesc{f8[j0], f8[j1 - 1] + 1, static_cast<int16_t>(i), 0, np++}, (j1 - j0) * b8))
-          return -1;
+        if (!emit(UnitDesc{f8[j0], f8[j1 - 1] + 1, 0, 0, np++}, (j1 - j0) * b8, i)) return -1;
         ++nu;
       }
     }
@@ -244,29 +245,25 @@ int64_t cut_units(const mkv_pool* p, const int32_t* seq_ids, int32_t n, int32_t 
       const int64_t u = units_at(unit_cost, n3 * b3, n3, kMinTq3PagesPerUnit);
       // unit k takes TQ3 pages number [k n3 / u, (k+1) n3 / u) in logical order; its range
       // starts at the logical page of its first TQ3 page (the first unit at page 0) and ends
-      // where the next one starts (the last at the end of the table)
+      // where the next one starts (the last at the end of the table).  Every page of the table
+      // is FP8 or TQ3, so TQ3 page number j sits at logical page j + c, c the number of FP8
+      // pages before it: one merge over the ascending FP8 list finds all boundaries, without
+      // walking the table.
       const int32_t pages = static_cast<int32_t>(s.table.size());
+      int64_t c = 0;
       int32_t start = 0;
-      int64_t seen = 0, k = 0, next = (k + 1) * n3 / u;
-      for (int32_t lp = 0; lp < pages && k < u; ++lp) {
-        const int32_t e = s.table[lp];
-        if (e < 0 || fmt_of(e) != 1) continue;
-        if (seen == next) {  // lp is the first TQ3 page of unit k + 1
-          const int64_t cnt = next - k * n3 / u;
-          if (cnt > 0) {
-            if (!emit(UnitDesc{start, lp, static_cast<int16_t>(i), 1, np++}, cnt * b3)) return -1;
-            ++nu;
-          }
-          start = lp;
-          ++k;
-          next = (k + 1) * n3 / u;
+      for (int64_t k = 0; k < u; ++k) {
+        const int64_t j0 = k * n3 / u, j1 = (k + 1) * n3 / u;
+        int32_t end = pages;
+        if (k + 1 < u) {
+          while (c < n8 && f8[c] <= j1 + c) ++c;
+          end = static_cast<int32_t>(j1 + c);
         }
-        ++seen;
-      }
-      const int64_t cnt = n3 - k * n3 / u;
-      if (cnt > 0) {
-        if (!emit(UnitDesc{start, pages, static_cast<int16_t>(i), 1, np++}, cnt * b3)) return -1;
-        ++nu;
+        if (j1 > j0) {
+          if (!emit(UnitDesc{start, end, 0, 1, np++}, (j1 - j0) * b3, i)) return -1;
+          ++nu;
+        }
+        start = end;
       }
     }
     n_parts[i] = np;
@@ -294,10 +291,12 @@ int plan_decode(mkv_pool_t p, const int32_t* seq_ids, int32_t n, int32_t q_len, 
   }
   plan->seq.resize(n);
   plan->unit.clear();
+  plan->pos.clear();
   plan->cost.clear();
   std::vector<int32_t> np(n);
-  cut_units(p, seq_ids, n, plan->NC, np.data(), [&](const UnitDesc& u, int64_t cost) {
+  cut_units(p, seq_ids, n, plan->NC, np.data(), [&](const UnitDesc& u, int64_t cost, int32_t i) {
     plan->unit.push_back(u);
+    plan->pos.push_back(i);
     plan->cost.push_back(cost);
     return true;
   });
@@ -589,6 +588,32 @@ int mkv_decode_workspace_bytes(mkv_pool_t p, const int32_t* seq_ids, int32_t n_s
   return ok();
 }
 
+int mkv_decode_plan(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, int32_t q_len,
+                    int32_t Hq, int32_t* units_out, int32_t cap, int32_t* n_units,
+                    int32_t* ctas_per_wave) {
+  if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
+  if (!n_units || cap < 0) return fail(MKV_ERR_INVALID_ARG, "n_units is NULL or cap < 0");
+  DecodePlan plan;
+  if (int e = plan_decode(p, seq_ids, n_seqs, q_len, Hq, &plan)) return e;
+  const int64_t nu = static_cast<int64_t>(plan.unit.size());
+  *n_units = static_cast<int32_t>(nu);
+  if (ctas_per_wave)
+    *ctas_per_wave = p->sm_count * partial_ctas_per_sm(p->cfg.head_dim, plan.NC);
+  if (!units_out) return ok();  // count query
+  if (nu > cap) return fail(MKV_ERR_INVALID_ARG, "%lld units do not fit in %d", (long long)nu, cap);
+  const int64_t b[2] = {kFp8PageCost, kTq3PageCost};
+  for (int64_t k = 0; k < nu; ++k) {
+    const UnitDesc& u = plan.unit[k];
+    int32_t* o = units_out + 5 * k;
+    o[0] = plan.pos[k];
+    o[1] = u.fmt;
+    o[2] = u.first;
+    o[3] = u.last;
+    o[4] = static_cast<int32_t>(plan.cost[k] / b[u.fmt]);
+  }
+  return ok();
+}
+
 int mkv_decode_attention(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, int32_t q_len,
                          const void* q_bf16, int32_t Hq, float sm_scale, float* out,
                          void* workspace, size_t ws_bytes, void* stream) {
@@ -641,7 +666,7 @@ int mkv_decode_attention(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, i
     size_t u1 = u0;
     while (s1 < n_seqs && s1 - s0 < kDecodeMaxSeqs) {
       size_t ue = u1;
-      while (ue < plan.unit.size() && plan.unit[ue].seq == s1) ++ue;
+      while (ue < plan.unit.size() && plan.pos[ue] == s1) ++ue;
       if (ue - u0 > static_cast<size_t>(kDecodeMaxUnits) && s1 > s0) break;
       if (ue - u0 > static_cast<size_t>(kDecodeMaxUnits)) {
         err = cudaErrorInvalidValue;
@@ -658,7 +683,7 @@ int mkv_decode_attention(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, i
                      [&](size_t x, size_t y) { return plan.cost[x] > plan.cost[y]; });
     for (size_t k = 0; k < order.size(); ++k) {
       prm->unit[k] = plan.unit[order[k]];
-      prm->unit[k].seq = static_cast<int16_t>(plan.unit[order[k]].seq - s0);
+      prm->unit[k].seq = static_cast<int16_t>(plan.pos[order[k]] - s0);
     }
     prm->n_seqs = s1 - s0;
     prm->n_units = static_cast<int32_t>(order.size());
@@ -721,12 +746,14 @@ int mkv_decode_attention_noalloc(mkv_pool_t p, const int32_t* seq_ids, int32_t n
   DecodeParams& prm = t.prm;
   int32_t np[kDecodeMaxSeqs];
   int32_t nu = 0;
-  const int64_t cut = cut_units(p, seq_ids, n_seqs, NC, np, [&](const UnitDesc& u, int64_t cost) {
+  auto keep = [&](const UnitDesc& u, int64_t cost, int32_t i) {
     if (nu >= kDecodeMaxUnits) return false;
     t.unit[nu] = u;
+    t.unit[nu].seq = static_cast<int16_t>(i);  // n_seqs <= kDecodeMaxSeqs: one launch
     t.cost[nu++] = cost;
     return true;
-  });
+  };
+  const int64_t cut = cut_units(p, seq_ids, n_seqs, NC, np, keep);
   if (cut < 0)
     return fail(MKV_ERR_UNSUPPORTED, "the no-allocation decode takes at most %d work units per call", kDecodeMaxUnits);
   int32_t parts = 0;

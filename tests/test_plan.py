@@ -1,0 +1,174 @@
+"""The decode work-unit cut (mkv_decode_plan) on host-only pools.
+
+The cut is host logic: every sequence's pages of each format are split into units of whole pages,
+one CTA per (unit, KV head).  These tests check what any correct cut must satisfy -- each page of a
+format in exactly one unit of that format, TQ3 units splitting the TQ3 pages into equal shares in
+logical order, the page limits per unit, the one-wave budget -- and, on small cases, that the
+longest unit is within one page of the best cut a brute-force search finds under the same rules.
+"""
+import numpy as np
+import pytest
+
+from mixed_format_paged_mkv_b200 import Pool
+
+FP8, TQ3 = 0, 1
+MAX_PAGES, MIN_PAGES = 512, {FP8: 4, TQ3: 8}
+PAGE_COST = {FP8: 11, TQ3: 10}   # relative time of one page per CTA, as the planner weighs them
+
+
+def mixed_pool(lens, Hkv=4, sink=1, window=64, protect_frac=0.03, seed=0):
+    """Host-only pool whose sequences hold FP8 anchors (sink pages, the window, random protected
+    pages) among TQ3 pages."""
+    rng = np.random.default_rng(seed)
+    pages = [-(-n // 16) for n in lens]
+    pool = Pool(Hkv, 128, len(lens), max(pages) + 1, sum(pages) + 8, sum(pages) + 8,
+                sink_pages=sink, host_only=True)
+    seqs = list(range(len(lens)))
+    pool.append(seqs, list(lens))
+    for s, n in zip(seqs, pages):
+        for p in rng.choice(n, size=int(protect_frac * n), replace=False):
+            pool.set_protected(s, int(p), True)
+    pool.demote(seqs, window)
+    return pool, seqs
+
+
+def formats(pool, s):
+    table, _ = pool.block_table(s)
+    return np.array([e >> 30 for e in table])
+
+
+def check_cut(pool, seqs, units, wave, Hkv):
+    units = np.asarray(units)
+    assert np.all(np.diff(units[:, 0]) >= 0), "units not in sequence order"
+    min_units = 0
+    for pos, s in enumerate(seqs):
+        fm = formats(pool, s)
+        mine = units[units[:, 0] == pos]
+        for f in (FP8, TQ3):
+            idx = np.nonzero(fm == f)[0]
+            us = mine[mine[:, 1] == f]
+            if idx.size == 0:
+                assert us.size == 0
+                continue
+            min_units += -(-idx.size // MAX_PAGES)
+            covered = []
+            for _, _, first, end, cnt in us:
+                inside = idx[(idx >= first) & (idx < end)]
+                assert inside.size == cnt > 0
+                assert cnt <= MAX_PAGES and cnt >= min(MIN_PAGES[f], idx.size)
+                covered.extend(inside.tolist())
+            assert covered == idx.tolist(), f"seq {s} fmt {f}: pages not covered exactly once"
+            if f == TQ3:
+                # ranges tile the table; unit k holds TQ3 pages number [k n / u, (k+1) n / u)
+                u, n = len(us), idx.size
+                assert us[0, 2] == 0 and us[-1, 3] == fm.size
+                assert np.array_equal(us[1:, 2], us[:-1, 3])
+                for k in range(u):
+                    assert us[k, 4] == (k + 1) * n // u - k * n // u
+                    if k:
+                        assert us[k, 2] == idx[k * n // u]
+            else:
+                # ranges start and end on FP8 pages
+                assert np.all(fm[us[:, 2]] == FP8) and np.all(fm[us[:, 3] - 1] == FP8)
+                sizes = us[:, 4]
+                assert sizes.max() - sizes.min() <= 1
+    budget = max(1, wave // Hkv)
+    if min_units <= budget:
+        assert len(units) <= budget, (len(units), budget)
+    return units
+
+
+def group_pages(pool, seqs):
+    out = []
+    for s in seqs:
+        fm = formats(pool, s)
+        for f in (FP8, TQ3):
+            n = int((fm == f).sum())
+            if n:
+                out.append((f, n))
+    return out
+
+
+def best_longest_unit(groups, budget):
+    """Brute force: the smallest possible cost of the longest unit when group (f, n) is cut into
+    u equal shares, ceil(n / MAX_PAGES) <= u <= max(1, n // MIN_PAGES[f]), sum of u <= budget."""
+    def need(f, n, c):
+        lo, hi = -(-n // MAX_PAGES), max(-(-n // MAX_PAGES), 1, n // MIN_PAGES[f])
+        for u in range(lo, hi + 1):
+            if -(-n // u) * PAGE_COST[f] <= c:
+                return u
+        return None
+    cands = sorted({-(-n // u) * PAGE_COST[f] for f, n in groups
+                    for u in range(1, max(1, n // MIN_PAGES[f]) + 1)})
+    for c in cands:
+        us = [need(f, n, c) for f, n in groups]
+        if all(u is not None for u in us) and sum(us) <= budget:
+            return c
+    return None
+
+
+@pytest.mark.parametrize("lens,Hkv,window", [
+    ((131072,) * 4, 4, 512),
+    ((8192,) * 8, 8, 256),
+    ((2048, 32768, 5000, 17, 16, 4, 900, 12000), 4, 512),
+    ((65536, 100, 40000), 2, 64),
+])
+def test_cut_covers_every_page_once_within_one_wave(lens, Hkv, window):
+    pool, seqs = mixed_pool(lens, Hkv=Hkv, window=window, seed=len(lens))
+    for q_len in (1, 4):
+        units, wave = pool.decode_plan(seqs, q_len, 2 * Hkv)
+        check_cut(pool, seqs, units, wave, Hkv)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_longest_unit_is_within_one_page_of_the_best_cut(seed):
+    rng = np.random.default_rng(100 + seed)
+    Hkv = int(rng.choice([2, 4, 8]))
+    lens = rng.integers(16, 20000, size=int(rng.integers(1, 7))).tolist()
+    pool, seqs = mixed_pool(lens, Hkv=Hkv, window=int(rng.choice([0, 64, 512])),
+                            protect_frac=float(rng.choice([0.0, 0.05, 0.3])), seed=seed)
+    units, wave = pool.decode_plan(seqs, 1, Hkv)
+    check_cut(pool, seqs, units, wave, Hkv)
+    longest = max(int(c) * PAGE_COST[int(f)] for _, f, _, _, c in units)
+    best = best_longest_unit(group_pages(pool, seqs), max(1, wave // Hkv))
+    if best is not None:
+        assert best <= longest <= best + max(PAGE_COST.values()), (longest, best)
+
+
+def test_one_long_tq3_run_splits_evenly():
+    pool, seqs = mixed_pool((16 * 8192,), Hkv=4, window=0, protect_frac=0.0)
+    units, wave = pool.decode_plan(seqs, 1, 4)
+    units = check_cut(pool, seqs, units, wave, 4)
+    tq3 = units[units[:, 1] == TQ3]
+    budget = wave // 4
+    assert len(units) <= budget
+    assert tq3[:, 4].max() - tq3[:, 4].min() <= 1 and tq3[:, 4].sum() == 8191
+
+
+def test_call_positions_beyond_int16():
+    n = 33000
+    pool = Pool(1, 64, n, 1, n, 1, host_only=True)
+    seqs = list(range(n))[::-1]
+    pool.append(seqs, [16] * n)
+    units, _ = pool.decode_plan(seqs, 1, 1)
+    assert units.shape == (n, 5)
+    assert np.array_equal(units[:, 0], np.arange(n))
+    assert np.all(units[:, 1:] == [FP8, 0, 1, 1])
+
+
+def test_plan_count_query_and_small_buffer():
+    from mixed_format_paged_mkv_b200.api import MkvError, lib, _I32P
+    import ctypes
+    pool, seqs = mixed_pool((4096, 4096), Hkv=2)
+    units, _ = pool.decode_plan(seqs, 1, 2)
+    assert len(units) > 1
+    s = np.array(seqs, dtype=np.int32)
+    buf = np.zeros((len(units) - 1, 5), dtype=np.int32)
+    n = ctypes.c_int32()
+    rc = lib().mkv_decode_plan(pool.handle, s.ctypes.data_as(_I32P), s.size, 1, 2,
+                               buf.ctypes.data_as(_I32P), len(units) - 1, ctypes.byref(n), None)
+    assert rc == -1 and n.value == len(units) and not buf.any()
+    with pytest.raises(MkvError):
+        pool.decode_plan(seqs, 1, 3)          # 3 query heads over 2 KV heads
+    with pytest.raises(MkvError):
+        pool.decode_plan([0, 0, 5], 1, 2)     # sequence outside the pool
