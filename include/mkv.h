@@ -91,7 +91,8 @@ typedef struct {
   int32_t head_dim;          /* D: 64, 128 or 256 */
   int32_t page_size;         /* must be 16 */
   int32_t max_seqs;          /* rows of the block table */
-  int32_t max_pages_per_seq; /* columns of the block table */
+  int32_t max_pages_per_seq; /* columns of the block table; 16 x it must fit int32 (token
+                                counts), and max_seqs x it must too (table entries) */
   int32_t fp8_slots;         /* slots in the FP8 slab */
   int32_t tq3_slots;         /* slots in the TQ3 slab */
   int32_t sink_pages;        /* leading pages of every sequence that stay FP8 (page 0: 1) */

@@ -147,6 +147,8 @@ int validate_config(const mkv_pool_config* c) {
   if (c->flags & ~MKV_POOL_HOST_ONLY) return fail(MKV_ERR_INVALID_ARG, "unknown flags");
   if (static_cast<int64_t>(c->max_seqs) * c->max_pages_per_seq > (1LL << 31) - 1)
     return fail(MKV_ERR_INVALID_ARG, "table too large");
+  if (c->max_pages_per_seq > INT32_MAX / kPageTokens)
+    return fail(MKV_ERR_INVALID_ARG, "max_pages_per_seq too large: token counts are int32");
   return MKV_OK;
 }
 

@@ -134,6 +134,10 @@ def test_errors_leave_pool_unchanged():
     with pytest.raises(MkvError) as e:
         Pool(2, 96, 1, 1, 1, 1, host_only=True)
     assert e.value.name == "UNSUPPORTED"
+    with pytest.raises(MkvError) as e:
+        Pool(1, 64, 1, 2 ** 27, 1, 1, host_only=True)   # 16 x pages would overflow int32 tokens
+    assert e.value.name == "INVALID_ARG"
+    Pool(1, 64, 1, 2 ** 27 - 1, 1, 1, host_only=True)
     lp.append([1], [16])                # FP8 slab now full (3 of 3)
     with pytest.raises(MkvError) as e:
         lp.append([2], [1])
