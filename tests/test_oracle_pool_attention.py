@@ -2,9 +2,10 @@
 
 Pool: the anchor policy reproduces the workloads' stated FP8 page sets, slots are unique,
 every live page is mapped, allocation follows the slot order.  Attention: merge of any page
-partition equals single-pass attention, equal keys give mean(V), one token gives V, the
-first query of a q_len-4 causal call equals a q_len-1 call three tokens earlier, and a
-50-digit Decimal brute force agrees on tiny inputs.
+partition equals single-pass attention, the per-format partials merged equal the materialised
+dense attention, the dequantised sequence equals the raw slot bytes parsed by layout, equal keys
+give mean(V), one token gives V, the first query of a q_len-4 causal call equals a q_len-1 call
+three tokens earlier, and a 50-digit Decimal brute force agrees on tiny inputs.
 """
 from decimal import Decimal, getcontext
 
@@ -139,6 +140,49 @@ def test_merge_of_any_page_partition_equals_single_pass():
             parts.append(A.partial_state(K, V, q, 0.125, toks))
         out = A.merge(parts)
         assert np.max(np.abs(out - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
+def test_per_format_partials_merge_to_the_materialised_attention():
+    # the method's identity: attention computed separately over the FP8 pages and over the TQ3
+    # pages, then merged with global normalisation, is the attention over the dense
+    # materialised cache (the pages' "materialising profile")
+    pool = small_pool(seed=5, L=203, W=40)
+    pool.set_protected(0, 3, 1)
+    fmts = [f for f, _ in pool.table[0]]
+    assert P.FP8 in fmts and P.TQ3 in fmts
+    K, V = pool.dequant_seq(0)
+    L = K.shape[0]
+    rng = np.random.default_rng(6)
+    q = F.bf16_bits_to_f64(bf16_bits(rng.standard_normal((2, 6, 64), dtype=np.float32)))
+    dense = A.materialise_and_attend(pool, 0, q, 0.125)
+    parts = []
+    for fmt in (P.FP8, P.TQ3):
+        toks = [t for p, f in enumerate(fmts) if f == fmt for t in range(16 * p, min(16 * p + 16, L))]
+        parts.append(A.partial_state(K, V, q, 0.125, toks))
+    merged = A.merge(parts)
+    assert np.max(np.abs(merged - dense)) <= 1e-12 * np.max(np.abs(dense))
+
+
+def test_dequantised_sequence_matches_the_raw_slot_bytes():
+    # dequant_seq reads the stored codes; the same values must come back from each page's raw
+    # slot bytes parsed by layout, page by page in table order
+    pool = small_pool(seed=7, L=150, W=32)
+    K, V = pool.dequant_seq(0)
+    Hkv, D = pool.Hkv, pool.D
+    for p, (fmt, slot) in enumerate(pool.table[0]):
+        raw = pool.slot_bytes((fmt << 30) | slot)
+        rows = slice(16 * p, min(16 * p + 16, K.shape[0]))
+        n = rows.stop - rows.start
+        if fmt == P.FP8:
+            kc, vc, ks, vs = F.parse_fp8_slot(raw, Hkv, D)
+            kd = F.e4m3_decode(kc) * ks[:, None, None]
+            vd = F.e4m3_decode(vc) * vs[:, None, None]
+        else:
+            kq, ks, vq, vs = F.parse_tq3_slot(raw, Hkv, D)
+            kd = (kq.reshape(Hkv, 16, -1, 32) - 3.5) * ks[..., None]
+            vd = (vq.reshape(Hkv, 16, -1, 32) - 3.5) * vs[..., None]
+        assert np.array_equal(K[rows], kd.reshape(Hkv, 16, D).transpose(1, 0, 2)[:n])
+        assert np.array_equal(V[rows], vd.reshape(Hkv, 16, D).transpose(1, 0, 2)[:n])
 
 
 def test_equal_keys_give_mean_of_values():
