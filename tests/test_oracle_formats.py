@@ -180,6 +180,22 @@ def test_tq3_scale_definition_and_error_bound():
     assert np.all(err <= s[:, None] / 2 + np.maximum(amax - 3.5 * s, 0)[:, None] + 1e-12)
 
 
+def test_tq3_scale_saturates_at_the_largest_f16():
+    # fp16 holds at most 65504; plain round-to-nearest-even sends 65520 and above to infinity,
+    # the scale rule clamps instead, so a group with a huge amax keeps a finite scale
+    assert F.f16_satfinite(65504.0) == 65504.0
+    assert F.f16_satfinite(65519.99) == 65504.0
+    assert F.f16_satfinite(65520.0) == 65504.0
+    assert F.f16_satfinite(1e30) == 65504.0 and F.f16_satfinite(-1e30) == -65504.0
+    assert F.f16_satfinite(65505.0) == 65504.0          # nearest f16 (spacing 32 there)
+    x = np.zeros(32)
+    x[0], x[1], x[2], x[3] = 1e9, -1e9, 3 * 65504.0, -3 * 65504.0 - 1
+    q, s = F.tq3_quantize(x[None])
+    assert s[0] == 65504.0
+    # code = number of thresholds k * s (k = -3..3) that x reaches
+    assert q[0, 0] == 7 and q[0, 1] == 0 and q[0, 2] == 7 and q[0, 3] == 0 and q[0, 4] == 4
+
+
 def test_tq3_zero_group():
     q, s = F.tq3_quantize(np.zeros((1, 32)))
     assert s[0] == 0.0 and np.all(q == 7)
