@@ -46,7 +46,9 @@
  *
  * Errors: every int-returning call returns MKV_OK or a negative MKV_ERR_* code and sets a
  * thread-local message readable with mkv_last_error().  Host validation runs before any
- * launch; a call that fails validation leaves the pool unchanged.  Device-side checks (bad
+ * launch; a call that fails validation leaves the pool unchanged.  When several arguments of a
+ * call taking a sequence list are wrong, an out-of-range id (BAD_SEQ) is reported before any
+ * other argument error (INVALID_ARG), and those before a capacity error (OUT_OF_PAGES).  Device-side checks (bad
  * table entries, bounded waits that ran out) are recorded in the caller's status word and
  * reported by mkv_get_device_status().
  */

@@ -132,6 +132,21 @@ int check_seq(mkv_pool_t p, int32_t s) {
   return MKV_OK;
 }
 
+// Sequence-list checks shared by the calls that take one, in the documented order: every id in
+// range (BAD_SEQ) before any other argument error (INVALID_ARG: an id listed twice, a negative
+// count).  `counts` may be NULL.
+int check_seq_list(mkv_pool_t p, const int32_t* seq_ids, int32_t n, const int32_t* counts) {
+  for (int32_t i = 0; i < n; ++i)
+    if (int e = check_seq(p, seq_ids[i])) return e;
+  std::vector<uint8_t> seen(p->cfg.max_seqs, 0);
+  for (int32_t i = 0; i < n; ++i) {
+    if (seen[seq_ids[i]]) return fail(MKV_ERR_INVALID_ARG, "sequence %d listed twice", seq_ids[i]);
+    seen[seq_ids[i]] = 1;
+    if (counts && counts[i] < 0) return fail(MKV_ERR_INVALID_ARG, "negative token count");
+  }
+  return MKV_OK;
+}
+
 int validate_config(const mkv_pool_config* c) {
   if (!c) return fail(MKV_ERR_INVALID_ARG, "config is NULL");
   if (c->num_kv_heads < 1) return fail(MKV_ERR_INVALID_ARG, "num_kv_heads must be >= 1");
@@ -426,12 +441,8 @@ int mkv_append_kv(mkv_pool_t p, const int32_t* seq_ids, const int32_t* n_new, in
     return fail(MKV_ERR_INVALID_ARG, "bad sequence list");
   const int32_t MP = p->cfg.max_pages_per_seq;
   int64_t need = 0, rows = 0;
-  std::vector<uint8_t> seen(p->cfg.max_seqs, 0);
+  if (int e = check_seq_list(p, seq_ids, n_seqs, n_new)) return e;
   for (int32_t i = 0; i < n_seqs; ++i) {
-    if (int e = check_seq(p, seq_ids[i])) return e;
-    if (seen[seq_ids[i]]) return fail(MKV_ERR_INVALID_ARG, "sequence %d listed twice", seq_ids[i]);
-    seen[seq_ids[i]] = 1;
-    if (n_new[i] < 0) return fail(MKV_ERR_INVALID_ARG, "negative token count");
     const Seq& s = p->seqs[seq_ids[i]];
     const int64_t pages_after = (static_cast<int64_t>(s.ctx) + n_new[i] + kPageTokens - 1) / kPageTokens;
     if (pages_after > MP)
@@ -514,14 +525,11 @@ int mkv_demote_pages(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, int32
                      int32_t* n_demoted, void* stream) {
   if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
   if (n_seqs < 0 || (n_seqs > 0 && !seq_ids)) return fail(MKV_ERR_INVALID_ARG, "bad sequence list");
+  if (int e = check_seq_list(p, seq_ids, n_seqs, nullptr)) return e;
   if (window < 0) return fail(MKV_ERR_INVALID_ARG, "window must be >= 0");
-  std::vector<uint8_t> seen(p->cfg.max_seqs, 0);
   struct Work { int32_t seq, page; };
   std::vector<Work> work;
   for (int32_t i = 0; i < n_seqs; ++i) {
-    if (int e = check_seq(p, seq_ids[i])) return e;
-    if (seen[seq_ids[i]]) return fail(MKV_ERR_INVALID_ARG, "sequence %d listed twice", seq_ids[i]);
-    seen[seq_ids[i]] = 1;
     const Seq& s = p->seqs[seq_ids[i]];
     const int64_t L = s.ctx;
     for (int32_t pg : s.fp8_pages) {
@@ -858,7 +866,13 @@ int mkv_prefill_kv(mkv_pool_t p, const int32_t* seq_ids, const int32_t* n_tokens
   if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
   if (n_seqs < 0 || (n_seqs > 0 && (!seq_ids || !n_tokens)))
     return fail(MKV_ERR_INVALID_ARG, "bad sequence list");
+  if (int e = check_seq_list(p, seq_ids, n_seqs, n_tokens)) return e;
   if (anchor_window_tokens < 0) return fail(MKV_ERR_INVALID_ARG, "negative anchor window");
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    const Seq& s = p->seqs[seq_ids[i]];
+    if (s.ctx || !s.table.empty())
+      return fail(MKV_ERR_INVALID_ARG, "prefill needs an empty sequence (%d is not)", seq_ids[i]);
+  }
   const int32_t MP = p->cfg.max_pages_per_seq, sink = p->cfg.sink_pages;
   // page p of a prefill of n tokens is packed to TQ3 at once iff the anchor policy would demote
   // it: p >= sink and 16p + 16 <= n - W (new pages carry no protection)
@@ -866,15 +880,7 @@ int mkv_prefill_kv(mkv_pool_t p, const int32_t* seq_ids, const int32_t* n_tokens
     return pg >= sink && kPageTokens * pg + kPageTokens <= n - anchor_window_tokens;
   };
   int64_t need[2] = {0, 0}, rows = 0;
-  std::vector<uint8_t> seen(p->cfg.max_seqs, 0);
   for (int32_t i = 0; i < n_seqs; ++i) {
-    if (int e = check_seq(p, seq_ids[i])) return e;
-    if (seen[seq_ids[i]]) return fail(MKV_ERR_INVALID_ARG, "sequence %d listed twice", seq_ids[i]);
-    seen[seq_ids[i]] = 1;
-    if (n_tokens[i] < 0) return fail(MKV_ERR_INVALID_ARG, "negative token count");
-    const Seq& s = p->seqs[seq_ids[i]];
-    if (s.ctx || !s.table.empty())
-      return fail(MKV_ERR_INVALID_ARG, "prefill needs an empty sequence (%d is not)", seq_ids[i]);
     const int64_t pages = (static_cast<int64_t>(n_tokens[i]) + kPageTokens - 1) / kPageTokens;
     if (pages > MP)
       return fail(MKV_ERR_OUT_OF_PAGES, "sequence %d would need %lld pages > %d", seq_ids[i],
