@@ -4,9 +4,9 @@ demotion counts after every operation, and the same error (with nothing changed)
 them rejects an operation.
 
 The streams mix appends of random sizes (sometimes over a sequence's page limit or the FP8
-slab), protection flags, demotions with random windows, prefill of empty sequences, copies and
-resets, with repeated and out-of-range sequence ids among them.  Every tenth step the decode
-cut of the live sequences is checked as in test_plan."""
+slab), protection flags, demotions with random windows, prefill of empty sequences, copies,
+resets and new slot orders, with repeated and out-of-range sequence ids among them.  Every
+tenth step the decode cut of the live sequences is checked as in test_plan."""
 import numpy as np
 import pytest
 
@@ -72,7 +72,7 @@ def test_random_operation_streams_match_the_oracle(seed):
 
     for step in range(250):
         kind = rng.choice(["append", "append", "append", "protect", "demote", "demote",
-                           "prefill", "copy", "reset"])
+                           "prefill", "copy", "reset", "order"])
         LAST_OP[0] = kind
         if kind == "append":
             ids = seqs()
@@ -103,9 +103,15 @@ def test_random_operation_streams_match_the_oracle(seed):
         elif kind == "copy":
             src, dst = (int(x) for x in rng.integers(0, n_seqs, size=2))
             both(lambda: lp.copy(src, dst), lambda: op.seq_copy(src, dst))
-        else:
+        elif kind == "reset":
             s = int(rng.integers(0, n_seqs))
             both(lambda: lp.reset(s), lambda: op.seq_reset(s))
+        else:
+            fmt, n = (P.FP8, fp8_slots) if rng.random() < 0.5 else (P.TQ3, tq3_slots)
+            order = rng.permutation(n).tolist()
+            if n > 1 and rng.random() < 0.1:
+                order[0] = order[1]                       # not a permutation
+            both(lambda: lp.set_slot_order(fmt, order), lambda: op.set_slot_order(fmt, order))
         state(lp, op, n_seqs)
         if step % 10 == 9:
             # the decode cut of every non-empty sequence covers its pages once
