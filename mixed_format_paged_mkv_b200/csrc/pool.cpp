@@ -317,6 +317,10 @@ int plan_decode(mkv_pool_t p, const int32_t* seq_ids, int32_t n, int32_t q_len, 
     plan->cost.push_back(cost);
     return true;
   });
+  for (int32_t i = 0; i < n; ++i)
+    if (np[i] > kDecodeMaxUnits)
+      return fail(MKV_ERR_UNSUPPORTED, "sequence %d needs %d work units; one launch holds %d",
+                  seq_ids[i], np[i], kDecodeMaxUnits);
   int64_t parts = 0;
   for (int32_t i = 0; i < n; ++i) {
     SeqDesc& d = plan->seq[i];

@@ -172,3 +172,19 @@ def test_plan_count_query_and_small_buffer():
         pool.decode_plan(seqs, 1, 3)          # 3 query heads over 2 KV heads
     with pytest.raises(MkvError):
         pool.decode_plan([0, 0, 5], 1, 2)     # sequence outside the pool
+
+
+def test_a_sequence_beyond_one_launch_is_rejected():
+    # 512 pages per unit at most and 1536 units per launch: a sequence of 786,433+ pages of one
+    # format cannot be decoded in one launch group, and the planner says so up front
+    pages = 1536 * 512 + 1
+    pool = Pool(1, 64, 1, pages, pages, 1, host_only=True)
+    pool.append([0], [16 * pages])
+    from mixed_format_paged_mkv_b200.api import MkvError
+    with pytest.raises(MkvError) as e:
+        pool.decode_plan([0], 1, 1)
+    assert e.value.name == "UNSUPPORTED"
+    pool.reset(0)
+    pool.append([0], [16 * (pages - 1)])
+    units, _ = pool.decode_plan([0], 1, 1)
+    assert len(units) == 1536 and units[:, 4].max() == 512
