@@ -179,8 +179,9 @@ MKV_API int mkv_decode_plan(mkv_pool_t pool, const int32_t* seq_ids, int32_t n_s
  *   q_bf16    device bf16 [n_seqs][q_len][num_q_heads][D]
  *   out       device fp32 [n_seqs][q_len][num_q_heads][D]
  *   workspace device scratch of ws_bytes >= mkv_decode_workspace_bytes(...), 256-B aligned
- * Constraints: num_q_heads % Hkv == 0, q_len * (num_q_heads / Hkv) <= 32,
- * n_seqs <= max_seqs (rows may repeat).
+ * Constraints: num_q_heads % Hkv == 0, q_len * (num_q_heads / Hkv) <= 32 (else UNSUPPORTED),
+ * n_seqs <= max_seqs (rows may repeat), at most 1536 x 512 pages of one format per sequence
+ * (else UNSUPPORTED: one launch group holds 1536 work units of at most 512 pages).
  * Errors: BAD_SEQ, EMPTY_CONTEXT, INVALID_ARG, UNSUPPORTED, WORKSPACE_TOO_SMALL, CUDA. */
 MKV_API int mkv_decode_attention(mkv_pool_t pool, const int32_t* seq_ids, int32_t n_seqs,
                                  int32_t q_len, const void* q_bf16, int32_t num_q_heads,
