@@ -232,6 +232,16 @@ def build_pool(w, layers, extra_pages, device):
     return pool
 
 
+def host_plan_us(pool, seq_ids, q_len, hq, reps=50):
+    """Host time of planning one decode call (the work-unit cut), microseconds per call, measured
+    after the timed region through the workspace query, which runs the same planner."""
+    pool.workspace_bytes(seq_ids, q_len, hq)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        pool.workspace_bytes(seq_ids, q_len, hq)
+    return round((time.perf_counter() - t0) / reps * 1e6, 1)
+
+
 def step_inputs_host(w, layers, steps, first_step):
     """[steps][layers] of (k, v, q) uint16 arrays stacked as k [S, Ly, B, Hkv, D] etc."""
     K = np.empty((steps, layers, w.B, w.Hkv, w.D), np.uint16)
@@ -395,6 +405,7 @@ def run_gpu(args, rank, world, local_rank):
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
         "build_s": round(build_s, 1),
+        "host_plan_us_per_call": host_plan_us(pool, seq_ids[0], w.q_len, w.Hq),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         gbs, per, runs, cores, desc = oracle_sample(w, target_s=args.cpu_seconds)
