@@ -48,6 +48,24 @@ def test_e4m3_golden_vectors():
         assert int(F.e4m3_encode(float(val))) == int(code, 16), line
 
 
+def test_fp8_page_write_golden_vectors():
+    codes = np.zeros((16, 4), dtype=np.uint8)
+    scale = 0.0
+    lines = [l for l in _golden_lines("fp8_page_vectors.txt")]
+    assert len(lines) == 8
+    for wl, el in zip(lines[0::2], lines[1::2]):
+        head, vals = wl.split(":")
+        assert head.split()[0] == "write"
+        n_old = int(head.split()[1])
+        x = np.array([[float(v) for v in vals.split()]])
+        codes, scale = F.fp8_write(codes, scale, n_old, x)
+        ehead, rows = el.split(":")
+        assert float(ehead.split()[1]) == scale, wl
+        want = [[int(c, 16) for c in r.split()] for r in rows.split("|")]
+        assert codes[:len(want)].tolist() == want, wl
+        assert not codes[len(want):].any()
+
+
 def _brute_nearest(x):
     """Nearest finite E4M3 value by exhaustive search; ties -> even code; saturating."""
     best = None
