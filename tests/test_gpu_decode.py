@@ -184,3 +184,33 @@ def test_corrupted_device_table_entry_is_flagged():
     assert e.value.name == "DEVICE_CHECK"
     tables[idx] = good
     run_and_check(w, lp=lp)
+
+
+def test_decode_argument_errors_are_caught_before_any_launch():
+    """A workspace below the planned size, a workspace that is not 256-byte aligned and a
+    non-finite sm_scale are rejected by the host before anything is launched; the pool then
+    decodes normally."""
+    from mixed_format_paged_mkv_b200 import MkvError
+    w = Workload("args", 31, B=2, Hq=4, Hkv=2, D=128, q_len=1, window=16, ctx=(300, 45))
+    lp = lib_pool(w)
+    op = oracle_pool(w)
+    seqs = [0, 1]
+    q = q_tensor(w)
+    need = lp.workspace_bytes(seqs, 1, w.Hq)
+    launches = lp.launch_count()
+    small = torch.empty(need // 2, dtype=torch.uint8, device="cuda")
+    with pytest.raises(MkvError) as e:
+        lp.decode(seqs, q, workspace=small)
+    assert e.value.name == "WORKSPACE_TOO_SMALL"
+    big = torch.empty(need + 512, dtype=torch.uint8, device="cuda")
+    with pytest.raises(MkvError) as e:
+        lp.decode(seqs, q, workspace=big[16:])
+    assert e.value.name == "INVALID_ARG"
+    with pytest.raises(MkvError) as e:
+        lp.decode(seqs, q, sm_scale=float("nan"), workspace=big)
+    assert e.value.name == "INVALID_ARG"
+    assert lp.launch_count() == launches
+    out = lp.decode(seqs, q, workspace=big).cpu().numpy()
+    lp.device_status()
+    for s in seqs:
+        assert_close(out[s], oracle_decode(op, w, s), what=f"seq {s}")
