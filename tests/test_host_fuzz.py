@@ -15,7 +15,6 @@ from oracle import pool as P
 
 from test_plan import check_cut
 
-HKV, D = 1, 64
 LAST_OP = [None]   # named in assertion messages
 
 
@@ -48,6 +47,7 @@ def both(fn_lib, fn_ora):
 
 @pytest.mark.parametrize("seed", range(8))
 def test_random_operation_streams_match_the_oracle(seed):
+    HKV, D = [(1, 64), (2, 128), (4, 256)][seed % 3]
     rng = np.random.default_rng(1000 + seed)
     n_seqs = int(rng.integers(2, 6))
     max_pages = int(rng.integers(3, 12))
