@@ -46,7 +46,14 @@
  *
  * Errors: every int-returning call returns MKV_OK or a negative MKV_ERR_* code and sets a
  * thread-local message readable with mkv_last_error().  Host validation runs before any
- * launch; a call that fails validation leaves the pool unchanged.  When several arguments of a
+ * launch; a call that fails validation leaves the pool unchanged.  A call whose launch fails
+ * (MKV_ERR_CUDA) leaves the pool's host state -- tables, free slots, lengths, flags -- unchanged
+ * too: state changes are staged and committed after the call's last launch.  On the device, a
+ * call issued as one launch either ran or did not; a call so large that it is split into several
+ * launches may, when a later one fails, have written pages into slots that stay free and, for
+ * an append, have re-encoded existing partial pages (rescale-on-grow): reset the sequences of
+ * such a call.  A split demotion publishes no table entry before all its pages are written.
+ * When several arguments of a
  * call taking a sequence list are wrong, an out-of-range id (BAD_SEQ) is reported before any
  * other argument error (INVALID_ARG), and those before a capacity error (OUT_OF_PAGES).  Device-side checks (bad
  * table entries, bounded waits that ran out) are recorded in the caller's status word and
@@ -290,6 +297,14 @@ MKV_API int mkv_get_device_status(mkv_pool_t pool, void* stream);
 MKV_API int mkv_timing_enable(mkv_pool_t pool, int32_t enable);
 MKV_API int mkv_timing_read(mkv_pool_t pool, double* ms_partial, double* ms_merge,
                             int64_t* calls);
+
+/* Test hook for the error paths (no counterpart in the pages): after `after` more device
+ * operations of the state-changing calls (append, prefill, demotion, copy, reset: each kernel
+ * launch or memset they issue; on a host-only pool each one they would issue) succeed, the next
+ * one reports MKV_ERR_CUDA without being issued, and the hook switches itself off.  -1 switches
+ * it off.  Lets a test make a launch fail on the host, with no device fault, and check that the
+ * failed call left the pool's host state unchanged.  Errors: INVALID_ARG. */
+MKV_API int mkv_test_fail_launch(mkv_pool_t pool, int32_t after);
 
 /* Number of kernels this pool has launched since creation. */
 MKV_API int mkv_launch_count(mkv_pool_t pool, int64_t* launches);

@@ -68,6 +68,7 @@ SIGNATURES = {
                                        ctypes.POINTER(ctypes.c_double),
                                        ctypes.POINTER(ctypes.c_int64)]),
     "mkv_launch_count": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int64)]),
+    "mkv_test_fail_launch": (ctypes.c_int, [_P, _I32]),
     "mkv_last_error": (ctypes.c_char_p, []),
 }
 
@@ -347,6 +348,10 @@ class Pool:
         _check(lib().mkv_timing_read(self.handle, ctypes.byref(v[0]), ctypes.byref(v[1]),
                                      ctypes.byref(n)), "mkv_timing_read")
         return dict(partial_ms=v[0].value, merge_ms=v[1].value, calls=n.value)
+
+    def test_fail_launch(self, after):
+        """Make the device operation after the next ``after`` ones fail (test hook; -1: off)."""
+        _check(lib().mkv_test_fail_launch(self.handle, int(after)), "mkv_test_fail_launch")
 
     def launch_count(self):
         n = ctypes.c_int64()

@@ -130,8 +130,13 @@ __global__ void __launch_bounds__(256) demote_kernel(const __grid_constant__ Dem
     const float x = __fmul_rn(e4m3_to_float(code), scales[which]);
     pack_group(x, lane, dst + which * (G * kPageTokens * 14), G, grp, t);
   }
-  if (h == 0 && threadIdx.x == 0)
+  if (p.publish && h == 0 && threadIdx.x == 0)
     p.tables[d.table_index] = static_cast<int32_t>((1u << kFmtShift) | static_cast<uint32_t>(d.dst_slot));
+}
+
+__global__ void __launch_bounds__(256) retag_kernel(const __grid_constant__ RetagParams p) {
+  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < p.n; k += gridDim.x * blockDim.x)
+    p.tables[p.index[k]] = p.entry[k];
 }
 
 // Prefill: a full page packed to TQ3 straight from the bf16 input rows (the values are exact in
@@ -248,6 +253,12 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
 cudaError_t launch_demote(const DemoteParams& p, cudaStream_t s) {
   if (p.n_desc <= 0) return cudaSuccess;
   demote_kernel<<<dim3(p.n_desc, p.Hkv), 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_retag(const RetagParams& p, cudaStream_t s) {
+  if (p.n <= 0) return cudaSuccess;
+  retag_kernel<<<(p.n + 255) / 256, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 

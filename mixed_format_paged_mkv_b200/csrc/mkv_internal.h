@@ -56,8 +56,20 @@ struct DemoteParams {
   int32_t* tables;
   int64_t fp8_slot_bytes, tq3_slot_bytes;
   int32_t Hkv, D;
+  int32_t publish;  // 1: also set each page's table entry to TQ3 (else a retag launch does)
   int32_t n_desc;
   DemoteDesc desc[kDemoteMaxDesc];
+};
+
+// ------------------------------------------------------------------ table retag
+// tables[index[k]] = entry[k]: publishes the entries of a demotion split over several launches
+// once every page is written.
+constexpr int kRetagMax = 3800;
+struct RetagParams {
+  int32_t* tables;
+  int32_t n;
+  int32_t index[kRetagMax];
+  int32_t entry[kRetagMax];
 };
 
 // ------------------------------------------------------------------ prefill (bf16 -> TQ3)
@@ -150,6 +162,7 @@ struct DecodeParams {
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 cudaError_t launch_demote(const DemoteParams& p, cudaStream_t s);
+cudaError_t launch_retag(const RetagParams& p, cudaStream_t s);
 cudaError_t launch_copy(const CopyParams& p, cudaStream_t s);
 cudaError_t launch_materialise(const MaterialiseParams& p, cudaStream_t s);
 cudaError_t launch_pack(const PackParams& p, cudaStream_t s);

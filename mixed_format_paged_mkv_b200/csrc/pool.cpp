@@ -117,6 +117,7 @@ struct mkv_pool {
   std::vector<Seq> seqs;
   Allocator alloc[2];
   int64_t launches = 0;
+  int64_t fail_after = -1;  // test hook: device operations that still succeed before one fails
   bool timing = false;
   std::vector<TimingRec> timing_recs;
   std::vector<cudaEvent_t> spare_events;
@@ -341,6 +342,23 @@ int plan_decode(mkv_pool_t p, const int32_t* seq_ids, int32_t n, int32_t q_len, 
   return MKV_OK;
 }
 
+// Every device operation of a state-changing call (kernel launch or memset) goes through here:
+// the test hook can make it fail, host-only pools skip it, and launches are counted.  The calls
+// stage their host-state changes and commit them only after all their device operations were
+// issued, so a failure here leaves the pool's host state as it was before the call.
+template <class F>
+int device_op(mkv_pool_t p, const char* what, F&& f) {
+  if (p->fail_after == 0) {
+    p->fail_after = -1;
+    return fail(MKV_ERR_CUDA, "%s: launch failure injected by mkv_test_fail_launch", what);
+  }
+  if (p->fail_after > 0) --p->fail_after;
+  if (p->host_only) return MKV_OK;
+  ++p->launches;
+  const cudaError_t e = f();
+  return e == cudaSuccess ? MKV_OK : cuda_fail(e, what);
+}
+
 cudaEvent_t get_event(mkv_pool_t p) {
   if (!p->spare_events.empty()) {
     cudaEvent_t e = p->spare_events.back();
@@ -462,24 +480,22 @@ int mkv_append_kv(mkv_pool_t p, const int32_t* seq_ids, const int32_t* n_new, in
     return fail(MKV_ERR_INVALID_ARG, "k/v are NULL");
   if (rows > INT32_MAX) return fail(MKV_ERR_INVALID_ARG, "too many tokens");
 
-  // ---- commit host state, collect page writes
+  // ---- stage: new FP8 slots and the page writes, against the tables as they will be
+  std::vector<int32_t> taken;      // new slots, sequences in order, pages ascending
+  std::vector<size_t> first_new(n_seqs);
   std::vector<AppendDesc> descs;
   int32_t row = 0;
   for (int32_t i = 0; i < n_seqs; ++i) {
-    Seq& s = p->seqs[seq_ids[i]];
-    const int32_t L0 = s.ctx, n = n_new[i];
+    const Seq& s = p->seqs[seq_ids[i]];
+    const int32_t L0 = s.ctx, n = n_new[i], before = static_cast<int32_t>(s.table.size());
     const int32_t pages_after = (L0 + n + kPageTokens - 1) / kPageTokens;
-    if (s.prot.size() < static_cast<size_t>(pages_after)) s.prot.resize(pages_after, 0);
-    while (static_cast<int32_t>(s.table.size()) < pages_after) {
-      const int32_t slot = p->alloc[0].take();
-      s.fp8_pages.push_back(static_cast<int32_t>(s.table.size()));
-      s.table.push_back(entry_of(MKV_FMT_FP8, slot));
-    }
+    first_new[i] = taken.size();
+    for (int32_t pg = before; pg < pages_after; ++pg) taken.push_back(p->alloc[0].take());
     for (int32_t t = 0; t < n;) {
       const int32_t pos = L0 + t, page = pos / kPageTokens, off = pos % kPageTokens;
       const int32_t cnt = std::min(kPageTokens - off, n - t);
       AppendDesc d;
-      d.slot = slot_of(s.table[page]);
+      d.slot = page < before ? slot_of(s.table[page]) : taken[first_new[i] + (page - before)];
       d.table_index = seq_ids[i] * MP + page;
       d.first_row = row + t;
       d.n_old = static_cast<int16_t>(off);
@@ -487,31 +503,43 @@ int mkv_append_kv(mkv_pool_t p, const int32_t* seq_ids, const int32_t* n_new, in
       descs.push_back(d);
       t += cnt;
     }
-    s.ctx = L0 + n;
     row += n;
   }
-  if (p->host_only) return ok();
-  AppendParams* prm = new AppendParams;
-  prm->fp8_slab = p->fp8_slab;
-  prm->tables = p->d_tables;
-  prm->status = p->d_status;
-  prm->k = static_cast<const uint16_t*>(k_bf16);
-  prm->v = static_cast<const uint16_t*>(v_bf16);
-  prm->slot_bytes = p->fp8_slot_bytes;
-  prm->Hkv = p->cfg.num_kv_heads;
-  prm->D = p->cfg.head_dim;
-  for (size_t b = 0; b < descs.size(); b += kAppendMaxDesc) {
-    const size_t m = std::min<size_t>(kAppendMaxDesc, descs.size() - b);
-    prm->n_desc = static_cast<int32_t>(m);
-    std::memcpy(prm->desc, descs.data() + b, m * sizeof(AppendDesc));
-    cudaError_t e = launch_append(*prm, as_stream(stream));
-    ++p->launches;
-    if (e != cudaSuccess) {
-      delete prm;
-      return cuda_fail(e, "append launch");
+  // ---- launch
+  int rc = MKV_OK;
+  if (!descs.empty()) {
+    AppendParams* prm = new AppendParams;
+    prm->fp8_slab = p->fp8_slab;
+    prm->tables = p->d_tables;
+    prm->status = p->d_status;
+    prm->k = static_cast<const uint16_t*>(k_bf16);
+    prm->v = static_cast<const uint16_t*>(v_bf16);
+    prm->slot_bytes = p->fp8_slot_bytes;
+    prm->Hkv = p->cfg.num_kv_heads;
+    prm->D = p->cfg.head_dim;
+    for (size_t b = 0; b < descs.size() && rc == MKV_OK; b += kAppendMaxDesc) {
+      const size_t m = std::min<size_t>(kAppendMaxDesc, descs.size() - b);
+      prm->n_desc = static_cast<int32_t>(m);
+      std::memcpy(prm->desc, descs.data() + b, m * sizeof(AppendDesc));
+      rc = device_op(p, "append launch", [&] { return launch_append(*prm, as_stream(stream)); });
     }
+    delete prm;
   }
-  delete prm;
+  if (rc != MKV_OK) {
+    for (auto it = taken.rbegin(); it != taken.rend(); ++it) p->alloc[0].give(*it);
+    return rc;
+  }
+  // ---- commit
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    Seq& s = p->seqs[seq_ids[i]];
+    const int32_t pages_after = (s.ctx + n_new[i] + kPageTokens - 1) / kPageTokens;
+    if (s.prot.size() < static_cast<size_t>(pages_after)) s.prot.resize(pages_after, 0);
+    for (size_t k = first_new[i]; static_cast<int32_t>(s.table.size()) < pages_after; ++k) {
+      s.fp8_pages.push_back(static_cast<int32_t>(s.table.size()));
+      s.table.push_back(entry_of(MKV_FMT_FP8, taken[k]));
+    }
+    s.ctx += n_new[i];
+  }
   return ok();
 }
 
@@ -527,6 +555,7 @@ int mkv_set_protected(mkv_pool_t p, int32_t seq, int32_t page, int32_t flag) {
 
 int mkv_demote_pages(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, int32_t window,
                      int32_t* n_demoted, void* stream) {
+  if (n_demoted) *n_demoted = 0;
   if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
   if (n_seqs < 0 || (n_seqs > 0 && !seq_ids)) return fail(MKV_ERR_INVALID_ARG, "bad sequence list");
   if (int e = check_seq_list(p, seq_ids, n_seqs, nullptr)) return e;
@@ -546,26 +575,20 @@ int mkv_demote_pages(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, int32
   }
   if (static_cast<int64_t>(work.size()) > p->alloc[1].n_free)
     return fail(MKV_ERR_OUT_OF_PAGES, "TQ3 slab has %d free slots, %zu needed", p->alloc[1].n_free, work.size());
+  // ---- stage: a TQ3 slot per page, in (sequence, page) order
   std::vector<DemoteDesc> descs;
-  std::vector<int32_t> freed;
   descs.reserve(work.size());
   for (const Work& w : work) {
-    Seq& s = p->seqs[w.seq];
-    const int32_t src = slot_of(s.table[w.page]);
-    const int32_t dst = p->alloc[1].take();
-    s.table[w.page] = entry_of(MKV_FMT_TQ3, dst);
-    s.n3 += 1;
-    descs.push_back({src, dst, w.seq * p->cfg.max_pages_per_seq + w.page});
-    freed.push_back(src);
+    const Seq& s = p->seqs[w.seq];
+    descs.push_back({slot_of(s.table[w.page]), p->alloc[1].take(),
+                     w.seq * p->cfg.max_pages_per_seq + w.page});
   }
-  for (int32_t i = 0; i < n_seqs; ++i) {
-    Seq& s = p->seqs[seq_ids[i]];
-    s.fp8_pages.erase(std::remove_if(s.fp8_pages.begin(), s.fp8_pages.end(),
-                                     [&](int32_t pg) { return fmt_of(s.table[pg]) != MKV_FMT_FP8; }),
-                      s.fp8_pages.end());
-  }
-  if (n_demoted) *n_demoted = static_cast<int32_t>(descs.size());
-  if (!p->host_only && !descs.empty()) {
+  // ---- launch: one launch writes the pages and publishes their table entries; a call that
+  // needs several launches publishes no entry until every page is written (retag launches
+  // last), so a failed launch never leaves a device entry naming an unwritten page
+  int rc = MKV_OK;
+  if (!descs.empty()) {
+    const bool single = descs.size() <= static_cast<size_t>(kDemoteMaxDesc);
     DemoteParams* prm = new DemoteParams;
     prm->fp8_slab = p->fp8_slab;
     prm->tq3_slab = p->tq3_slab;
@@ -574,21 +597,47 @@ int mkv_demote_pages(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, int32
     prm->tq3_slot_bytes = p->tq3_slot_bytes;
     prm->Hkv = p->cfg.num_kv_heads;
     prm->D = p->cfg.head_dim;
-    for (size_t b = 0; b < descs.size(); b += kDemoteMaxDesc) {
+    prm->publish = single ? 1 : 0;
+    for (size_t b = 0; b < descs.size() && rc == MKV_OK; b += kDemoteMaxDesc) {
       const size_t m = std::min<size_t>(kDemoteMaxDesc, descs.size() - b);
       prm->n_desc = static_cast<int32_t>(m);
       std::memcpy(prm->desc, descs.data() + b, m * sizeof(DemoteDesc));
-      cudaError_t e = launch_demote(*prm, as_stream(stream));
-      ++p->launches;
-      if (e != cudaSuccess) {
-        delete prm;
-        for (int32_t s : freed) p->alloc[0].give(s);
-        return cuda_fail(e, "demote launch");
-      }
+      rc = device_op(p, "demote launch", [&] { return launch_demote(*prm, as_stream(stream)); });
     }
     delete prm;
+    if (!single && rc == MKV_OK) {
+      RetagParams* rp = new RetagParams;
+      rp->tables = p->d_tables;
+      for (size_t b = 0; b < descs.size() && rc == MKV_OK; b += kRetagMax) {
+        const size_t m = std::min<size_t>(kRetagMax, descs.size() - b);
+        rp->n = static_cast<int32_t>(m);
+        for (size_t k = 0; k < m; ++k) {
+          rp->index[k] = descs[b + k].table_index;
+          rp->entry[k] = entry_of(MKV_FMT_TQ3, descs[b + k].dst_slot);
+        }
+        rc = device_op(p, "retag launch", [&] { return launch_retag(*rp, as_stream(stream)); });
+      }
+      delete rp;
+    }
   }
-  for (int32_t s : freed) p->alloc[0].give(s);
+  if (rc != MKV_OK) {
+    for (auto it = descs.rbegin(); it != descs.rend(); ++it) p->alloc[1].give(it->dst_slot);
+    return rc;
+  }
+  // ---- commit: retag, then free the FP8 slots (reusable by later calls in stream order)
+  for (size_t k = 0; k < work.size(); ++k) {
+    Seq& s = p->seqs[work[k].seq];
+    s.table[work[k].page] = entry_of(MKV_FMT_TQ3, descs[k].dst_slot);
+    s.n3 += 1;
+  }
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    Seq& s = p->seqs[seq_ids[i]];
+    s.fp8_pages.erase(std::remove_if(s.fp8_pages.begin(), s.fp8_pages.end(),
+                                     [&](int32_t pg) { return fmt_of(s.table[pg]) != MKV_FMT_FP8; }),
+                      s.fp8_pages.end());
+  }
+  for (const DemoteDesc& d : descs) p->alloc[0].give(d.src_slot);
+  if (n_demoted) *n_demoted = static_cast<int32_t>(descs.size());
   return ok();
 }
 
@@ -832,13 +881,15 @@ int mkv_seq_reset(mkv_pool_t p, int32_t seq, void* stream) {
   if (int e = check_seq(p, seq)) return e;
   Seq& s = p->seqs[seq];
   const size_t n = s.table.size();
+  if (n > 0) {
+    const int rc = device_op(p, "reset", [&] {
+      return cudaMemsetAsync(p->d_tables + static_cast<int64_t>(seq) * p->cfg.max_pages_per_seq,
+                             0xFF, n * 4, as_stream(stream));
+    });
+    if (rc != MKV_OK) return rc;
+  }
   for (int32_t e : s.table) p->alloc[fmt_of(e)].give(slot_of(e));
   s = Seq();
-  if (!p->host_only && n > 0) {
-    cudaError_t e = cudaMemsetAsync(p->d_tables + static_cast<int64_t>(seq) * p->cfg.max_pages_per_seq,
-                                    0xFF, n * 4, as_stream(stream));
-    if (e != cudaSuccess) return cuda_fail(e, "reset");
-  }
   return ok();
 }
 
@@ -900,26 +951,22 @@ int mkv_prefill_kv(mkv_pool_t p, const int32_t* seq_ids, const int32_t* n_tokens
     return fail(MKV_ERR_INVALID_ARG, "k/v are NULL");
   if (rows > INT32_MAX) return fail(MKV_ERR_INVALID_ARG, "too many tokens");
 
-  // ---- commit host state: pages ascending, each taking a slot of its own format
+  // ---- stage: pages ascending, each taking a slot of its own format
+  std::vector<int32_t> taken[2];   // slots per format, in the order taken
   std::vector<AppendDesc> fp8_descs;
   std::vector<PackDesc> tq3_descs;
   int32_t row = 0;
   for (int32_t i = 0; i < n_seqs; ++i) {
-    Seq& s = p->seqs[seq_ids[i]];
     const int32_t n = n_tokens[i], pages = (n + kPageTokens - 1) / kPageTokens;
-    s.prot.assign(pages, 0);
     for (int32_t pg = 0; pg < pages; ++pg) {
       const int32_t first_row = row + kPageTokens * pg;
       const int32_t table_index = seq_ids[i] * MP + pg;
-      if (direct(pg, n)) {
-        const int32_t slot = p->alloc[1].take();
-        s.table.push_back(entry_of(MKV_FMT_TQ3, slot));
-        ++s.n3;
+      const int f = direct(pg, n) ? 1 : 0;
+      const int32_t slot = p->alloc[f].take();
+      taken[f].push_back(slot);
+      if (f == 1) {
         tq3_descs.push_back({slot, table_index, first_row});
       } else {
-        const int32_t slot = p->alloc[0].take();
-        s.fp8_pages.push_back(pg);
-        s.table.push_back(entry_of(MKV_FMT_FP8, slot));
         AppendDesc d;
         d.slot = slot;
         d.table_index = table_index;
@@ -929,46 +976,66 @@ int mkv_prefill_kv(mkv_pool_t p, const int32_t* seq_ids, const int32_t* n_tokens
         fp8_descs.push_back(d);
       }
     }
-    s.ctx = n;
     row += n;
   }
-  if (p->host_only) return ok();
+  // ---- launch (new pages only: their table entries were unmapped, so entries published by an
+  // earlier launch of a failed call are ignored and later overwritten)
   cudaStream_t st = as_stream(stream);
-  AppendParams* ap = new AppendParams;
-  ap->fp8_slab = p->fp8_slab;
-  ap->tables = p->d_tables;
-  ap->status = p->d_status;
-  ap->k = static_cast<const uint16_t*>(k_bf16);
-  ap->v = static_cast<const uint16_t*>(v_bf16);
-  ap->slot_bytes = p->fp8_slot_bytes;
-  ap->Hkv = p->cfg.num_kv_heads;
-  ap->D = p->cfg.head_dim;
-  cudaError_t e = cudaSuccess;
-  for (size_t b = 0; b < fp8_descs.size() && e == cudaSuccess; b += kAppendMaxDesc) {
-    const size_t m = std::min<size_t>(kAppendMaxDesc, fp8_descs.size() - b);
-    ap->n_desc = static_cast<int32_t>(m);
-    std::memcpy(ap->desc, fp8_descs.data() + b, m * sizeof(AppendDesc));
-    e = launch_append(*ap, st);
-    ++p->launches;
+  int rc = MKV_OK;
+  if (!fp8_descs.empty()) {
+    AppendParams* ap = new AppendParams;
+    ap->fp8_slab = p->fp8_slab;
+    ap->tables = p->d_tables;
+    ap->status = p->d_status;
+    ap->k = static_cast<const uint16_t*>(k_bf16);
+    ap->v = static_cast<const uint16_t*>(v_bf16);
+    ap->slot_bytes = p->fp8_slot_bytes;
+    ap->Hkv = p->cfg.num_kv_heads;
+    ap->D = p->cfg.head_dim;
+    for (size_t b = 0; b < fp8_descs.size() && rc == MKV_OK; b += kAppendMaxDesc) {
+      const size_t m = std::min<size_t>(kAppendMaxDesc, fp8_descs.size() - b);
+      ap->n_desc = static_cast<int32_t>(m);
+      std::memcpy(ap->desc, fp8_descs.data() + b, m * sizeof(AppendDesc));
+      rc = device_op(p, "prefill launch", [&] { return launch_append(*ap, st); });
+    }
+    delete ap;
   }
-  delete ap;
-  PackParams* pp = new PackParams;
-  pp->k = static_cast<const uint16_t*>(k_bf16);
-  pp->v = static_cast<const uint16_t*>(v_bf16);
-  pp->tq3_slab = p->tq3_slab;
-  pp->tables = p->d_tables;
-  pp->tq3_slot_bytes = p->tq3_slot_bytes;
-  pp->Hkv = p->cfg.num_kv_heads;
-  pp->D = p->cfg.head_dim;
-  for (size_t b = 0; b < tq3_descs.size() && e == cudaSuccess; b += kPackMaxDesc) {
-    const size_t m = std::min<size_t>(kPackMaxDesc, tq3_descs.size() - b);
-    pp->n_desc = static_cast<int32_t>(m);
-    std::memcpy(pp->desc, tq3_descs.data() + b, m * sizeof(PackDesc));
-    e = launch_pack(*pp, st);
-    ++p->launches;
+  if (!tq3_descs.empty() && rc == MKV_OK) {
+    PackParams* pp = new PackParams;
+    pp->k = static_cast<const uint16_t*>(k_bf16);
+    pp->v = static_cast<const uint16_t*>(v_bf16);
+    pp->tq3_slab = p->tq3_slab;
+    pp->tables = p->d_tables;
+    pp->tq3_slot_bytes = p->tq3_slot_bytes;
+    pp->Hkv = p->cfg.num_kv_heads;
+    pp->D = p->cfg.head_dim;
+    for (size_t b = 0; b < tq3_descs.size() && rc == MKV_OK; b += kPackMaxDesc) {
+      const size_t m = std::min<size_t>(kPackMaxDesc, tq3_descs.size() - b);
+      pp->n_desc = static_cast<int32_t>(m);
+      std::memcpy(pp->desc, tq3_descs.data() + b, m * sizeof(PackDesc));
+      rc = device_op(p, "prefill launch", [&] { return launch_pack(*pp, st); });
+    }
+    delete pp;
   }
-  delete pp;
-  if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+  if (rc != MKV_OK) {
+    for (int f = 0; f < 2; ++f)
+      for (auto it = taken[f].rbegin(); it != taken[f].rend(); ++it) p->alloc[f].give(*it);
+    return rc;
+  }
+  // ---- commit
+  size_t next[2] = {0, 0};
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    Seq& s = p->seqs[seq_ids[i]];
+    const int32_t n = n_tokens[i], pages = (n + kPageTokens - 1) / kPageTokens;
+    s.prot.assign(pages, 0);
+    for (int32_t pg = 0; pg < pages; ++pg) {
+      const int f = direct(pg, n) ? 1 : 0;
+      s.table.push_back(entry_of(f, taken[f][next[f]++]));
+      if (f == 1) ++s.n3;
+      else s.fp8_pages.push_back(pg);
+    }
+    s.ctx = n;
+  }
   return ok();
 }
 
@@ -1014,6 +1081,7 @@ int mkv_seq_copy(mkv_pool_t p, int32_t src, int32_t dst, void* stream) {
   for (int32_t e : s.table) need[fmt_of(e)]++;
   for (int f = 0; f < 2; ++f)
     if (need[f] > p->alloc[f].n_free) return fail(MKV_ERR_OUT_OF_PAGES, "slab %d exhausted", f);
+  // ---- stage: a slot of the same format per page, pages ascending
   Seq d;
   d.ctx = s.ctx;
   d.prot = s.prot;
@@ -1026,26 +1094,28 @@ int mkv_seq_copy(mkv_pool_t p, int32_t src, int32_t dst, void* stream) {
     d.table.push_back(entry_of(f, ns));
     descs.push_back({slot_of(s.table[pg]), ns, f, dst * p->cfg.max_pages_per_seq + static_cast<int32_t>(pg)});
   }
-  p->seqs[dst] = d;
-  if (p->host_only) return ok();
-  CopyParams* prm = new CopyParams;
-  prm->fp8_slab = p->fp8_slab;
-  prm->tq3_slab = p->tq3_slab;
-  prm->tables = p->d_tables;
-  prm->fp8_slot_bytes = p->fp8_slot_bytes;
-  prm->tq3_slot_bytes = p->tq3_slot_bytes;
-  for (size_t b = 0; b < descs.size(); b += kCopyMaxDesc) {
-    const size_t m = std::min<size_t>(kCopyMaxDesc, descs.size() - b);
-    prm->n_desc = static_cast<int32_t>(m);
-    std::memcpy(prm->desc, descs.data() + b, m * sizeof(CopyDesc));
-    cudaError_t e = launch_copy(*prm, as_stream(stream));
-    ++p->launches;
-    if (e != cudaSuccess) {
-      delete prm;
-      return cuda_fail(e, "copy launch");
+  // ---- launch (the destination was empty: entries published before a failure are ignored)
+  int rc = MKV_OK;
+  if (!descs.empty()) {
+    CopyParams* prm = new CopyParams;
+    prm->fp8_slab = p->fp8_slab;
+    prm->tq3_slab = p->tq3_slab;
+    prm->tables = p->d_tables;
+    prm->fp8_slot_bytes = p->fp8_slot_bytes;
+    prm->tq3_slot_bytes = p->tq3_slot_bytes;
+    for (size_t b = 0; b < descs.size() && rc == MKV_OK; b += kCopyMaxDesc) {
+      const size_t m = std::min<size_t>(kCopyMaxDesc, descs.size() - b);
+      prm->n_desc = static_cast<int32_t>(m);
+      std::memcpy(prm->desc, descs.data() + b, m * sizeof(CopyDesc));
+      rc = device_op(p, "copy launch", [&] { return launch_copy(*prm, as_stream(stream)); });
     }
+    delete prm;
   }
-  delete prm;
+  if (rc != MKV_OK) {
+    for (auto it = descs.rbegin(); it != descs.rend(); ++it) p->alloc[it->fmt].give(it->dst_slot);
+    return rc;
+  }
+  p->seqs[dst] = std::move(d);
   return ok();
 }
 
@@ -1143,6 +1213,13 @@ int mkv_timing_read(mkv_pool_t p, double* ms_partial, double* ms_merge, int64_t*
   if (ms_partial) *ms_partial = a;
   if (ms_merge) *ms_merge = b;
   if (calls) *calls = n;
+  return ok();
+}
+
+int mkv_test_fail_launch(mkv_pool_t p, int32_t after) {
+  if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
+  if (after < -1) return fail(MKV_ERR_INVALID_ARG, "after must be >= -1");
+  p->fail_after = after;
   return ok();
 }
 
