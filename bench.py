@@ -34,14 +34,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "decode-attention µs/step and KV GB/s read (fraction of B200 HBM roofline)"
 FALLBACK_HBM_GBS = 6650.0
-# dram__bytes_read.sum + dram__bytes_write.sum per launch of the partial-attention kernel, from
-# the ncu capture summarised in profiles/, keyed by the hash of the kernel sources it measured.
-NCU_TRAFFIC = {
-    # profiles/decode_kernel_long_ctx128k_1layer.md: 494,519,552 B read + 4,348,928 B written
-    # (re-keyed: since that capture only the D 64/128 launch bound changed; the captured
-    # decode_kernel<256,1> is the same)
-    "53ddc387bee37f97": 498868480,
-}
+PROFILES = os.path.join(ROOT, "profiles")
 
 
 def kernel_hash() -> str:
@@ -50,6 +43,28 @@ def kernel_hash() -> str:
         with open(os.path.join(ROOT, "mixed_format_paged_mkv_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str):
+    """dram__bytes_read.sum + dram__bytes_write.sum per launch of `kernel` from the ncu summaries
+    under profiles/: a summary states it on a line
+    ``traffic_bytes_per_launch: <kernel> <bytes> sources <hash>``, where <hash> is kernel_hash() of
+    the sources that were captured.  None when no summary matches the current sources."""
+    want = kernel_hash()
+    try:
+        names = sorted(os.listdir(PROFILES))
+    except OSError:
+        return None
+    for n in names:
+        if not n.endswith((".md", ".txt")):
+            continue
+        with open(os.path.join(PROFILES, n)) as f:
+            for line in f:
+                parts = line.strip().strip("`").split()
+                if (len(parts) == 5 and parts[0] == "traffic_bytes_per_launch:" and
+                        parts[1] == kernel and parts[3] == "sources" and parts[4] == want):
+                    return int(parts[2])
+    return None
 
 
 def hbm_peak():
@@ -69,13 +84,14 @@ def decode_bytes(tables, ctxs, Hkv, D, Hq, q_len):
     ent = 0
     for t, L in zip(tables, ctxs):
         t = np.asarray(t, dtype=np.int64)
-        fmt = t >> 30
+        fmt = (t >> 30) & 3
         toks = np.full(t.size, 16, dtype=np.int64)
         toks[-1] = L - 16 * (t.size - 1)
         n8 = toks[fmt == 0].sum()
         p8 = int((fmt == 0).sum())
         n3 = toks[fmt == 1].sum()
-        kv += n8 * 2 * Hkv * D + p8 * 8 * Hkv + n3 * 0.875 * Hkv * D
+        n16 = toks[fmt == 2].sum()          # BF16 control pages
+        kv += n8 * 2 * Hkv * D + p8 * 8 * Hkv + n3 * 0.875 * Hkv * D + n16 * 4 * Hkv * D
         ent += t.size
     q = len(ctxs) * q_len * Hq * D * 2
     out = len(ctxs) * q_len * Hq * D * 4
@@ -101,27 +117,73 @@ def job_throughput(bytes_per_rank: float, world: int, elapsed_max_ms: float) -> 
 
 # ---------------------------------------------------------------------------- clocks
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons of one GPU, sampled every `period` seconds by a host
+    thread through NVML queries while the block runs (read only: no setting is changed).
+    Falls back to `nvidia-smi -lms` when NVML is not importable."""
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
+    def __init__(self, device_index: int, period: float = 0.005):
+        self.device_index = device_index
+        self.period = period
+        self.samples = []
+        self.max_mhz = None
+        self.source = None
+
+    def _handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.device_index).uuid)
+            return pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.device_index)
+
+    def _loop(self, h):
+        import pynvml
+        reason_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                r = reason_fn(h)
+                self.samples.append((sm, r))
+            except Exception:
+                pass
+            self._stop.wait(self.period)
 
     def __enter__(self):
+        import threading
+        self._stop = threading.Event()
+        self.thread = None
+        self.proc = None
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", str(self.index)],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            import pynvml
+            h = self._handle()
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.thread = threading.Thread(target=self._loop, args=(h,), daemon=True)
+            self.thread.start()
+            self.source = f"nvml every {self.period * 1000:.0f} ms"
         except Exception:
-            self.proc = None
-        time.sleep(0.3)
+            fields = ("clocks.sm,clocks.max.sm,clocks_event_reasons.sw_power_cap,"
+                      "clocks_event_reasons.hw_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                      "clocks_event_reasons.hw_thermal_slowdown")
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--query-gpu={fields}", "--format=csv,noheader,nounits",
+                     "-lms", "20", "-i", str(self.device_index)],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.source = "nvidia-smi every 20 ms"
+                time.sleep(0.3)
+            except Exception:
+                self.proc = None
         return self
 
     def __exit__(self, *a):
-        self.lines = []
+        if self.thread is not None:
+            self._stop.set()
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -129,41 +191,39 @@ class ClockSampler:
             except Exception:
                 self.proc.kill()
                 out = ""
-            self.lines = [l for l in out.splitlines() if l.strip()]
+            names = ["sw_power_cap", "hw_slowdown", "sw_thermal_slowdown", "hw_thermal_slowdown"]
+            for l in out.splitlines():
+                f = [x.strip() for x in l.split(",")]
+                try:
+                    mask = sum(self.REASONS[n] for n, v in zip(names, f[2:6]) if v.lower() == "active")
+                    self.samples.append((float(f[0]), mask))
+                    self.max_mhz = float(f[1])
+                except (ValueError, IndexError):
+                    continue
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in getattr(self, "lines", []):
-            f = [x.strip() for x in l.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "source": self.source}
+        reasons = sorted(n for n, bit in self.REASONS.items()
+                         if any(r & bit for _, r in self.samples))
+        return {"sm_mhz": statistics.median(sm for sm, _ in self.samples),
+                "sm_min_mhz": min(sm for sm, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples), "source": self.source}
 
 
 # ---------------------------------------------------------------------------- oracle (CPU)
-def oracle_sample(w, seq=0, head=0, target_s=10.0, max_runs=None, warmup=0):
+def oracle_sample(w, seq=0, head=0, target_s=10.0, max_runs=None, warmup=0, threads=None):
     """Time the CPU oracle's decode (dequantise the pages + float64 attention) of one sequence's
-    one KV-head group over its full context.  Returns (GB/s, seconds per run, runs, cores, desc)."""
+    one KV-head group over its full context, with its BLAS limited to `threads` (None: all the
+    host's cores).  Returns (GB/s, seconds per run, runs, threads used, desc)."""
+    from threadpoolctl import threadpool_info, threadpool_limits
+
     from oracle import attention as A
     from oracle import formats as F
     from oracle import pool as P
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        cores = 1
+    limiter = threadpool_limits(limits=threads)
+    cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     L = w.lengths()[seq]
     k, v = w.kv(seq, 0)
     k, v = k[:, [head]], v[:, [head]]
@@ -192,6 +252,7 @@ def oracle_sample(w, seq=0, head=0, target_s=10.0, max_runs=None, warmup=0):
             break
         if max_runs is None and time.perf_counter() - t_start >= target_s:
             break
+    limiter.restore_original_limits()
     per = sum(times) / len(times)
     desc = (f"decode of sequence {seq}, KV head {head} ({w.g} query heads) over {L} tokens "
             f"of layer 0: dequantise {len(table)} pages + float64 attention, {len(times)} runs")
@@ -199,7 +260,7 @@ def oracle_sample(w, seq=0, head=0, target_s=10.0, max_runs=None, warmup=0):
 
 
 # ---------------------------------------------------------------------------- GPU arm
-def build_pool(w, layers, extra_pages, device):
+def build_pool(w, layers, extra_pages, device, bf16_control=False):
     import torch
     from mixed_format_paged_mkv_b200 import Pool
     pages = w.pages()
@@ -207,7 +268,10 @@ def build_pool(w, layers, extra_pages, device):
     anchors = [1 + w.window // 16 + 1 + n for n in n_prot]
     fp8 = max(max(pages) + sum(anchors), layers * sum(a + extra_pages for a in anchors)) + 64
     tq3 = layers * (sum(pages) + w.B * extra_pages) + 64
-    pool = Pool(w.Hkv, w.D, w.B * layers, max(pages) + extra_pages, fp8, tq3, device=device)
+    if bf16_control:      # every page stays in the first slab as BF16
+        fp8, tq3 = layers * (sum(pages) + w.B * extra_pages) + 64, 0
+    pool = Pool(w.Hkv, w.D, w.B * layers, max(pages) + extra_pages, fp8, tq3, device=device,
+                bf16_control=bf16_control)
     for fmt, n in ((0, fp8), (1, tq3)):
         order = w.slot_permutation(fmt, n)
         if order is not None:
@@ -262,7 +326,9 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.set_device(device)
     w = WORKLOADS[4]
     layers = args.layers
-    total_steps = args.warmup + args.steps + (args.warmup + args.steps if not args.no_e2e else 0)
+    # three timed passes (value, kernel share, end to end) after their warm-ups append tokens
+    n_dev = args.warmup + 2 * args.steps
+    total_steps = n_dev + (args.warmup + args.steps if not args.no_e2e else 0)
     extra = total_steps // 16 + 3
     t_build = time.time()
     pool = build_pool(w, layers, extra, device)
@@ -273,7 +339,6 @@ def run_gpu(args, rank, world, local_rank):
 
     seq_ids = [np.arange(l * w.B, (l + 1) * w.B, dtype=np.int32) for l in range(layers)]
     ones = np.ones(w.B, dtype=np.int32)
-    n_dev = args.warmup + args.steps
     Kh, Vh, Qh = step_inputs_host(w, layers, n_dev, 0)
     Kd, Vd, Qd = as_bf16(Kh).to(device), as_bf16(Vh).to(device), as_bf16(Qh).to(device)
     outs = torch.empty((layers, w.B, w.q_len, w.Hq, w.D), dtype=torch.float32, device=device)
@@ -304,41 +369,49 @@ def run_gpu(args, rank, world, local_rank):
     def max_over_ranks(x):
         return rank_max(x, world, device)
 
-    # ---------------- device-resident run (value)
+    def timed(first):
+        """Steps [first, first + steps) between two events on the stream; returns ms."""
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        e0.record(stream)
+        for s in range(first, first + args.steps):
+            one_step(Kd[s], Vd[s], Qd[s])
+        e1.record(stream)
+        barrier()
+        return max_over_ranks(e0.elapsed_time(e1))
+
+    # ---------------- pass 1: the headline, no per-call instrumentation
     for s in range(args.warmup):
         one_step(Kd[s], Vd[s], Qd[s])
     barrier()
     b0 = tables_now()
     launches0 = pool.launch_count()
-    pool.timing(True)
-    pool.timing_read()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[local_rank]) \
-        if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit() else local_rank
-    with ClockSampler(gpu_index) as clk:
-        barrier()
-        ev0.record(stream)
-        for s in range(args.warmup, args.warmup + args.steps):
-            one_step(Kd[s], Vd[s], Qd[s])
-        ev1.record(stream)
-        barrier()
-    elapsed_ms = max_over_ranks(ev0.elapsed_time(ev1))
-    tm = pool.timing_read()
-    pool.timing(False)
+    with ClockSampler(local_rank) as clk:
+        elapsed_ms = timed(args.warmup)
     launches = pool.launch_count() - launches0
     b1 = tables_now()
     pool.device_status()
     per_call_total = 0.5 * (b0[0] + b1[0])
-    per_call_partial = 0.5 * (b0[1] + b1[1])
     value_gbs = job_throughput(per_call_total * layers * args.steps, world, elapsed_ms)
+
+    # ---------------- pass 2: the same steps with the library's per-call kernel events (three
+    # per decode call, on the stream the kernels run on) for the partial-attention kernel's time
+    pool.timing(True)
+    pool.timing_read()
+    instrumented_ms = timed(args.warmup + args.steps)
+    tm = pool.timing_read()
+    pool.timing(False)
+    b2 = tables_now()
+    pool.device_status()
+    per_call_partial = 0.5 * (b1[1] + b2[1])
     partial_ms = tm["partial_ms"] / max(tm["calls"], 1)
     achieved = per_call_partial / (partial_ms * 1e-3) / 1e9
     peak, peak_src = hbm_peak()
 
-    # ---------------- end to end through the public API with host buffers
+    # ---------------- pass 3: end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        first = args.warmup + args.steps
+        first = n_dev
         Kh2, Vh2, Qh2 = step_inputs_host(w, layers, args.warmup + args.steps, first)
         Kp = as_bf16(Kh2).pin_memory()
         Vp = as_bf16(Vh2).pin_memory()
@@ -367,8 +440,8 @@ def run_gpu(args, rank, world, local_rank):
         e1.record(stream)
         barrier()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-        b2 = tables_now()
-        e2e_gbs = job_throughput(0.5 * (b1[0] + b2[0]) * layers * args.steps, world, e2e_ms)
+        b3 = tables_now()
+        e2e_gbs = job_throughput(0.5 * (b2[0] + b3[0]) * layers * args.steps, world, e2e_ms)
         e2e = {"value": round(e2e_gbs, 2), "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": round(e2e_ms / args.steps, 4)}
@@ -386,7 +459,7 @@ def run_gpu(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f16xf16->f32 (e4m3 and 3-bit codes, exact f16 images)",
+        "dtype": "f16 MMA, f32 accumulate (e4m3 and 3-bit codes, exact f16 images)",
         "data": "synthetic (seeded bf16 N(0,1), 4 outlier K channels x8 per head)",
         "config": {"workload": w.name, "batch": w.B, "context": w.lengths()[0],
                    "layers": layers, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.D,
@@ -397,10 +470,12 @@ def run_gpu(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "kernel": "decode_kernel (FP8 + TQ3 partial attention)",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_source": peak_src,
-                     "traffic": NCU_TRAFFIC.get(kernel_hash()),
+                     "traffic": ncu_traffic("decode_kernel"),
                      "bytes_per_launch": int(per_call_partial),
                      "launch_ms": round(partial_ms, 5),
-                     "merge_ms": round(tm["merge_ms"] / max(tm["calls"], 1), 5)},
+                     "merge_ms": round(tm["merge_ms"] / max(tm["calls"], 1), 5),
+                     "timed": "second pass of the same steps with per-call events on the stream",
+                     "instrumented_ms_per_step": round(instrumented_ms / args.steps, 4)},
         "e2e": e2e,
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
@@ -409,9 +484,12 @@ def run_gpu(args, rank, world, local_rank):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         gbs, per, runs, cores, desc = oracle_sample(w, target_s=args.cpu_seconds)
+        gbs1, per1, _, _, _ = oracle_sample(w, target_s=args.cpu_seconds / 2, threads=1)
         res["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores,
                                "kind": "oracle", "sample": desc,
-                               "seconds_per_run": round(per, 3)}
+                               "seconds_per_run": round(per, 3),
+                               "single_thread": {"value": round(gbs1, 4), "unit": "GB/s",
+                                                 "cores": 1, "seconds_per_run": round(per1, 3)}}
     return res
 
 
@@ -461,9 +539,22 @@ def _bf16_tensor(bits, device):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
 
 
+_FLUSH = None
+
+
+def _flush_l2(device):
+    """Write a buffer twice the size of the 126 MB L2, so the next call reads its pages from HBM."""
+    global _FLUSH
+    import torch
+    if _FLUSH is None:
+        _FLUSH = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    _FLUSH.zero_()
+
+
 def _time_decode(pool, w, device, reps=20, warm=3):
     """Partial and merge time (µs) and algorithmic bytes of one decode call over all sequences
-    of one layer, averaged over `reps` calls after `warm` untimed ones."""
+    of one layer, averaged over `reps` calls after `warm` untimed ones; L2 is flushed before
+    every call (the library's per-call events exclude the flush)."""
     import torch
     seqs = list(range(w.B))
     q = _bf16_tensor(np.stack([w.q(s) for s in seqs]), device)
@@ -476,13 +567,14 @@ def _time_decode(pool, w, device, reps=20, warm=3):
     pool.timing(True)
     pool.timing_read()
     for _ in range(reps):
+        _flush_l2(device)
         pool.decode(seqs, q, out=out, workspace=ws)
     tm = pool.timing_read()
     pool.timing(False)
     pool.device_status()
     tabs, ctxs = zip(*(pool.block_table(s) for s in seqs))
     total, partial = decode_bytes(tabs, ctxs, w.Hkv, w.D, w.Hq, w.q_len)
-    n8 = sum(1 for t in tabs for e in t if (e >> 30) == 0)
+    n8 = sum(1 for t in tabs for e in t if ((e >> 30) & 3) != 1)
     return dict(partial_us=1000 * tm["partial_ms"] / tm["calls"],
                 merge_us=1000 * tm["merge_ms"] / tm["calls"], bytes=partial,
                 fp8_page_share=n8 / sum(len(t) for t in tabs), out=out)
@@ -509,26 +601,71 @@ def run_extra(args):
                               kv_bytes_per_token=round(pool.stats()[3], 1)))
             del pool
             torch.cuda.empty_cache()
-    elif args.mode == "canary":
-        res = {}
-        for name, frac in (("mixed", 0.0), ("fp8_control", 1.0)):
-            w = WORKLOADS[4].scaled(B=2, ctx=(59008, 59008), fp8_page_frac=frac, layers=1)
+    elif args.mode == "ablation":
+        # one grid per page format (default) against one fused grid, on the long-context layer
+        # and on the FP8-share sweep points
+        for frac in (0.0, 0.04, 0.25, 1.0):
+            w = WORKLOADS[4].scaled(fp8_page_frac=frac, layers=1)
             pool = build_pool(w, 1, 3, device)
+            for fused in (False, True):
+                pool.set_decode_kernels(fused)
+                r = _time_decode(pool, w, device)
+                gbs = r["bytes"] / (r["partial_us"] * 1e-6) / 1e9
+                lines.append(dict(mode="ablation", kernels="fused" if fused else "split",
+                                  workload=w.name, fp8_page_share=round(r["fp8_page_share"], 4),
+                                  partial_us=round(r["partial_us"], 2),
+                                  merge_us=round(r["merge_us"], 2),
+                                  bytes_per_call=int(r["bytes"]), gbs=round(gbs, 1),
+                                  frac=round(gbs / peak, 4), peak_source=peak_src))
+            del pool
+            torch.cuda.empty_cache()
+    elif args.mode == "profile":
+        # a small target for ncu: one layer of the long-context workload, a few decode calls
+        w = WORKLOADS[4].scaled(layers=1)
+        pool = build_pool(w, 1, 3, device)
+        pool.set_decode_kernels(args.fused)
+        seqs = list(range(w.B))
+        q = _bf16_tensor(np.stack([w.q(s) for s in seqs]), device)
+        out = torch.empty((w.B, w.q_len, w.Hq, w.D), dtype=torch.float32, device=device)
+        ws = torch.empty(pool.workspace_bytes(seqs, w.q_len, w.Hq) + (1 << 20), dtype=torch.uint8,
+                         device=device)
+        for _ in range(args.steps):
+            pool.decode(seqs, q, out=out, workspace=ws)
+        torch.cuda.synchronize()
+        pool.device_status()
+        tabs, ctxs = zip(*(pool.block_table(s) for s in seqs))
+        total, partial = decode_bytes(tabs, ctxs, w.Hkv, w.D, w.Hq, w.q_len)
+        lines.append(dict(mode="profile", workload=w.name, calls=args.steps,
+                          partial_bytes_per_call=int(partial), kernel_sources=kernel_hash()))
+    elif args.mode == "canary":
+        # two 59,008-token decodes at the long workload's head shape: the mixed cache against
+        # an all-FP8 control and a BF16 control (pages stored as bf16), L2 flushed before every
+        # timed call of every arm
+        res = {}
+        for name, frac, ctl in (("mixed", 0.0, False), ("fp8_control", 1.0, False),
+                                ("bf16_control", 0.0, True)):
+            w = WORKLOADS[4].scaled(B=2, ctx=(59008, 59008), fp8_page_frac=frac, layers=1)
+            pool = build_pool(w, 1, 3, device, bf16_control=ctl)
             r = _time_decode(pool, w, device)
             res[name] = dict(r, bpt=pool.stats()[3])
             del pool
             torch.cuda.empty_cache()
-        m, c = res["mixed"], res["fp8_control"]
-        diff = (m["out"] - c["out"]).abs().max().item()
-        tm, tc = m["partial_us"] + m["merge_us"], c["partial_us"] + c["merge_us"]
-        lines.append(dict(mode="canary", sequences=2, context=59008, q_heads=24, kv_heads=4, head_dim=256,
-                          mixed_us=round(tm, 2), control_us=round(tc, 2),
-                          throughput_vs_control=round(tc / tm, 4),
-                          kv_bytes_per_token_mixed=round(m["bpt"], 1),
-                          kv_bytes_per_token_control=round(c["bpt"], 1),
-                          active_kv_ratio=round(c["bpt"] / m["bpt"], 4),
-                          fp8_page_share_mixed=round(m["fp8_page_share"], 4),
-                          max_abs_output_difference=diff))
+        m = res["mixed"]
+        tm = m["partial_us"] + m["merge_us"]
+        line = dict(mode="canary", sequences=2, context=59008, q_heads=24, kv_heads=4, head_dim=256,
+                    mixed_us=round(tm, 2), kv_bytes_per_token_mixed=round(m["bpt"], 1),
+                    fp8_page_share_mixed=round(m["fp8_page_share"], 4),
+                    l2="flushed (256 MB write) before every timed call of every arm")
+        for name in ("fp8_control", "bf16_control"):
+            c = res[name]
+            tc = c["partial_us"] + c["merge_us"]
+            line.update({f"{name}_us": round(tc, 2),
+                         f"throughput_vs_{name}": round(tc / tm, 4),
+                         f"kv_bytes_per_token_{name}": round(c["bpt"], 1),
+                         f"active_kv_ratio_vs_{name}": round(c["bpt"] / m["bpt"], 4),
+                         f"max_abs_output_difference_vs_{name}":
+                             (m["out"] - c["out"]).abs().max().item()})
+        lines.append(line)
     elif args.mode == "pack":
         w = WORKLOADS[2]
         pages = w.pages()
@@ -541,10 +678,12 @@ def run_extra(args):
         work = list(range(w.B, 2 * w.B))
         stream = torch.cuda.current_stream()
         times, demoted = [], 0
+        times, dev_times = [], []
         for rep in range(8):
             for s in range(w.B):
                 pool.copy(s, w.B + s)
             torch.cuda.synchronize()
+            # call span: host planning and launches included
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             demoted = pool.demote(work, w.window)
@@ -554,14 +693,29 @@ def run_extra(args):
                 times.append(e0.elapsed_time(e1))
             for s in work:
                 pool.reset(s)
+            for s in range(w.B):
+                pool.copy(s, w.B + s)
+            torch.cuda.synchronize()
+            # device time only: a spin kernel keeps the GPU busy while the host plans
+            torch.cuda._sleep(20_000_000)
+            e0.record(stream)
+            pool.demote(work, w.window)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if rep >= 2:
+                dev_times.append(e0.elapsed_time(e1))
+            for s in work:
+                pool.reset(s)
         pool.device_status()
         per_page = w.Hkv * ((32 * w.D + 8) + 14 * w.D)
-        ms = statistics.median(times)
-        gbs = demoted * per_page / (ms * 1e-3) / 1e9
+        ms, dms = statistics.median(times), statistics.median(dev_times)
+        gbs, dgbs = demoted * per_page / (ms * 1e-3) / 1e9, demoted * per_page / (dms * 1e-3) / 1e9
         lines.append(dict(mode="pack", workload=w.name, pages_demoted=demoted, bytes=demoted * per_page,
                           ms=round(ms, 4), gbs=round(gbs, 1), frac=round(gbs / peak, 4),
-                          peak_source=peak_src,
-                          note="one mkv_demote_pages call, host planning included in the span"))
+                          device_ms=round(dms, 4), device_gbs=round(dgbs, 1),
+                          device_frac=round(dgbs / peak, 4), peak_source=peak_src,
+                          note="one mkv_demote_pages call: ms is the call span with host "
+                               "planning, device_ms the device work alone"))
     elif args.mode == "prefill":
         # direct bf16 -> TQ3 packing of the batch-8 workload's prompts (256-token window FP8)
         w = WORKLOADS[2]
@@ -572,7 +726,7 @@ def run_extra(args):
         kd, vd = _bf16_tensor(np.concatenate(ks), device), _bf16_tensor(np.concatenate(vs), device)
         seqs, lens = list(range(w.B)), w.lengths()
         stream = torch.cuda.current_stream()
-        times = []
+        times, dev_times = [], []
         for rep in range(8):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
@@ -581,6 +735,15 @@ def run_extra(args):
             torch.cuda.synchronize()
             if rep >= 2:
                 times.append(e0.elapsed_time(e1))
+            for s in seqs:
+                pool.reset(s)
+            torch.cuda._sleep(20_000_000)
+            e0.record(stream)
+            pool.prefill(seqs, lens, kd, vd, window=w.window)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if rep >= 2:
+                dev_times.append(e0.elapsed_time(e1))
             if rep < 7:
                 for s in seqs:
                     pool.reset(s)
@@ -590,12 +753,14 @@ def run_extra(args):
         n8 = sum(len(t) for t in tabs) - n3
         rd = sum(lens) * w.Hkv * w.D * 2 * 2
         wr = n3 * w.Hkv * 14 * w.D + n8 * w.Hkv * (32 * w.D + 16)
-        ms = statistics.median(times)
-        gbs = (rd + wr) / (ms * 1e-3) / 1e9
+        ms, dms = statistics.median(times), statistics.median(dev_times)
+        gbs, dgbs = (rd + wr) / (ms * 1e-3) / 1e9, (rd + wr) / (dms * 1e-3) / 1e9
         lines.append(dict(mode="prefill", workload=w.name, tokens=sum(lens), tq3_pages=n3, fp8_pages=n8,
                           bytes=rd + wr, ms=round(ms, 4), gbs=round(gbs, 1), frac=round(gbs / peak, 4),
-                          peak_source=peak_src,
-                          note="one mkv_prefill_kv call (bf16 read, TQ3/FP8 pages written), host planning included"))
+                          device_ms=round(dms, 4), device_gbs=round(dgbs, 1),
+                          device_frac=round(dgbs / peak, 4), peak_source=peak_src,
+                          note="one mkv_prefill_kv call (bf16 read, TQ3/FP8 pages written): ms is "
+                               "the call span with host planning, device_ms the device work alone"))
     elif args.mode == "materialise":
         w = WORKLOADS[2]
         pool = build_pool(w, 1, 3, device)
@@ -713,8 +878,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--fused", action="store_true", help="--mode profile: the fused kernel")
     ap.add_argument("--mode", choices=["bench", "sweep", "canary", "pack", "prefill", "materialise",
-                                       "configs"],
+                                       "configs", "ablation", "profile"],
                     default="bench",
                     help="extra studies on one GPU (one JSON line per point); default: the bench")
     args = ap.parse_args()

@@ -33,8 +33,9 @@
  *       K records [G][16 tokens][12 B] | K scales [G][16] f16 | V records [G][16][12 B] | V scales [G][16] f16
  *
  * Block-table entry (int32): -1 = unmapped, else (format << 30) | slot, format 0 = FP8,
- * 1 = TQ3.  Sequence ids are rows of the table; a multi-layer cache uses one row per
- * (layer, sequence).
+ * 1 = TQ3, 2 = BF16 (control pools only; such an entry is negative as an int32, so test for
+ * -1, not for the sign).  Sequence ids are rows of the table; a multi-layer cache uses one row
+ * per (layer, sequence).
  *
  * Ownership: every device buffer is allocated and owned by the caller (e.g. by PyTorch) and
  * must outlive the pool; the pool owns only host state (allocators, the host copy of the
@@ -87,11 +88,18 @@ enum {
 
 #define MKV_FMT_FP8 0
 #define MKV_FMT_TQ3 1
+#define MKV_FMT_BF16 2 /* pages of a BF16 control pool */
 #define MKV_PAGE_TOKENS 16
 #define MKV_ENTRY_UNMAPPED (-1)
 
 /* Pool flags. */
 #define MKV_POOL_HOST_ONLY 1 /* track tables on the host only: no device buffers, no launches */
+/* A control pool, the comparator the pages measure the method against (sections "Memória e
+ * compressão" and "Verificação canário"): every page holds its bf16 values as they are (format
+ * MKV_FMT_BF16, in the first slab: per KV head K rows [16][D] then V rows [16][D], bf16, rows
+ * not yet written zero; 64*D bytes per head), no page is ever demoted, and decode runs a BF16
+ * partial kernel over them.  The TQ3 slab is unused (tq3_slots may be 0). */
+#define MKV_POOL_BF16_CONTROL 2
 
 typedef struct mkv_pool* mkv_pool_t;
 
@@ -207,7 +215,11 @@ MKV_API int mkv_decode_attention(mkv_pool_t pool, const int32_t* seq_ids, int32_
  *   - The array is allocated when the library's device code is loaded and is held by every
  *     GPU that loads it until the process exits.
  *   - The first call on a device resolves the array's device address (cudaGetSymbolAddress
- *     with that device current); make that first call before any stream capture.
+ *     with that device current) and keeps it for the life of the process; make that first call
+ *     before any stream capture.  After cudaDeviceReset on that device the kept address is
+ *     stale: do not call this entry point on that device again in the same process.
+ *   - The call plans its launch in a block of about 75 KB on the calling thread's stack: call
+ *     it from threads with at least 128 KB of stack to spare.
  *   - All calls share the array and it keeps the last call's contents; nothing in it needs to
  *     start at zero.  Calls that overlap on the GPU (other streams, other pools on the same
  *     device) race on it: order them.
@@ -216,6 +228,17 @@ MKV_API int mkv_decode_attention(mkv_pool_t pool, const int32_t* seq_ids, int32_
 MKV_API int mkv_decode_attention_noalloc(mkv_pool_t pool, const int32_t* seq_ids, int32_t n_seqs,
                                          int32_t q_len, const void* q_bf16, int32_t num_q_heads,
                                          float sm_scale, float* out, void* stream);
+
+/* Which partial-attention kernels decode uses (both compute the same partial states, so the
+ * results are identical; this exists to compare the two designs):
+ *   MKV_DECODE_SPLIT (default) -- a separate kernel per page format, as the pages describe
+ *     (section "Como os resultados parciais são combinados"): the TQ3 grid, then the FP8 grid
+ *     launched as its programmatic dependent so that FP8 CTAs take SM room as TQ3 CTAs retire;
+ *   MKV_DECODE_FUSED -- one grid whose CTAs branch on their unit's format.
+ * Host only; applies to later decode calls on this pool.  Errors: INVALID_ARG. */
+#define MKV_DECODE_SPLIT 0
+#define MKV_DECODE_FUSED 1
+MKV_API int mkv_set_decode_kernels(mkv_pool_t pool, int32_t mode);
 
 /* Free every page of a sequence and clear its table row and flags. */
 MKV_API int mkv_seq_reset(mkv_pool_t pool, int32_t seq, void* stream);

@@ -15,8 +15,8 @@ import numpy as np
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libmkv.so")
 
-FMT_FP8, FMT_TQ3 = 0, 1
-POOL_HOST_ONLY = 1
+FMT_FP8, FMT_TQ3, FMT_BF16 = 0, 1, 2
+POOL_HOST_ONLY, POOL_BF16_CONTROL = 1, 2
 ERRORS = {0: "OK", -1: "INVALID_ARG", -2: "BAD_SEQ", -3: "OUT_OF_PAGES", -4: "EMPTY_CONTEXT",
           -5: "PAGE_NOT_FULL", -6: "WORKSPACE_TOO_SMALL", -7: "CUDA", -8: "DEVICE_CHECK",
           -9: "DEVICE_TIMEOUT", -10: "UNSUPPORTED"}
@@ -69,6 +69,7 @@ SIGNATURES = {
                                        ctypes.POINTER(ctypes.c_int64)]),
     "mkv_launch_count": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int64)]),
     "mkv_test_fail_launch": (ctypes.c_int, [_P, _I32]),
+    "mkv_set_decode_kernels": (ctypes.c_int, [_P, _I32]),
     "mkv_last_error": (ctypes.c_char_p, []),
 }
 
@@ -129,9 +130,11 @@ class Pool:
     """A mixed-format paged KV cache over device buffers owned by this object (torch)."""
 
     def __init__(self, num_kv_heads, head_dim, max_seqs, max_pages_per_seq, fp8_slots,
-                 tq3_slots, sink_pages=1, device=None, host_only=False):
+                 tq3_slots, sink_pages=1, device=None, host_only=False, bf16_control=False):
+        flags = (POOL_HOST_ONLY if host_only else 0) | (POOL_BF16_CONTROL if bf16_control else 0)
         self.cfg = PoolConfig(num_kv_heads, head_dim, 16, max_seqs, max_pages_per_seq,
-                              fp8_slots, tq3_slots, sink_pages, POOL_HOST_ONLY if host_only else 0)
+                              fp8_slots, tq3_slots, sink_pages, flags)
+        self.bf16_control = bf16_control
         self.Hkv, self.D = num_kv_heads, head_dim
         self.host_only = host_only
         L = lib()
@@ -319,7 +322,7 @@ class Pool:
         return b.value
 
     def read_slot(self, entry, stream=None):
-        nb = self.slot_bytes(entry >> 30)
+        nb = self.slot_bytes((entry >> 30) & 3)  # format tag (a BF16 entry is negative)
         buf = np.zeros(nb, dtype=np.uint8)
         _check(lib().mkv_read_slot(self.handle, entry, buf.ctypes.data_as(_P), nb,
                                    _stream_ptr(stream)), "mkv_read_slot")
@@ -348,6 +351,11 @@ class Pool:
         _check(lib().mkv_timing_read(self.handle, ctypes.byref(v[0]), ctypes.byref(v[1]),
                                      ctypes.byref(n)), "mkv_timing_read")
         return dict(partial_ms=v[0].value, merge_ms=v[1].value, calls=n.value)
+
+    def set_decode_kernels(self, fused):
+        """Decode with one fused partial grid (True) or a grid per page format (False)."""
+        _check(lib().mkv_set_decode_kernels(self.handle, 1 if fused else 0),
+               "mkv_set_decode_kernels")
 
     def test_fail_launch(self, after):
         """Make the device operation after the next ``after`` ones fail (test hook; -1: off)."""

@@ -6,17 +6,24 @@
 // normalisation combines them -- no page is converted to a common format first and no dense
 // copy of the cache is made (section "... sem a chamada sombra densa").
 //
-// Two launches per call.  The host cuts every sequence into work units -- (format, logical page
-// range) -- and orders them largest first.  A CTA takes one (unit, KV head):
-//   1. its producer warp scans the block-table entries of the range and keeps the pages of the
-//      unit's format (FP8 units run fp8_page, TQ3 units tq3_page: separate per-format code and
-//      separate partial states);
-//   2. the producer streams those pages through a shared-memory ring with bulk async copies
-//      completing on mbarriers;
-//   3. consumer warps (pages round-robin) compute per page the logits, the online softmax
-//      (running max m and denominator l per query column) and P.V;
+// The host cuts every sequence into work units -- (format, logical page range) -- and orders
+// them largest first.  Three launches per call (per launch group): the TQ3 partial kernel over
+// the TQ3 units, the FP8 partial kernel over the FP8 units and the merge kernel.  The FP8 and
+// merge kernels are programmatic dependents of the kernel before them: the FP8 CTAs take SM
+// room as soon as TQ3 CTAs retire (one wave of both formats), the merge CTAs are resident
+// before the partial kernels end and wait for their results with griddepcontrol.wait.  (A fused
+// variant runs both formats in one grid, branching per CTA; it is kept for the comparison.)
+//
+// A partial CTA takes one (unit, KV head):
+//   1. one warp scans the block-table entries of the range, keeps the pages of the unit's format
+//      and starts the first bulk async copies of those pages into a shared-memory ring;
+//   2. the warps take pages round-robin; each ring stage always belongs to the same warp(s),
+//      which refill it with the page one ring-length ahead as soon as they are done with it (no
+//      producer warp: the stage's copy completes on its mbarrier);
+//   3. per page the logits, the online softmax (running max m and denominator l per query
+//      column) and P.V;
 //   4. the CTA combines its warps and writes its partial state (m, l, acc) per query column.
-// A second kernel merges, per (sequence, KV head, query column), all partial states of both
+// The merge kernel combines, per (sequence, KV head, query column), all partial states of both
 // formats: M = max m, L = sum l 2^(m-M), O = sum acc 2^(m-M) / L.
 //
 // Tensor-core use: per page the logits are a 16-token x 8-column tile (tokens are the MMA M
@@ -26,7 +33,9 @@
 //   TQ3 K: codes -> exact f16 images (base + c); each group's MMA starts from the correction
 //          -(base + 3.5) * (sum of the matching query values), so it yields sum q (c - 3.5);
 //          the per-(token, group) scale multiplies the group's result (summed in fp32).
-//   TQ3 V: codes -> (c - 3.5) exactly; the per-(token, group) scale multiplies P in f16.
+//   TQ3 V: codes -> (c - 3.5) exactly; the per-(token, group) scale multiplies P in f16, with a
+//          per-group power of two taken out first on pages whose scales would leave the f16
+//          range.
 //   FP8:   e4m3x2 -> f16x2 conversions; the per-page scales multiply logits / the page's P.V.
 // Softmax runs in log2 units with a lazily raised reference maximum (raised only when a
 // logit exceeds it by more than 8), so probabilities fed to the MMA are < 2^8.
@@ -41,60 +50,74 @@ namespace {
 
 constexpr float kLazyRescale = 8.f;  // log2 units
 
-template <int D, int NT>
+// Partial-kernel kinds: one format per grid, both mixed formats (branching per CTA), or the
+// BF16 control pages.
+enum Kind { kKindFp8 = 0, kKindTq3 = 1, kKindFused = 2, kKindBf16 = 3 };
+// Page formats (block-table tags).
+enum Fmt { kFp8 = 0, kTq3 = 1, kBf16 = 2 };
+
+template <int D, int NT, int K>
 struct Cfg {
-  static constexpr int PW = NT == 1 ? 4 : (NT == 2 ? 2 : 1);  // page-parallel warps
-  static constexpr int NWC = NT * PW;                          // consumer warps
-  static constexpr int THREADS = 32 * (NWC + 1);               // + 1 producer warp
-  static constexpr int PRODUCER = NWC;
+  static constexpr int PW = NT == 1 ? 4 : (NT == 2 ? 2 : 1);  // page-parallel warp groups
+  static constexpr int WARPS = NT * PW;                        // warp nt of group pw: nt + NT*pw
+  static constexpr int THREADS = 32 * WARPS;
   static constexpr int FP8_STAGE = 32 * D + 16;
   static constexpr int TQ3_STAGE = 14 * D;
-  // Every stage must always be consumed by the same warp(s): a warp waits on a stage's fill f
-  // with parity f & 1, which is only unambiguous if fill f-1 of that stage was its own (and so
-  // already completed).  Hence ring depths are multiples of PW.
+  // BF16 control page: its 32 rows (16 K, 16 V) copied one by one into rows padded by 16
+  // bytes, so the 8 rows an ldmatrix reads fall on distinct banks
+  static constexpr int BF16_ROW = 2 * D + 16;
+  static constexpr int BF16_STAGE = 32 * BF16_ROW;
+  // Stage s only ever holds pages i with i % NST == s, and they belong to warp group i % PW:
+  // with NST a multiple of PW each stage has a fixed owner, which refills it when done.
   static constexpr int FP8_NST = 8;
-  static constexpr int TQ3_NST = 16;
-  static_assert(FP8_NST % PW == 0 && TQ3_NST % PW == 0, "stage ownership");
-  static constexpr int RING_FP8 = FP8_NST * FP8_STAGE;
-  static constexpr int RING_TQ3 = TQ3_NST * TQ3_STAGE;
-  // end-of-unit combine: (m, l) and acc of every consumer warp
+  static constexpr int TQ3_NST = 8;
+  static constexpr int BF16_NST = 8;
+  static_assert(FP8_NST % PW == 0 && TQ3_NST % PW == 0 && BF16_NST % PW == 0, "stage ownership");
+  static constexpr int RING_FP8 = (K == kKindFp8 || K == kKindFused) ? FP8_NST * FP8_STAGE : 0;
+  static constexpr int RING_TQ3 = (K == kKindTq3 || K == kKindFused) ? TQ3_NST * TQ3_STAGE
+                                  : (K == kKindBf16 ? BF16_NST * BF16_STAGE : 0);
+  // end-of-unit combine: (m, l) and acc of every warp
   static constexpr int COMBINE = PW * NT * 8 * (D + 2) * 4;
   static constexpr int RING = RING_FP8 > RING_TQ3 ? (RING_FP8 > COMBINE ? RING_FP8 : COMBINE)
                                                   : (RING_TQ3 > COMBINE ? RING_TQ3 : COMBINE);
-  // header: full[16] | empty[16] mbarriers | stage tags | misc | page list | Q fragments |
-  //         TQ3 K corrections | ring
-  static constexpr int OFF_TAG = 256;
-  static constexpr int OFF_MISC = OFF_TAG + 64;
+  // header: full[16] mbarriers | release counters | fills issued | misc | page list |
+  //         Q fragments | TQ3 K corrections | ring
+  static constexpr int OFF_CNT = 128;
+  static constexpr int OFF_FILLS = OFF_CNT + 64;
+  static constexpr int OFF_MISC = OFF_FILLS + 64;
   static constexpr int OFF_LIST = OFF_MISC + 64;
   static constexpr int OFF_QF = (OFF_LIST + kMaxPagesPerUnit * 8 + 127) / 128 * 128;
   static constexpr int QF = NT * D * 16;
   static constexpr int OFF_CORR = OFF_QF + QF;
-  static constexpr int OFF_RING = (OFF_CORR + NT * (D / 32) * 64 + 127) / 128 * 128;
+  static constexpr int OFF_RING = (OFF_CORR + NT * (D / 32) * 32 + 127) / 128 * 128;
   static constexpr int SMEM = OFF_RING + RING;
+  // CTAs per SM the launch bounds aim at (registers: 65536 / (THREADS * that))
+  // (an FP8 CTA fits beside three TQ3 CTAs: both kernels at 4 for D 256)
+  static constexpr int MINB = K == kKindBf16 ? 1 : D == 256 ? (K == kKindFused ? 3 : 4) : (D == 128 ? 5 : 6);
 };
 
 struct Smem {
-  uint64_t* full;   // [stage]: page landed (producer arrive + bulk-copy bytes)
-  uint64_t* empty;  // [stage]: the page's consumer warps are done with it
-  int32_t* tag;     // logical page of each stage
+  uint64_t* full;   // [stage]: the stage's page landed (arrive + bulk-copy bytes)
+  int32_t* cnt;     // [stage]: warps done with the stage's page (several n-tiles per page)
+  int32_t* fills;   // [stage]: copies issued into the stage
   int32_t* misc;    // [0] page count, [1] abort flag, [4..7] logit scales per n-tile
   int2* list;       // {slot, logical page} of the unit's pages
   uint4* qf;        // Q fragments [NT][D/32][32 lanes]
-  float4* corr;     // TQ3 K corrections [NT][D/32][4 column pairs] as {c0, c1, c0, c1}
+  float2* corr;     // TQ3 K corrections [NT][D/32][4 column pairs]
   uint8_t* ring;
 };
 
-template <int D, int NT>
+template <int D, int NT, int K>
 __device__ __forceinline__ Smem carve(uint8_t* base) {
-  using C = Cfg<D, NT>;
+  using C = Cfg<D, NT, K>;
   Smem s;
   s.full = reinterpret_cast<uint64_t*>(base);
-  s.empty = s.full + 16;
-  s.tag = reinterpret_cast<int32_t*>(base + C::OFF_TAG);
+  s.cnt = reinterpret_cast<int32_t*>(base + C::OFF_CNT);
+  s.fills = reinterpret_cast<int32_t*>(base + C::OFF_FILLS);
   s.misc = reinterpret_cast<int32_t*>(base + C::OFF_MISC);
   s.list = reinterpret_cast<int2*>(base + C::OFF_LIST);
   s.qf = reinterpret_cast<uint4*>(base + C::OFF_QF);
-  s.corr = reinterpret_cast<float4*>(base + C::OFF_CORR);
+  s.corr = reinterpret_cast<float2*>(base + C::OFF_CORR);
   s.ring = base + C::OFF_RING;
   return s;
 }
@@ -117,11 +140,12 @@ struct VState {
 };
 
 // Logits -> probabilities for one page (thread holds logits x[0..3] for tokens (r, r+8) x
-// columns (2c, 2c+1), in log2 units).  Gives P^T as two B fragments (tokens 0-7, 8-15) and the
+// columns (2c, 2c+1), in log2 units).  Gives the probabilities pr (same positions) and the
 // factors (a0, a1) by which earlier accumulations of the two columns must be rescaled (1 when
-// the reference maximum did not move).
-__device__ __forceinline__ void softmax_k(KState& st, float (&x)[4], uint32_t& pb0,
-                                          uint32_t& pb1, float& a0, float& a1) {
+// the reference maximum did not move).  P^T as B fragments (tokens 0-7, 8-15) is the movmatrix
+// transpose of the packed pairs (pr0, pr1) and (pr2, pr3).
+__device__ __forceinline__ void softmax_k(KState& st, float (&x)[4], float (&pr)[4], float& a0,
+                                          float& a1) {
   float mx0 = fmaxf(x[0], x[2]);
   float mx1 = fmaxf(x[1], x[3]);
   a0 = a1 = 1.f;
@@ -142,12 +166,12 @@ __device__ __forceinline__ void softmax_k(KState& st, float (&x)[4], uint32_t& p
   }
   const float r0 = st.m[0] == -INFINITY ? 0.f : st.m[0];
   const float r1 = st.m[1] == -INFINITY ? 0.f : st.m[1];
-  const float p0 = fast_exp2(x[0] - r0), p1 = fast_exp2(x[1] - r1);
-  const float p2 = fast_exp2(x[2] - r0), p3 = fast_exp2(x[3] - r1);
-  st.l[0] += p0 + p2;
-  st.l[1] += p1 + p3;
-  pb0 = movmatrix_trans(pack_f16x2(p0, p1));
-  pb1 = movmatrix_trans(pack_f16x2(p2, p3));
+  pr[0] = fast_exp2(x[0] - r0);
+  pr[1] = fast_exp2(x[1] - r1);
+  pr[2] = fast_exp2(x[2] - r0);
+  pr[3] = fast_exp2(x[3] - r1);
+  st.l[0] += pr[0] + pr[2];
+  st.l[1] += pr[1] + pr[3];
 }
 
 __device__ __forceinline__ void mask_page(float (&x)[4], int tok0, int r, int lim0, int lim1) {
@@ -163,14 +187,15 @@ __device__ __forceinline__ void mask_page(float (&x)[4], int tok0, int r, int li
 // un-permuted when stored): TQ3 K, group G, lane quad column c: MMA k 2c,2c+1 <- channels
 // 8c+0, 8c+4 (k-block 0), 8c+1, 8c+5 (k-block 0, upper k), 8c+2, 8c+6 / 8c+3, 8c+7 (k-block 1).
 template <int D>
-__device__ __forceinline__ void tq3_logits(const uint8_t* pg, const uint4* qf, const float4* corr,
-                                           int lane, int kw, int ks5, float (&x)[4]) {
+__device__ __forceinline__ void tq3_logits(const uint8_t* pg, const uint4* qf, const float2* corr,
+                                           int lane, int kw, int ks, float (&x)[4]) {
   constexpr int G = D / 32;
   const int r = lane >> 2, c = lane & 3;
   const uint8_t* krec = pg;
   const __half* kscale = reinterpret_cast<const __half*>(pg + G * 16 * 12);
-  // K images: code k of a pair lands in mantissa bits 7-9 of the low half (value 8 + c) and
-  // code k+4 in bits 3-5 of the high half (value 128 + c); both exact.  The offsets 11.5 and
+  // K images: the window puts code j of the lane's 8-code chunk at bit 7 + 3j, so code k of a
+  // pair lands in mantissa bits 7-9 of the low half (value 8 + c) and code k+4 in bits 3-5 of
+  // the high half (value 128 + c) after a right shift by 3k; both exact.  The offsets 11.5 and
   // 131.5 (base + 3.5) times the query sums are the group's starting accumulator (corr).
   uint32_t kMask = 0x00380380u, kMagic = 0x58004800u;
   opaque(kMask, kMagic);
@@ -179,16 +204,16 @@ __device__ __forceinline__ void tq3_logits(const uint8_t* pg, const uint4* qf, c
   for (int g = 0; g < G; ++g) {
     const uint32_t* ra = reinterpret_cast<const uint32_t*>(krec + 12 * (16 * g + r));
     const uint32_t* rb = ra + 24;  // token r + 8
-    const uint32_t xa = __funnelshift_r(ra[kw], ra[kw + 1], ks5);  // code j at bit 3j+5
-    const uint32_t xb = __funnelshift_r(rb[kw], rb[kw + 1], ks5);
-    const uint32_t a0 = and_or(xa << 2, kMask, kMagic), b0 = and_or(xb << 2, kMask, kMagic);
-    const uint32_t a1 = and_or(xa >> 1, kMask, kMagic), b1 = and_or(xb >> 1, kMask, kMagic);
-    const uint32_t a2 = and_or(xa >> 4, kMask, kMagic), b2 = and_or(xb >> 4, kMask, kMagic);
-    const uint32_t a3 = and_or(xa >> 7, kMask, kMagic), b3 = and_or(xb >> 7, kMask, kMagic);
+    const uint32_t xa = __funnelshift_r(ra[kw], ra[kw + 1], ks);  // code j at bit 3j+7
+    const uint32_t xb = __funnelshift_r(rb[kw], rb[kw + 1], ks);
+    const uint32_t a0 = and_or(xa, kMask, kMagic), b0 = and_or(xb, kMask, kMagic);
+    const uint32_t a1 = and_or(xa >> 3, kMask, kMagic), b1 = and_or(xb >> 3, kMask, kMagic);
+    const uint32_t a2 = and_or(xa >> 6, kMask, kMagic), b2 = and_or(xb >> 6, kMask, kMagic);
+    const uint32_t a3 = and_or(xa >> 9, kMask, kMagic), b3 = and_or(xb >> 9, kMask, kMagic);
     const uint4 qb = qf[32 * g + lane];
-    const float4 cr = corr[4 * g + c];
-    float cg[4] = {cr.x, cr.y, cr.z, cr.w};
-    mma_f16_16816(cg, a0, b0, a1, b1, qb.x, qb.y, cg);
+    const float2 cr = corr[4 * g + c];
+    float cg[4];
+    mma_f16_16816(cg, a0, b0, a1, b1, qb.x, qb.y, {cr.x, cr.y, cr.x, cr.y});
     mma_f16_16816(cg, a2, b2, a3, b3, qb.z, qb.w, cg);
     const float sa = __half2float(kscale[16 * g + r]);
     const float sb = __half2float(kscale[16 * g + r + 8]);
@@ -199,10 +224,41 @@ __device__ __forceinline__ void tq3_logits(const uint8_t* pg, const uint4* qf, c
   }
 }
 
+// Largest V scale of a TQ3 page (f16 bits; scales are never negative), the same on every lane:
+// each lane folds G bytes of the page's [G][16] f16 V scales, then one warp reduction.
+template <int D>
+__device__ __forceinline__ uint32_t tq3_v_scale_max(const uint8_t* pg, int lane) {
+  constexpr int G = D / 32;
+  const uint8_t* vs = pg + G * 16 * 14 + G * 16 * 12;
+  uint32_t w;
+  if constexpr (G == 8) {
+    const uint2 x = reinterpret_cast<const uint2*>(vs)[lane];
+    w = hmax2_u32(x.x, x.y);
+  } else if constexpr (G == 4) {
+    w = reinterpret_cast<const uint32_t*>(vs)[lane];
+  } else {
+    w = reinterpret_cast<const uint16_t*>(vs)[lane];
+  }
+  return __reduce_max_sync(0xffffffffu, max(w & 0xffffu, w >> 16));
+}
+
+// A page's V scales all lie at or below 2^7 and the largest at or above 2^-6 (f16 bits): then
+// P * s, with P <= 2^8 under the lazy softmax reference, is at most 2^15 and, for the page's
+// largest scales, a normal f16 down to P = 2^-8, so the plain f16 product keeps full precision.
+constexpr uint32_t kVScaleLo = 0x2400u;  // 2^-6
+constexpr uint32_t kVScaleHi = 0x5800u;  // 2^7
+
 // V: A = V^T tile (channels x tokens); lane row r holds channels 32G+4r+{0,1} (tile 2G) and
 // 32G+4r+{2,3} (tile 2G+1) for tokens (2c, 2c+1) and (2c+8, 2c+9); codes -> exact (c - 3.5);
 // the per-(token, group) scale multiplies P in f16.
-template <int D>
+//
+// WIDE is the path for pages whose scale maximum is outside [2^-6, 2^7]: each group's 16 token
+// scales are first divided by a power of two 2^(e-16) taken from the group's largest scale on
+// the page (quad reduction; e its biased f16 exponent, at least 1), so the scaled values are
+// below 4 and P * s / 2^(e-16) < 2^10 cannot overflow, while the group's largest products stay
+// normal f16 down to P = 2^-16; the group's P.V tiles are computed from zero and added to the
+// accumulator times 2^(e-16) in fp32, exactly undoing the division.
+template <int D, bool WIDE>
 __device__ __forceinline__ void tq3_pv(VState<D>& st, const uint8_t* pg, int lane, int vw,
                                        int vs1, uint32_t pb0, uint32_t pb1) {
   constexpr int G = D / 32;
@@ -228,11 +284,31 @@ __device__ __forceinline__ void tq3_pv(VState<D>& st, const uint8_t* pg, int lan
     const uint32_t a2 = hsub2_u32(and_or(z01, m2, g2), s2), b2 = hsub2_u32(and_or(z89, m2, g2), s2);
     const uint32_t a3 = hsub2_u32(and_or(z01 >> 3, m2, g2), s2);
     const uint32_t b3 = hsub2_u32(and_or(z89 >> 3, m2, g2), s2);
-    const uint32_t sv0 = *reinterpret_cast<const uint32_t*>(vscale + 16 * g + 2 * c);
-    const uint32_t sv8 = *reinterpret_cast<const uint32_t*>(vscale + 16 * g + 2 * c + 8);
-    const uint32_t q0 = hmul2_u32(pb0, sv0), q1 = hmul2_u32(pb1, sv8);
-    mma_f16_16816(st.acc[2 * g], a0, a1, b0, b1, q0, q1, st.acc[2 * g]);
-    mma_f16_16816(st.acc[2 * g + 1], a2, a3, b2, b3, q0, q1, st.acc[2 * g + 1]);
+    uint32_t sv0 = *reinterpret_cast<const uint32_t*>(vscale + 16 * g + 2 * c);
+    uint32_t sv8 = *reinterpret_cast<const uint32_t*>(vscale + 16 * g + 2 * c + 8);
+    if constexpr (!WIDE) {
+      const uint32_t q0 = hmul2_u32(pb0, sv0), q1 = hmul2_u32(pb1, sv8);
+      mma_f16_16816(st.acc[2 * g], a0, a1, b0, b1, q0, q1, st.acc[2 * g]);
+      mma_f16_16816(st.acc[2 * g + 1], a2, a3, b2, b3, q0, q1, st.acc[2 * g + 1]);
+    } else {
+      uint32_t m = hmax2_u32(sv0, sv8);  // tokens 2c, 2c+1, 2c+8, 2c+9; the quad holds all 16
+      m = hmax2_u32(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = hmax2_u32(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      const int e = max(static_cast<int>(max(m & 0xffffu, m >> 16) >> 10), 1);
+      const uint32_t down = static_cast<uint32_t>(31 - e) * 0x04000400u;  // f16x2 2^(16-e)
+      const float up = __int_as_float((e + 111) << 23);                   // fp32 2^(e-16)
+      sv0 = hmul2_u32(sv0, down);
+      sv8 = hmul2_u32(sv8, down);
+      const uint32_t q0 = hmul2_u32(pb0, sv0), q1 = hmul2_u32(pb1, sv8);
+      float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
+      mma_f16_16816(t0, a0, a1, b0, b1, q0, q1, t0);
+      mma_f16_16816(t1, a2, a3, b2, b3, q0, q1, t1);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        st.acc[2 * g][j] = fmaf(up, t0[j], st.acc[2 * g][j]);
+        st.acc[2 * g + 1][j] = fmaf(up, t1[j], st.acc[2 * g + 1][j]);
+      }
+    }
   }
 }
 
@@ -294,6 +370,59 @@ __device__ __forceinline__ void fp8_pv(VState<D>& st, const uint8_t* pg, int lan
     }
   }
 }
+
+// ------------------------------------------------------------------ BF16 control page
+// Stage rows (ROW = 2D + 16 bytes): K token t at t*ROW, V token t at (16 + t)*ROW.  The values
+// are the stored bf16, so both contractions use bf16 MMAs on them directly; Q is bf16 too.
+// Logits: A = K (16 tokens x 16 channels per k-step) by ldmatrix, B = Q fragments
+// [D/32][32 lanes] {k-step 2w: b0, b1 | k-step 2w+1: b0, b1}.
+template <int D>
+__device__ __forceinline__ void bf16_logits(const uint8_t* pg, const uint4* qf, int lane,
+                                            float (&x)[4]) {
+  constexpr int ROW = 2 * D + 16;
+  const int m = lane >> 3;
+  const uint8_t* base = pg + ((m & 1) * 8 + (lane & 7)) * ROW + (m >> 1) * 16;
+  float cg[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int w = 0; w < D / 32; ++w) {
+    const uint4 qb = qf[32 * w + lane];
+    uint32_t a[4];
+    ldmatrix_x4(a, base + 64 * w);
+    mma_bf16_16816(cg, a[0], a[1], a[2], a[3], qb.x, qb.y, cg);
+    ldmatrix_x4(a, base + 64 * w + 32);
+    mma_bf16_16816(cg, a[0], a[1], a[2], a[3], qb.z, qb.w, cg);
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) x[j] = cg[j];
+}
+
+// P.V: A = V^T tile mt (channels 16mt.., tokens) by transposing ldmatrix of the V rows; P is
+// split into bf16 hi + lo parts (about 16 significant bits) and both are multiplied in.
+// acc[mt]: rows r, r+8 = channels 16mt + r, 16mt + 8 + r.
+template <int D>
+__device__ __forceinline__ void bf16_pv(VState<D>& st, const uint8_t* pg, int lane,
+                                        const float (&pr)[4]) {
+  constexpr int ROW = 2 * D + 16;
+  const uint32_t h01 = pack_bf16x2(pr[0], pr[1]), h23 = pack_bf16x2(pr[2], pr[3]);
+  const uint32_t l01 = pack_bf16x2(pr[0] - bf16_lo(h01), pr[1] - bf16_hi(h01));
+  const uint32_t l23 = pack_bf16x2(pr[2] - bf16_lo(h23), pr[3] - bf16_hi(h23));
+  const uint32_t ph0 = movmatrix_trans(h01), ph1 = movmatrix_trans(h23);
+  const uint32_t pl0 = movmatrix_trans(l01), pl1 = movmatrix_trans(l23);
+  const uint8_t* base =
+      pg + (16 + (lane & 7) + 8 * (lane >> 4)) * ROW + 16 * ((lane >> 3) & 1);
+#pragma unroll
+  for (int mt = 0; mt < D / 16; ++mt) {
+    uint32_t a[4];
+    ldmatrix_x4_trans(a, base + 32 * mt);
+    mma_bf16_16816(st.acc[mt], a[0], a[1], a[2], a[3], ph0, ph1, st.acc[mt]);
+    mma_bf16_16816(st.acc[mt], a[0], a[1], a[2], a[3], pl0, pl1, st.acc[mt]);
+  }
+}
+
+// bf16 Q fragments of n-tile nt in natural channel order (exact; no scaling, no correction).
+template <int D>
+__device__ __forceinline__ float build_q_bf16(const DecodeParams& p, const SeqDesc& sd, int h,
+                                              int nt, int lane, uint4* qf);
 
 // Query column n of this CTA's KV head -> its bf16 row, or nullptr for padding columns.
 __device__ __forceinline__ const uint16_t* q_row(const DecodeParams& p, const SeqDesc& sd,
@@ -357,21 +486,32 @@ __device__ __forceinline__ float build_q(const DecodeParams& p, const SeqDesc& s
       float part = -(11.5f * lo + 131.5f * hi);
       part += __shfl_xor_sync(0xffffffffu, part, 1);
       part += __shfl_xor_sync(0xffffffffu, part, 2);
-      if (c == 0) {  // stored twice per column pair: {col 2k, col 2k+1, col 2k, col 2k+1}
-        float* c4 = corr + 16 * w + 4 * (r >> 1) + (r & 1);
-        c4[0] = part;
-        c4[2] = part;
-      }
+      if (c == 0) corr[8 * w + r] = part;  // [group][column pair][2]: column r = 2(r/2) + r%2
     }
     qf[32 * w + lane] = f;
   }
   return p.logit_scale * ldexpf(1.f, -e);
 }
 
-// Producer warp: collect the unit's pages of format fmt from table entries [first, last).
+template <int D>
+__device__ __forceinline__ float build_q_bf16(const DecodeParams& p, const SeqDesc& sd, int h,
+                                              int nt, int lane, uint4* qf) {
+  const int r = lane >> 2, c = lane & 3;
+  const uint16_t* qr = q_row(p, sd, h, 8 * nt + r);
+  auto pair = [&](int ch) -> uint32_t {
+    return qr ? static_cast<uint32_t>(qr[ch]) | (static_cast<uint32_t>(qr[ch + 1]) << 16) : 0u;
+  };
+#pragma unroll
+  for (int w = 0; w < D / 32; ++w)
+    qf[32 * w + lane] = make_uint4(pair(32 * w + 2 * c), pair(32 * w + 8 + 2 * c),
+                                   pair(32 * w + 16 + 2 * c), pair(32 * w + 24 + 2 * c));
+  return p.logit_scale;
+}
+
+// Scanner warp: collect the unit's pages of format fmt from table entries [first, last).
 __device__ __forceinline__ int scan_range(const DecodeParams& p, const int32_t* row, int first,
                                           int last, int fmt, int lane, int2* list) {
-  const int nslots = fmt == 0 ? p.fp8_slots : p.tq3_slots;
+  const int nslots = fmt == 1 ? p.tq3_slots : p.fp8_slots;
   const unsigned lt = (1u << lane) - 1u;
   int count = 0;
   bool bad = false;
@@ -380,15 +520,16 @@ __device__ __forceinline__ int scan_range(const DecodeParams& p, const int32_t* 
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int idx = base + 32 * j + lane;
-      e[j] = idx < last ? row[idx] : -2;
+      e[j] = idx < last ? row[idx] : -1;
     }
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int idx = base + 32 * j + lane;
       const uint32_t f = static_cast<uint32_t>(e[j]) >> kFmtShift;
       const int slot = static_cast<int>(static_cast<uint32_t>(e[j]) & kSlotMask);
-      const bool mapped = e[j] >= 0;
-      bad |= (idx < last) && (!mapped || f > 1 || slot >= (f == 0 ? p.fp8_slots : p.tq3_slots));
+      const bool mapped = e[j] != -1;  // a BF16 entry (format 2) has the sign bit set
+      const bool known = f == 1 || static_cast<int>(f) == p.page_fmt;
+      bad |= (idx < last) && (!mapped || !known || slot >= (f == 1 ? p.tq3_slots : p.fp8_slots));
       const bool take = mapped && static_cast<int>(f) == fmt && slot < nslots;
       const unsigned b = __ballot_sync(0xffffffffu, take);
       const int pos = count + __popc(b & lt);
@@ -404,46 +545,79 @@ __device__ __forceinline__ int scan_range(const DecodeParams& p, const int32_t* 
   return count;
 }
 
-template <int D, int NT, bool FP8>
+// Page geometry of a format inside a partial kernel of kind K.
+template <int D, int NT, int K, int F>
+struct Page {
+  using C = Cfg<D, NT, K>;
+  static constexpr int STAGE = F == kFp8 ? C::FP8_STAGE : (F == kTq3 ? C::TQ3_STAGE : C::BF16_STAGE);
+  static constexpr int NST = F == kFp8 ? C::FP8_NST : (F == kTq3 ? C::TQ3_NST : C::BF16_NST);
+  // bytes of one KV head in a slot of the format
+  static constexpr int HEAD = F == kFp8 ? 32 * D + 16 : (F == kTq3 ? 14 * D : 64 * D);
+};
+
+// Warp-collective: start the bulk copy of page i of the unit (list entry i) into its ring
+// stage.  FP8 and TQ3 pages are one contiguous copy issued by lane 0; a BF16 page is 32 row
+// copies, one per lane, into padded stage rows.
+template <class PG, int F>
+__device__ __forceinline__ void fill_stage(const Smem& sm, const uint8_t* slab, int64_t slot_bytes,
+                                           int h, int i, int lane) {
+  const int s = i % PG::NST;
+  const int2 e = sm.list[i];
+  const uint8_t* src = slab + static_cast<int64_t>(e.x) * slot_bytes +
+                       static_cast<int64_t>(h) * PG::HEAD;
+  if (lane == 0) {
+    sm.fills[s] += 1;
+    mbar_arrive_expect_tx(&sm.full[s], PG::HEAD);
+  }
+  if constexpr (F == kBf16) {
+    constexpr int ROWB = PG::HEAD / 32;  // 2D bytes
+    __syncwarp();
+    bulk_g2s(sm.ring + s * PG::STAGE + lane * (ROWB + 16), src + lane * ROWB, ROWB, &sm.full[s]);
+  } else {
+    if (lane == 0) bulk_g2s(sm.ring + s * PG::STAGE, src, PG::STAGE, &sm.full[s]);
+  }
+}
+
+template <int D, int NT, int K, int F>
 __device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDesc& u, int h,
                          Smem sm) {
-  using C = Cfg<D, NT>;
-  constexpr int STAGE = FP8 ? C::FP8_STAGE : C::TQ3_STAGE;
-  constexpr int NST = FP8 ? C::FP8_NST : C::TQ3_NST;
+  using C = Cfg<D, NT, K>;
+  using PG = Page<D, NT, K, F>;
+  constexpr int STAGE = PG::STAGE;
+  constexpr int NST = PG::NST;
+  constexpr int SCANNER = C::WARPS - 1;  // the warp that scans the range and starts the copies
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = lane >> 2, c = lane & 3;
   const int nt = warp % NT, pw = warp / NT;
 
-  const uint8_t* slab = FP8 ? p.fp8_slab : p.tq3_slab;
-  const int64_t slot_bytes = FP8 ? p.fp8_slot_bytes : p.tq3_slot_bytes;
-  if (warp == C::PRODUCER) {
-    // the producer owns the ring set-up, so its first fills (which need no free stage) are in
-    // flight while the consumers build their Q fragments
+  const uint8_t* slab = F == kTq3 ? p.tq3_slab : p.fp8_slab;
+  const int64_t slot_bytes = F == kTq3 ? p.tq3_slot_bytes : p.fp8_slot_bytes;
+  if (warp == SCANNER) {
+    // the first fills are in flight while the other warps build their Q fragments
     if (lane == 0) {
       for (int s = 0; s < NST; ++s) {
         mbar_init(&sm.full[s], 1);
-        mbar_init(&sm.empty[s], NT);
+        sm.cnt[s] = 0;
+        sm.fills[s] = 0;
       }
       sm.misc[1] = 0;
       mbar_fence_init();
     }
-    const int32_t* row = p.tables + static_cast<int64_t>(sd.row) * p.max_pages;
-    const int n = scan_range(p, row, u.first, u.last, FP8 ? 0 : 1, lane, sm.list);
     __syncwarp();
-    if (lane == 0) {
-      sm.misc[0] = n;
-      for (int i = 0; i < min(n, NST); ++i) {
-        const int2 e = sm.list[i];
-        sm.tag[i] = e.y;
-        mbar_arrive_expect_tx(&sm.full[i], STAGE);
-        bulk_g2s(sm.ring + i * STAGE,
-                 slab + static_cast<int64_t>(e.x) * slot_bytes + static_cast<int64_t>(h) * STAGE,
-                 STAGE, &sm.full[i]);
-      }
-    }
-  } else if (pw == 0) {
-    const float ls = build_q<D, FP8>(p, sd, h, nt, lane, sm.qf + nt * (D / 32) * 32,
-                                     reinterpret_cast<float*>(sm.corr + nt * (D / 32) * 4));
+    const int32_t* row = p.tables + static_cast<int64_t>(sd.row) * p.max_pages;
+    const int n = scan_range(p, row, u.first, u.last, F, lane, sm.list);
+    __syncwarp();
+    if (lane == 0) sm.misc[0] = n;
+    for (int i = 0; i < min(n, NST); ++i) fill_stage<PG, F>(sm, slab, slot_bytes, h, i, lane);
+  }
+  if (pw == 0) {
+    uint4* qf = sm.qf + nt * (D / 32) * 32;
+    float ls;
+    if constexpr (F == kBf16)
+      ls = build_q_bf16<D>(p, sd, h, nt, lane, qf);
+    else
+      ls = build_q<D, F == kFp8>(p, sd, h, nt, lane, qf,
+                                 reinterpret_cast<float*>(sm.corr + nt * (D / 32) * 4));
     if (lane == 0) reinterpret_cast<float*>(sm.misc)[4 + nt] = ls;
   }
   __syncthreads();
@@ -453,43 +627,17 @@ __device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDes
   VState<D> vs;
   ks.m[0] = ks.m[1] = -INFINITY;
   ks.l[0] = ks.l[1] = 0.f;
-  if (warp == C::PRODUCER) {
-    // ---------------- producer: one lane streams the unit's pages into the ring
-    if (lane == 0) {
-      int issued = min(count, NST);
-      for (int i = issued; i < count; ++i) {
-        const int s = i % NST;
-        if (i >= NST && !mbar_wait(&sm.empty[s], ((i / NST) - 1) & 1)) {
-          flag_status(p.status, kStatusTimeout);
-          atomicExch(&sm.misc[1], 1);
-          break;
-        }
-        const int2 e = sm.list[i];
-        sm.tag[s] = e.y;
-        mbar_arrive_expect_tx(&sm.full[s], STAGE);
-        bulk_g2s(sm.ring + s * STAGE,
-                 slab + static_cast<int64_t>(e.x) * slot_bytes + static_cast<int64_t>(h) * STAGE,
-                 STAGE, &sm.full[s]);
-        issued = i + 1;
-      }
-      if (*reinterpret_cast<volatile int32_t*>(&sm.misc[1])) {
-        // drain: wait (bounded) for the last fill of every stage so no copy is in flight
-        for (int i = max(0, issued - NST); i < issued; ++i)
-          mbar_wait(&sm.full[i % NST], (i / NST) & 1, 100000000ull);
-      }
-    }
-  } else {
-    // ---------------- consumers: logits, online softmax, P.V per page
+  {
     const int n0 = 8 * nt + 2 * c, n1 = n0 + 1;
     const int lim0 = n0 < p.NC ? sd.ctx - p.q_len + n0 / p.g : sd.ctx - 1;
     const int lim1 = n1 < p.NC ? sd.ctx - p.q_len + n1 / p.g : sd.ctx - 1;
     const int min_lim = sd.ctx - p.q_len;
     const float ls = reinterpret_cast<const float*>(sm.misc)[4 + nt];
     const uint4* qf = sm.qf + nt * (D / 32) * 32;
-    const float4* corr = sm.corr + nt * (D / 32) * 4;
-    // TQ3 K chunk c of a record starts at bit 24c; read from bit 24c-5 (codes at 5+3k).
+    const float2* corr = sm.corr + nt * (D / 32) * 4;
+    // TQ3 K chunk c of a record starts at bit 24c; read from bit 24c-7 (codes at 7+3k).
     // TQ3 V field of row r starts at bit 12r; read from bit 12r-1 (codes at 1+3k).
-    const int kbit = 24 * c - 5, vbit = 12 * r - 1;
+    const int kbit = 24 * c - 7, vbit = 12 * r - 1;
     const int kw = kbit >= 0 ? kbit >> 5 : -1, ks5 = kbit & 31;
     const int vw = vbit >= 0 ? vbit >> 5 : -1, vs1 = vbit & 31;
 #pragma unroll
@@ -497,6 +645,7 @@ __device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDes
 #pragma unroll
       for (int e = 0; e < 4; ++e) vs.acc[mt][e] = 0.f;
 
+    bool aborted = false;
     for (int i = pw; i < count; i += C::PW) {
       const int s = i % NST;
       if (!mbar_wait_warp(&sm.full[s], (i / NST) & 1)) {
@@ -504,21 +653,24 @@ __device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDes
           flag_status(p.status, kStatusTimeout);
           atomicExch(&sm.misc[1], 1);
         }
+        aborted = true;
         break;
       }
-      const int tok0 = 16 * sm.tag[s];
+      const int tok0 = 16 * sm.list[i].y;
       const uint8_t* pg = sm.ring + s * STAGE;
       float x[4];
-      if constexpr (FP8)
+      if constexpr (F == kFp8)
         fp8_logits<D>(pg, qf, lane, x);
-      else
+      else if constexpr (F == kTq3)
         tq3_logits<D>(pg, qf, corr, lane, kw, ks5, x);
+      else
+        bf16_logits<D>(pg, qf, lane, x);
 #pragma unroll
       for (int j = 0; j < 4; ++j) x[j] *= ls;
       if (tok0 + 15 > min_lim) mask_page(x, tok0, r, lim0, lim1);
-      uint32_t pb0, pb1;
+      float pr[4];
       float a0, a1;
-      softmax_k(ks, x, pb0, pb1, a0, a1);
+      softmax_k(ks, x, pr, a0, a1);
       if (__any_sync(0xffffffffu, a0 != 1.f || a1 != 1.f)) {
 #pragma unroll
         for (int mt = 0; mt < D / 16; ++mt) {
@@ -528,17 +680,51 @@ __device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDes
           vs.acc[mt][3] *= a1;
         }
       }
-      if constexpr (FP8)
-        fp8_pv<D>(vs, pg, lane, pb0, pb1);
-      else
-        tq3_pv<D>(vs, pg, lane, vw, vs1, pb0, pb1);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.empty[s]);
+      if constexpr (F == kBf16) {
+        bf16_pv<D>(vs, pg, lane, pr);
+      } else {
+        const uint32_t pb0 = movmatrix_trans(pack_f16x2(pr[0], pr[1]));
+        const uint32_t pb1 = movmatrix_trans(pack_f16x2(pr[2], pr[3]));
+        if constexpr (F == kFp8) {
+          fp8_pv<D>(vs, pg, lane, pb0, pb1);
+        } else {
+          const uint32_t vmax = tq3_v_scale_max<D>(pg, lane);
+          if (vmax >= kVScaleLo && vmax <= kVScaleHi)
+            tq3_pv<D, false>(vs, pg, lane, vw, vs1, pb0, pb1);
+          else
+            tq3_pv<D, true>(vs, pg, lane, vw, vs1, pb0, pb1);
+        }
+      }
+      // release the stage: its owner refills it with the page one ring-length ahead.  Every
+      // lane's reads of the stage are ordered before the async-proxy overwrite.
+      if (i + NST < count) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        bool last = true;
+        if constexpr (NT > 1) {  // the n-tile warps of this page: the last one done refills
+          if (lane == 0) {
+            __threadfence_block();
+            last = atomicAdd(&sm.cnt[s], 1) == NT - 1;
+            if (last) sm.cnt[s] = 0;
+            __threadfence_block();
+          }
+          last = __shfl_sync(0xffffffffu, last, 0);
+        }
+        if (last) fill_stage<PG, F>(sm, slab, slot_bytes, h, i + NST, lane);
+      }
     }
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
       ks.l[0] += __shfl_xor_sync(0xffffffffu, ks.l[0], o);
       ks.l[1] += __shfl_xor_sync(0xffffffffu, ks.l[1], o);
+    }
+    if (aborted && lane == 0) {
+      // drain: wait (bounded) for the last copy issued into each of this group's stages, so
+      // none is in flight when the CTA's shared memory is released
+      for (int s = pw; s < NST; s += C::PW) {
+        const int f = *reinterpret_cast<volatile int32_t*>(&sm.fills[s]);
+        if (f > 0) mbar_wait(&sm.full[s], (f - 1) & 1, 100000000ull);
+      }
     }
   }
   __syncthreads();  // ring no longer needed: reuse it for the cross-warp combine
@@ -547,7 +733,7 @@ __device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDes
   // columns' channels: M = max m, l = sum l 2^(m-M), acc = sum acc 2^(m-M)
   float* cmb = reinterpret_cast<float*>(sm.ring);
   constexpr int REGION = 8 * (D + 2);  // per (warp, n-tile): (m, l) of 8 columns, then acc [8][D]
-  if (warp < C::NWC) {
+  {
     float* reg = cmb + (pw * NT + nt) * REGION;
     if (r == 0) {
       reg[2 * (2 * c)] = ks.m[0];
@@ -558,15 +744,17 @@ __device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDes
     float* ra = reg + 16;
 #pragma unroll
     for (int mt = 0; mt < D / 16; ++mt) {
-      const int ch = 32 * (mt >> 1) + 4 * r + 2 * (mt & 1);
-      ra[(2 * c) * D + ch] = vs.acc[mt][0];
-      ra[(2 * c + 1) * D + ch] = vs.acc[mt][1];
-      ra[(2 * c) * D + ch + 1] = vs.acc[mt][2];
-      ra[(2 * c + 1) * D + ch + 1] = vs.acc[mt][3];
+      // channels of accumulator rows r and r + 8 of tile mt
+      const int ch0 = F == kBf16 ? 16 * mt + r : 32 * (mt >> 1) + 4 * r + 2 * (mt & 1);
+      const int ch1 = F == kBf16 ? ch0 + 8 : ch0 + 1;
+      ra[(2 * c) * D + ch0] = vs.acc[mt][0];
+      ra[(2 * c + 1) * D + ch0] = vs.acc[mt][1];
+      ra[(2 * c) * D + ch1] = vs.acc[mt][2];
+      ra[(2 * c + 1) * D + ch1] = vs.acc[mt][3];
     }
   }
   __syncthreads();
-  if (warp < C::NWC) {
+  {
     const int part = sd.part0 + u.part;
     const float* regs = cmb + nt * REGION;  // warp w's region: regs + w * NT * REGION
     for (int q = pw * 32 + lane; q < 8 * (D / 4); q += 32 * C::PW) {
@@ -612,6 +800,9 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
   __shared__ float w[kDecodeMaxUnits];
   __shared__ float red[kMergeThreads / 32];
   __shared__ float4 part[kMergeThreads];
+  // launched as a programmatic dependent of the partial kernels: resident early, it reads the
+  // partial states only once they are complete and visible
+  pdl_wait();
   const int pair = blockIdx.x / p.NC, n = blockIdx.x % p.NC;
   const SeqDesc& sd = p.seq[pair / p.Hkv];
   const int h = pair % p.Hkv;
@@ -668,33 +859,49 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
   }
 }
 
-template <int D, int NT>
-__global__ void __launch_bounds__(Cfg<D, NT>::THREADS, D == 256 ? 3 : 4)
-    decode_kernel(const __grid_constant__ DecodeParams p) {
+// Partial-attention kernel of one kind.  Grid = units x KV heads; the FP8 grid covers units
+// [0, n_fp8), the TQ3 grid [n_fp8, n_units), the fused and BF16 grids all of them.
+template <int D, int NT, int K>
+__global__ void __launch_bounds__(Cfg<D, NT, K>::THREADS, Cfg<D, NT, K>::MINB)
+    partial_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  const Smem sm = carve<D, NT>(smem_raw);
+  // let the next kernel of the call (the TQ3 grid or the merge) start once every CTA of this
+  // grid is resident: it reads nothing this grid writes before its griddepcontrol.wait
+  pdl_launch_dependents();
+  const Smem sm = carve<D, NT, K>(smem_raw);
   const int h = blockIdx.x % p.Hkv;
-  const UnitDesc& u = p.unit[blockIdx.x / p.Hkv];
+  const UnitDesc& u = p.unit[(K == kKindTq3 ? p.n_fp8 : 0) + blockIdx.x / p.Hkv];
   const SeqDesc& sd = p.seq[u.seq];
-  if (u.fmt == 0)
-    run_unit<D, NT, true>(p, sd, u, h, sm);
-  else
-    run_unit<D, NT, false>(p, sd, u, h, sm);
+  if constexpr (K == kKindFp8) {
+    run_unit<D, NT, K, kFp8>(p, sd, u, h, sm);
+  } else if constexpr (K == kKindTq3) {
+    run_unit<D, NT, K, kTq3>(p, sd, u, h, sm);
+    // the TQ3 grid, a programmatic dependent of the FP8 grid, ends only after it: the merge, a
+    // dependent of this grid, then sees both grids' partial states
+    pdl_wait();
+  } else if constexpr (K == kKindBf16) {
+    run_unit<D, NT, K, kBf16>(p, sd, u, h, sm);
+  } else {
+    if (u.fmt == kFp8)
+      run_unit<D, NT, K, kFp8>(p, sd, u, h, sm);
+    else
+      run_unit<D, NT, K, kTq3>(p, sd, u, h, sm);
+  }
 }
 
 // Per-instantiation launch set-up, done once: the dynamic shared-memory opt-in and the number of
 // CTAs the SM keeps resident (the planner sizes work units from it).
-template <int D, int NT>
+template <int D, int NT, int K>
 struct KernelInfo {
   cudaError_t err = cudaSuccess;
   int ctas_per_sm = 1;
   KernelInfo() {
-    using C = Cfg<D, NT>;
-    err = cudaFuncSetAttribute(decode_kernel<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               C::SMEM);
+    using C = Cfg<D, NT, K>;
+    err = cudaFuncSetAttribute(partial_kernel<D, NT, K>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     int n = 0;
     if (err == cudaSuccess)
-      err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<D, NT>, C::THREADS,
+      err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, partial_kernel<D, NT, K>, C::THREADS,
                                                           C::SMEM);
     ctas_per_sm = n > 0 ? n : 1;
   }
@@ -704,44 +911,82 @@ struct KernelInfo {
   }
 };
 
-template <int D, int NT>
-cudaError_t launch_t(const DecodeParams& p, cudaStream_t s) {
-  using C = Cfg<D, NT>;
-  const KernelInfo<D, NT>& info = KernelInfo<D, NT>::get();
-  if (info.err != cudaSuccess) return info.err;
-  decode_kernel<D, NT><<<p.n_units * p.Hkv, C::THREADS, C::SMEM, s>>>(p);
-  return cudaGetLastError();
+// Launch with or without the programmatic-dependent attribute (overlap with the previous
+// kernel of the stream, which then has to be one that only triggers it).
+template <class... Args>
+cudaError_t launch_ex(void (*kernel)(Args...), dim3 grid, int threads, int smem, bool dependent,
+                      cudaStream_t s, const DecodeParams& p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = dependent ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
-template <int D>
+template <int D, int NT, int K>
+cudaError_t launch_t(const DecodeParams& p, int n_units, bool dependent, cudaStream_t s) {
+  using C = Cfg<D, NT, K>;
+  const KernelInfo<D, NT, K>& info = KernelInfo<D, NT, K>::get();
+  if (info.err != cudaSuccess) return info.err;
+  return launch_ex(partial_kernel<D, NT, K>, dim3(n_units * p.Hkv), C::THREADS, C::SMEM,
+                   dependent, s, p);
+}
+
+template <int D, int K>
 int ctas_per_sm_d(int nt) {
   switch (nt) {
-    case 1: return KernelInfo<D, 1>::get().ctas_per_sm;
-    case 2: return KernelInfo<D, 2>::get().ctas_per_sm;
-    case 3: return KernelInfo<D, 3>::get().ctas_per_sm;
-    default: return KernelInfo<D, 4>::get().ctas_per_sm;
+    case 1: return KernelInfo<D, 1, K>::get().ctas_per_sm;
+    case 2: return KernelInfo<D, 2, K>::get().ctas_per_sm;
+    case 3: return KernelInfo<D, 3, K>::get().ctas_per_sm;
+    default: return KernelInfo<D, 4, K>::get().ctas_per_sm;
   }
 }
 
-template <int D>
-cudaError_t launch_d(const DecodeParams& p, cudaStream_t s) {
+template <int D, int K>
+cudaError_t launch_d(const DecodeParams& p, int n_units, bool dependent, cudaStream_t s) {
   switch ((p.NC + 7) / 8) {
-    case 1: return launch_t<D, 1>(p, s);
-    case 2: return launch_t<D, 2>(p, s);
-    case 3: return launch_t<D, 3>(p, s);
-    case 4: return launch_t<D, 4>(p, s);
+    case 1: return launch_t<D, 1, K>(p, n_units, dependent, s);
+    case 2: return launch_t<D, 2, K>(p, n_units, dependent, s);
+    case 3: return launch_t<D, 3, K>(p, n_units, dependent, s);
+    case 4: return launch_t<D, 4, K>(p, n_units, dependent, s);
     default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int K>
+cudaError_t launch_kind(const DecodeParams& p, int n_units, bool dependent, cudaStream_t s) {
+  if (n_units <= 0) return cudaSuccess;
+  switch (p.D) {
+    case 64: return launch_d<64, K>(p, n_units, dependent, s);
+    case 128: return launch_d<128, K>(p, n_units, dependent, s);
+    case 256: return launch_d<256, K>(p, n_units, dependent, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int K>
+int ctas_per_sm_kind(int D, int NC) {
+  const int nt = (NC + 7) / 8;
+  switch (D) {
+    case 64: return ctas_per_sm_d<64, K>(nt);
+    case 128: return ctas_per_sm_d<128, K>(nt);
+    default: return ctas_per_sm_d<256, K>(nt);
   }
 }
 
 }  // namespace
 
-int partial_ctas_per_sm(int D, int NC) {
-  const int nt = (NC + 7) / 8;
-  switch (D) {
-    case 64: return ctas_per_sm_d<64>(nt);
-    case 128: return ctas_per_sm_d<128>(nt);
-    default: return ctas_per_sm_d<256>(nt);
+int partial_ctas_per_sm(int D, int NC, int mode) {
+  switch (mode) {
+    case kDecodeFused: return ctas_per_sm_kind<kKindFused>(D, NC);
+    case kDecodeBf16: return ctas_per_sm_kind<kKindBf16>(D, NC);
+    default: return ctas_per_sm_kind<kKindTq3>(D, NC);
   }
 }
 
@@ -749,22 +994,24 @@ bool partial_supported(int D, int NC) {
   return (D == 64 || D == 128 || D == 256) && NC >= 1 && NC <= 32;
 }
 
+// The merge follows the last partial grid of the call as its programmatic dependent.
 cudaError_t launch_merge(const DecodeParams& p, cudaStream_t s) {
   if (p.n_seqs <= 0) return cudaSuccess;
-  merge_kernel<<<p.n_seqs * p.Hkv * p.NC, kMergeThreads, 0, s>>>(p);
-  return cudaGetLastError();
+  return launch_ex(merge_kernel, dim3(p.n_seqs * p.Hkv * p.NC), kMergeThreads, 0,
+                   p.n_units > 0, s, p);
 }
 
+// Split: the FP8 grid (units [0, n_fp8)), then the TQ3 grid as its programmatic dependent, so
+// the TQ3 CTAs fill the SM room the FP8 CTAs leave in the same wave.  Fused: one grid over all
+// units.  The first partial grid waits for everything before it.
 cudaError_t launch_partial(const DecodeParams& p, cudaStream_t s) {
   if (p.n_units <= 0) return cudaSuccess;
-  switch (p.D) {
-    case 64: return launch_d<64>(p, s);
-    case 128: return launch_d<128>(p, s);
-    case 256: return launch_d<256>(p, s);
-    default: return cudaErrorInvalidValue;
-  }
+  if (p.page_fmt == kBf16) return launch_kind<kKindBf16>(p, p.n_units, false, s);
+  if (p.fused) return launch_kind<kKindFused>(p, p.n_units, false, s);
+  cudaError_t e = launch_kind<kKindFp8>(p, p.n_fp8, false, s);
+  if (e == cudaSuccess) e = launch_kind<kKindTq3>(p, p.n_units - p.n_fp8, p.n_fp8 > 0, s);
+  return e;
 }
-
 
 // ------------------------------------------------------------------ static decode scratch
 // Partial-state scratch for mkv_decode_attention_noalloc: a file-scope device array, so that

@@ -32,6 +32,26 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ App
   __shared__ float red[8];
   const AppendDesc d = p.desc[blockIdx.x];
   const int h = blockIdx.y, which = blockIdx.z, D = p.D;
+  if (p.bf16) {
+    // BF16 control page: the rows are stored as they are; a fresh page zeroes its other rows
+    uint16_t* rows = reinterpret_cast<uint16_t*>(p.fp8_slab + static_cast<int64_t>(d.slot) * p.slot_bytes +
+                                                 static_cast<int64_t>(h) * (64 * D)) +
+                     which * kPageTokens * D;
+    const uint16_t* src = (which ? p.v : p.k) + (static_cast<int64_t>(d.first_row) * p.Hkv + h) * D;
+    const int64_t src_stride = static_cast<int64_t>(p.Hkv) * D;
+    bool finite = true;
+    for (int i = threadIdx.x; i < d.n_new * D; i += blockDim.x) {
+      const uint16_t b = src[(i / D) * src_stride + (i % D)];
+      finite &= (b & 0x7F80u) != 0x7F80u;
+      rows[d.n_old * D + i] = b;
+    }
+    if (__syncthreads_or(!finite) && threadIdx.x == 0) flag_status(p.status, kStatusCheck);
+    if (d.n_old == 0)
+      for (int i = d.n_new * D + threadIdx.x; i < kPageTokens * D; i += blockDim.x) rows[i] = 0;
+    if (threadIdx.x == 0 && d.n_old == 0 && h == 0 && which == 0)
+      p.tables[d.table_index] = static_cast<int32_t>((2u << kFmtShift) | static_cast<uint32_t>(d.slot));
+    return;
+  }
   uint8_t* head = p.fp8_slab + static_cast<int64_t>(d.slot) * p.slot_bytes +
                   static_cast<int64_t>(h) * (32 * D + 16);
   uint8_t* rows = head + which * kPageTokens * D;
@@ -80,56 +100,82 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ App
   }
 }
 
-// TQ3 record of one (token, KV head, K-or-V, group of 32 channels), one channel per lane:
-// s = fp16(min(fp32(amax/3.5), 65504)); q = #{k in -3..3 : x >= k*s}; the 32 codes packed
-// LSB-first into the 12-byte record, the scale into the area's scale array.
-__device__ __forceinline__ void pack_group(float x, int lane, uint8_t* area, int G, int grp, int t) {
-  float amax = fabsf(x);
-  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  const __half sh = __float2half_rn(fminf(__fdiv_rn(amax, 3.5f), 65504.f));
+// TQ3 record of one (token, KV head, K-or-V, group of 32 channels), computed by one thread from
+// its 32 values x (fp32) and their largest magnitude amax:
+//   s = fp16(min(fp32(amax/3.5), 65504)); q_j = #{k in -3..3 : x_j >= k*s};
+//   code j in bits 3j..3j+2 of the 96-bit record (w0, w1, w2), least significant first.
+// The threshold count is exact and needs no division: for x >= 0 (-0 included) it is
+// 4 + #{k in 1..3 : x >= k*s}, for x < 0 it is 3 - #{k in 1..3 : |x| > k*s}; comparing the
+// fp32 bit patterns of |x| (less one for negative x, which turns > into >=) with those of k*s
+// (exact products) decides both as integer compares.
+__device__ __forceinline__ void tq3_record(const float (&x)[32], float amax, uint32_t& w0,
+                                           uint32_t& w1, uint32_t& w2, __half& sh) {
+  sh = __float2half_rn(fminf(__fdiv_rn(amax, 3.5f), 65504.f));
   const float s = __half2float(sh);
-  uint32_t q = 0;
+  const int t1 = __float_as_int(s), t2 = __float_as_int(2.f * s), t3 = __float_as_int(3.f * s);
+  uint32_t acc[3] = {0u, 0u, 0u};
 #pragma unroll
-  for (int k = -3; k <= 3; ++k) q += (x >= __fmul_rn(static_cast<float>(k), s)) ? 1u : 0u;
-  // bit 3*lane + i of the 96-bit record holds bit i of q
-  const int bit = 3 * lane;
-  uint32_t w0 = 0, w1 = 0, w2 = 0;
-  if (bit < 32) w0 = q << bit;
-  if (bit + 2 >= 32 && bit < 64) w1 = (bit >= 32) ? (q << (bit - 32)) : (q >> (32 - bit));
-  if (bit + 2 >= 64) w2 = (bit >= 64) ? (q << (bit - 64)) : (q >> (64 - bit));
-  w0 = __reduce_or_sync(0xffffffffu, w0);
-  w1 = __reduce_or_sync(0xffffffffu, w1);
-  w2 = __reduce_or_sync(0xffffffffu, w2);
-  uint32_t* rec = reinterpret_cast<uint32_t*>(area + 12 * (grp * kPageTokens + t));
-  if (lane == 0) rec[0] = w0;
-  if (lane == 1) rec[1] = w1;
-  if (lane == 2) rec[2] = w2;
-  if (lane == 3) {
-    __half* sc = reinterpret_cast<__half*>(area + G * kPageTokens * 12);
-    sc[grp * kPageTokens + t] = sh;
+  for (int j = 0; j < 32; ++j) {
+    const uint32_t xb = __float_as_uint(x[j]);
+    const int neg = xb > 0x80000000u ? 1 : 0;
+    const int u = static_cast<int>(xb & 0x7fffffffu) - neg;
+    const int cnt = (u >= t1) + (u >= t2) + (u >= t3);
+    const uint32_t q = static_cast<uint32_t>(neg ? 3 - cnt : 4 + cnt);
+    const int bit = 3 * j;  // constant after unrolling
+    acc[bit >> 5] |= q << (bit & 31);
+    if ((bit & 31) > 29) acc[(bit >> 5) + 1] |= q >> (32 - (bit & 31));
   }
+  w0 = acc[0];
+  w1 = acc[1];
+  w2 = acc[2];
 }
 
-// One block per (page, KV head); one warp per (K-or-V, group of 32 channels, token), lane =
-// channel.  x = fp32(dec(code) * page scale), packed by pack_group.
+// Stores one record and its scale into a TQ3 page-head area ([G][16] records, then [G][16]
+// scales) for (group grp, token t).
+__device__ __forceinline__ void store_record(uint8_t* area, int G, int grp, int t, uint32_t w0,
+                                             uint32_t w1, uint32_t w2, __half sh) {
+  uint32_t* rec = reinterpret_cast<uint32_t*>(area + 12 * (grp * kPageTokens + t));
+  rec[0] = w0;
+  rec[1] = w1;
+  rec[2] = w2;
+  reinterpret_cast<__half*>(area + G * kPageTokens * 12)[grp * kPageTokens + t] = sh;
+}
+
+// One CTA per (page, KV head) with 32 * G threads; thread = (K-or-V, group, token), tokens
+// fastest, so the records and scales a warp writes are contiguous.  The thread reads its 32 FP8
+// codes with two 16-byte loads; x = fp32(dec(code) * page scale), and since that rounding is
+// monotonic, amax = fp32(max |dec| * page scale).
 __global__ void __launch_bounds__(256) demote_kernel(const __grid_constant__ DemoteParams p) {
   const DemoteDesc d = p.desc[blockIdx.x];
   const int h = blockIdx.y, D = p.D, G = D / 32;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = threadIdx.x & 15, grp = (threadIdx.x >> 4) % G, which = threadIdx.x / (16 * G);
   const uint8_t* src = p.fp8_slab + static_cast<int64_t>(d.src_slot) * p.fp8_slot_bytes +
                        static_cast<int64_t>(h) * (32 * D + 16);
   uint8_t* dst = p.tq3_slab + static_cast<int64_t>(d.dst_slot) * p.tq3_slot_bytes +
                  static_cast<int64_t>(h) * (14 * D);
-  const float* scales = reinterpret_cast<const float*>(src + 32 * D);
-  const int units = 2 * G * kPageTokens;
-  for (int u = warp; u < units; u += blockDim.x >> 5) {
-    const int which = u / (G * kPageTokens);
-    const int grp = (u / kPageTokens) % G;
-    const int t = u % kPageTokens;
-    const uint8_t code = src[which * kPageTokens * D + t * D + grp * 32 + lane];
-    const float x = __fmul_rn(e4m3_to_float(code), scales[which]);
-    pack_group(x, lane, dst + which * (G * kPageTokens * 14), G, grp, t);
+  const float scale = reinterpret_cast<const float*>(src + 32 * D)[which];
+  const uint4* c4 = reinterpret_cast<const uint4*>(src + which * kPageTokens * D + t * D + 32 * grp);
+  const uint4 ca = c4[0], cb = c4[1];
+  const uint32_t cw[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+  float x[32];
+  uint32_t mx = 0;  // f16x2 of the largest |dec| (max.f16x2 skips NaN codes, like fmaxf)
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t lo = e4m3x2_to_f16x2(cw[k]), hi = e4m3x2_to_f16x2(cw[k] >> 16);
+    mx = hmax2_u32(mx, hmax2_u32(lo & 0x7fff7fffu, hi & 0x7fff7fffu));
+    const __half2 hl = *reinterpret_cast<const __half2*>(&lo);
+    const __half2 hh = *reinterpret_cast<const __half2*>(&hi);
+    x[4 * k + 0] = __fmul_rn(__low2float(hl), scale);
+    x[4 * k + 1] = __fmul_rn(__high2float(hl), scale);
+    x[4 * k + 2] = __fmul_rn(__low2float(hh), scale);
+    x[4 * k + 3] = __fmul_rn(__high2float(hh), scale);
   }
+  const __half2 m2 = *reinterpret_cast<const __half2*>(&mx);
+  const float amax = __fmul_rn(fmaxf(__low2float(m2), __high2float(m2)), scale);
+  uint32_t w0, w1, w2;
+  __half sh;
+  tq3_record(x, amax, w0, w1, w2, sh);
+  store_record(dst + which * (G * kPageTokens * 14), G, grp, t, w0, w1, w2, sh);
   if (p.publish && h == 0 && threadIdx.x == 0)
     p.tables[d.table_index] = static_cast<int32_t>((1u << kFmtShift) | static_cast<uint32_t>(d.dst_slot));
 }
@@ -140,23 +186,41 @@ __global__ void __launch_bounds__(256) retag_kernel(const __grid_constant__ Reta
 }
 
 // Prefill: a full page packed to TQ3 straight from the bf16 input rows (the values are exact in
-// fp32), with the same per-group packing as demotion.  One block per (page, KV head).
+// fp32), with the same per-record packing as demotion.  One CTA per (page, KV head) with 32 * G
+// threads, thread = (K-or-V, group, token); four 16-byte loads bring a record's 32 values.
 __global__ void __launch_bounds__(256) pack_kernel(const __grid_constant__ PackParams p) {
   const PackDesc d = p.desc[blockIdx.x];
   const int h = blockIdx.y, D = p.D, G = D / 32;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = threadIdx.x & 15, grp = (threadIdx.x >> 4) % G, which = threadIdx.x / (16 * G);
   uint8_t* dst = p.tq3_slab + static_cast<int64_t>(d.dst_slot) * p.tq3_slot_bytes +
                  static_cast<int64_t>(h) * (14 * D);
-  const int units = 2 * G * kPageTokens;
-  for (int u = warp; u < units; u += blockDim.x >> 5) {
-    const int which = u / (G * kPageTokens);
-    const int grp = (u / kPageTokens) % G;
-    const int t = u % kPageTokens;
-    const uint16_t* src = which ? p.v : p.k;
-    const float x = bf16_bits_to_float(
-        src[(static_cast<int64_t>(d.first_row + t) * p.Hkv + h) * D + grp * 32 + lane]);
-    pack_group(x, lane, dst + which * (G * kPageTokens * 14), G, grp, t);
+  const uint16_t* src = (which ? p.v : p.k) +
+                        (static_cast<int64_t>(d.first_row + t) * p.Hkv + h) * D + 32 * grp;
+  float x[32];
+  float amax = 0.f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    uint32_t w[4];
+    if (p.vec16) {  // both input arrays 16-byte aligned (checked on the host)
+      const uint4 v = reinterpret_cast<const uint4*>(src)[k];
+      w[0] = v.x, w[1] = v.y, w[2] = v.z, w[3] = v.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        w[e] = static_cast<uint32_t>(src[8 * k + 2 * e]) |
+               (static_cast<uint32_t>(src[8 * k + 2 * e + 1]) << 16);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      x[8 * k + 2 * e] = __uint_as_float(w[e] << 16);
+      x[8 * k + 2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+      amax = fmaxf(amax, fmaxf(fabsf(x[8 * k + 2 * e]), fabsf(x[8 * k + 2 * e + 1])));
+    }
   }
+  uint32_t w0, w1, w2;
+  __half sh;
+  tq3_record(x, amax, w0, w1, w2, sh);
+  store_record(dst + which * (G * kPageTokens * 14), G, grp, t, w0, w1, w2, sh);
   if (h == 0 && threadIdx.x == 0)
     p.tables[d.table_index] = static_cast<int32_t>((1u << kFmtShift) | static_cast<uint32_t>(d.dst_slot));
 }
@@ -185,13 +249,18 @@ __global__ void __launch_bounds__(256) materialise_kernel(const __grid_constant_
   const int32_t e = p.table[page];
   const int fmt = static_cast<int>(static_cast<uint32_t>(e) >> kFmtShift);
   const int64_t slot = static_cast<int64_t>(static_cast<uint32_t>(e) & kSlotMask);
-  if (e < 0 || fmt > 1 || slot >= (fmt == 0 ? p.fp8_slots : p.tq3_slots)) {
+  if (e == -1 || (fmt != 1 && fmt != p.page_fmt) || slot >= (fmt == 1 ? p.tq3_slots : p.fp8_slots)) {
     if (threadIdx.x == 0) flag_status(p.status, kStatusCheck);
     return;
   }
   float* out = (kv ? p.v_out : p.k_out) + (static_cast<int64_t>(kPageTokens) * page * p.Hkv + h) * D;
   const int64_t row_stride = static_cast<int64_t>(p.Hkv) * D;
-  if (fmt == 0) {
+  if (fmt == 2) {
+    const uint16_t* rows = reinterpret_cast<const uint16_t*>(p.fp8_slab + slot * p.fp8_slot_bytes +
+                                                             h * (64LL * D)) + kv * kPageTokens * D;
+    for (int i = threadIdx.x; i < n * D; i += blockDim.x)
+      out[(i / D) * row_stride + i % D] = bf16_bits_to_float(rows[i]);
+  } else if (fmt == 0) {
     const uint8_t* base = p.fp8_slab + slot * p.fp8_slot_bytes + h * (32LL * D + 16);
     const uint8_t* codes = base + kv * kPageTokens * D;
     const float scale = reinterpret_cast<const float*>(base + 2 * kPageTokens * D)[kv];
@@ -233,7 +302,7 @@ cudaError_t launch_wait_selftest(int32_t* status, uint64_t limit_ns, cudaStream_
 
 cudaError_t launch_pack(const PackParams& p, cudaStream_t s) {
   if (p.n_desc <= 0) return cudaSuccess;
-  pack_kernel<<<dim3(p.n_desc, p.Hkv), 256, 0, s>>>(p);
+  pack_kernel<<<dim3(p.n_desc, p.Hkv), p.D, 0, s>>>(p);  // 32 * (D / 32) threads
   return cudaGetLastError();
 }
 
@@ -252,7 +321,7 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
 
 cudaError_t launch_demote(const DemoteParams& p, cudaStream_t s) {
   if (p.n_desc <= 0) return cudaSuccess;
-  demote_kernel<<<dim3(p.n_desc, p.Hkv), 256, 0, s>>>(p);
+  demote_kernel<<<dim3(p.n_desc, p.Hkv), p.D, 0, s>>>(p);  // 32 * (D / 32) threads
   return cudaGetLastError();
 }
 

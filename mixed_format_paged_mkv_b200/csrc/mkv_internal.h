@@ -21,6 +21,7 @@ constexpr int32_t kStatusTimeout = 2;  // a bounded wait ran out
 // Bytes of one KV head inside a slot.
 inline int64_t fp8_head_bytes(int D) { return 32LL * D + 16; }
 inline int64_t tq3_head_bytes(int D) { return 14LL * D; }
+inline int64_t bf16_head_bytes(int D) { return 64LL * D; }
 
 // ------------------------------------------------------------------ append (FP8 page write)
 struct AppendDesc {
@@ -39,6 +40,7 @@ struct AppendParams {
   const uint16_t* v;
   int64_t slot_bytes;
   int32_t Hkv, D;
+  int32_t bf16;       // 1: a control pool's BF16 pages (values stored as they are)
   int32_t n_desc;
   AppendDesc desc[kAppendMaxDesc];
 };
@@ -86,6 +88,7 @@ struct PackParams {
   int32_t* tables;
   int64_t tq3_slot_bytes;
   int32_t Hkv, D;
+  int32_t vec16;  // 1: k and v are 16-byte aligned (vector loads), 0: element loads
   int32_t n_desc;
   PackDesc desc[kPackMaxDesc];
 };
@@ -115,6 +118,7 @@ struct MaterialiseParams {
   float* v_out;
   int64_t fp8_slot_bytes, tq3_slot_bytes;
   int32_t Hkv, D, ctx, fp8_slots, tq3_slots;
+  int32_t page_fmt;  // format of the first slab's pages: 0 FP8, 2 BF16 (control pool)
 };
 
 // ------------------------------------------------------------------ decode
@@ -155,10 +159,19 @@ struct DecodeParams {
   int32_t max_pages, fp8_slots, tq3_slots;
   float logit_scale;  // sm_scale * log2(e)
   int32_t n_seqs;     // sequences in this launch
-  int32_t n_units;    // units in this launch (grid = n_units * Hkv CTAs)
+  int32_t n_units;    // units in this launch: FP8 units [0, n_fp8), then TQ3 units
+  int32_t n_fp8;      // (the fused kernel takes every unit in one grid of n_units * Hkv CTAs)
+  int32_t fused;      // 1: one grid branching per unit; 0: an FP8 grid, then a TQ3 grid
+  int32_t page_fmt;   // format of written pages: 0 FP8 (mixed pools), 2 BF16 (control pools)
   SeqDesc seq[kDecodeMaxSeqs];
   UnitDesc unit[kDecodeMaxUnits];
 };
+
+// Every parameter block fits the 32,764-byte kernel-parameter limit.
+static_assert(sizeof(AppendParams) <= 32764 && sizeof(DemoteParams) <= 32764 &&
+                  sizeof(RetagParams) <= 32764 && sizeof(PackParams) <= 32764 &&
+                  sizeof(CopyParams) <= 32764 && sizeof(DecodeParams) <= 32764,
+              "kernel parameter block too large");
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 cudaError_t launch_demote(const DemoteParams& p, cudaStream_t s);
@@ -169,8 +182,10 @@ cudaError_t launch_pack(const PackParams& p, cudaStream_t s);
 cudaError_t launch_partial(const DecodeParams& p, cudaStream_t s);
 cudaError_t launch_merge(const DecodeParams& p, cudaStream_t s);
 bool partial_supported(int D, int NC);
-// CTAs of the partial kernel for (D, NC) that one SM keeps resident (queried once).
-int partial_ctas_per_sm(int D, int NC);
+// CTAs of the partial kernel for (D, NC) that one SM keeps resident (queried once): the TQ3
+// kernel's (per-format grids), the fused kernel's or the BF16 control kernel's.
+constexpr int kDecodeSplit = 0, kDecodeFused = 1, kDecodeBf16 = 2;
+int partial_ctas_per_sm(int D, int NC, int mode);
 cudaError_t static_decode_scratch(void** ptr, size_t* bytes);
 
 }  // namespace mkv

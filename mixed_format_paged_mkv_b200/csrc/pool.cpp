@@ -87,7 +87,7 @@ struct Allocator {
 
 struct Seq {
   std::vector<int32_t> table;     // block-table entries
-  std::vector<int32_t> fp8_pages; // logical pages currently FP8, ascending
+  std::vector<int32_t> fp8_pages; // logical pages currently FP8 (BF16 in a control pool), ascending
   std::vector<uint8_t> prot;      // protected flag per logical page
   int32_t ctx = 0;
   int32_t n3 = 0;
@@ -97,6 +97,9 @@ inline int32_t entry_of(int fmt, int32_t slot) {
   return static_cast<int32_t>((static_cast<uint32_t>(fmt) << kFmtShift) | static_cast<uint32_t>(slot));
 }
 inline int fmt_of(int32_t e) { return static_cast<int>(static_cast<uint32_t>(e) >> kFmtShift); }
+// Slab (and allocator) of a format: TQ3 pages have their own; FP8 pages, or the BF16 pages of a
+// control pool, use the first.
+inline int slab_of(int fmt) { return fmt == MKV_FMT_TQ3 ? 1 : 0; }
 inline int32_t slot_of(int32_t e) { return static_cast<int32_t>(static_cast<uint32_t>(e) & kSlotMask); }
 
 struct TimingRec {
@@ -118,6 +121,8 @@ struct mkv_pool {
   Allocator alloc[2];
   int64_t launches = 0;
   int64_t fail_after = -1;  // test hook: device operations that still succeed before one fails
+  bool fused_decode = false;  // decode kernels: per-format grids (default) or one fused grid
+  int page_fmt = MKV_FMT_FP8;  // format of written pages: FP8, or BF16 in a control pool
   bool timing = false;
   std::vector<TimingRec> timing_recs;
   std::vector<cudaEvent_t> spare_events;
@@ -126,6 +131,14 @@ struct mkv_pool {
 namespace {
 
 bool valid_pool(mkv_pool_t p) { return p != nullptr; }
+
+int decode_mode(const mkv_pool* p) {
+  return p->page_fmt == MKV_FMT_BF16 ? kDecodeBf16 : (p->fused_decode ? kDecodeFused : kDecodeSplit);
+}
+
+int64_t page_head_bytes(const mkv_pool_config& c) {
+  return (c.flags & MKV_POOL_BF16_CONTROL) ? bf16_head_bytes(c.head_dim) : fp8_head_bytes(c.head_dim);
+}
 
 int check_seq(mkv_pool_t p, int32_t s) {
   if (s < 0 || s >= p->cfg.max_seqs)
@@ -160,7 +173,8 @@ int validate_config(const mkv_pool_config* c) {
       c->tq3_slots > static_cast<int32_t>(kSlotMask))
     return fail(MKV_ERR_INVALID_ARG, "slot counts out of range");
   if (c->sink_pages < 0) return fail(MKV_ERR_INVALID_ARG, "sink_pages must be >= 0");
-  if (c->flags & ~MKV_POOL_HOST_ONLY) return fail(MKV_ERR_INVALID_ARG, "unknown flags");
+  if (c->flags & ~(MKV_POOL_HOST_ONLY | MKV_POOL_BF16_CONTROL))
+    return fail(MKV_ERR_INVALID_ARG, "unknown flags");
   if (static_cast<int64_t>(c->max_seqs) * c->max_pages_per_seq > (1LL << 31) - 1)
     return fail(MKV_ERR_INVALID_ARG, "table too large");
   if (c->max_pages_per_seq > INT32_MAX / kPageTokens)
@@ -216,7 +230,7 @@ int64_t cut_units(const mkv_pool* p, const int32_t* seq_ids, int32_t n, int32_t 
     total += static_cast<int64_t>(s.fp8_pages.size()) * b8 + static_cast<int64_t>(s.n3) * b3;
   }
   const int64_t slots =
-      static_cast<int64_t>(p->sm_count) * partial_ctas_per_sm(p->cfg.head_dim, NC);
+      static_cast<int64_t>(p->sm_count) * partial_ctas_per_sm(p->cfg.head_dim, NC, decode_mode(p));
   const int64_t U = std::max<int64_t>(1, slots / Hkv);
   // units of a group at unit cost c: as many as its cost needs, clamped to the page limits
   auto units_at = [](double c, int64_t cost, int64_t pages, int min_pages) -> int64_t {
@@ -254,7 +268,9 @@ int64_t cut_units(const mkv_pool* p, const int32_t* seq_ids, int32_t n, int32_t 
       for (int64_t k = 0; k < u; ++k) {
         const int64_t j0 = k * n8 / u, j1 = (k + 1) * n8 / u;
         if (j1 <= j0) continue;
-        if (!emit(UnitDesc{f8[j0], f8[j1 - 1] + 1, 0, 0, np++}, (j1 - j0) * b8, i)) return -1;
+        if (!emit(UnitDesc{f8[j0], f8[j1 - 1] + 1, 0, static_cast<int16_t>(p->page_fmt), np++},
+                  (j1 - j0) * b8, i))
+          return -1;
         ++nu;
       }
     }
@@ -359,6 +375,20 @@ int device_op(mkv_pool_t p, const char* what, F&& f) {
   return e == cudaSuccess ? MKV_OK : cuda_fail(e, what);
 }
 
+// Launch order of a group's units: largest cost first; with per-format grids the FP8 units
+// (first grid) before the TQ3 units (second grid).  Returns the FP8 unit count.
+template <class Fmt, class Cost>
+int32_t order_units(int32_t* order, int32_t n, bool fused, Fmt&& fmt, Cost&& cost) {
+  for (int32_t k = 0; k < n; ++k) order[k] = k;
+  std::sort(order, order + n, [&](int32_t x, int32_t y) {
+    if (!fused && fmt(x) != fmt(y)) return fmt(x) < fmt(y);  // FP8 (0) first
+    return cost(x) != cost(y) ? cost(x) > cost(y) : x < y;
+  });
+  int32_t n8 = 0;
+  for (int32_t k = 0; k < n; ++k) n8 += fmt(k) == 0 ? 1 : 0;
+  return fused ? 0 : n8;
+}
+
 cudaEvent_t get_event(mkv_pool_t p) {
   if (!p->spare_events.empty()) {
     cudaEvent_t e = p->spare_events.back();
@@ -381,7 +411,7 @@ int mkv_pool_required_bytes(const mkv_pool_config* cfg, size_t* fp8_slab, size_t
                             size_t* tables, size_t* status) {
   if (int e = validate_config(cfg)) return e;
   const size_t Hkv = cfg->num_kv_heads, D = cfg->head_dim;
-  if (fp8_slab) *fp8_slab = static_cast<size_t>(cfg->fp8_slots) * Hkv * fp8_head_bytes(D);
+  if (fp8_slab) *fp8_slab = static_cast<size_t>(cfg->fp8_slots) * Hkv * page_head_bytes(*cfg);
   if (tq3_slab) *tq3_slab = static_cast<size_t>(cfg->tq3_slots) * Hkv * tq3_head_bytes(D);
   if (tables) *tables = static_cast<size_t>(cfg->max_seqs) * cfg->max_pages_per_seq * 4;
   if (status) *status = status_bytes(*cfg);
@@ -410,7 +440,8 @@ int mkv_pool_create(const mkv_pool_config* cfg, void* fp8_slab, void* tq3_slab,
   p->tq3_slab = static_cast<uint8_t*>(tq3_slab);
   p->d_tables = d_tables;
   p->d_status = d_status;
-  p->fp8_slot_bytes = static_cast<int64_t>(cfg->num_kv_heads) * fp8_head_bytes(cfg->head_dim);
+  p->fp8_slot_bytes = static_cast<int64_t>(cfg->num_kv_heads) * page_head_bytes(*cfg);
+  p->page_fmt = (cfg->flags & MKV_POOL_BF16_CONTROL) ? MKV_FMT_BF16 : MKV_FMT_FP8;
   p->tq3_slot_bytes = static_cast<int64_t>(cfg->num_kv_heads) * tq3_head_bytes(cfg->head_dim);
   p->seqs.resize(cfg->max_seqs);
   p->alloc[0].init(cfg->fp8_slots);
@@ -442,8 +473,9 @@ void mkv_pool_destroy(mkv_pool_t p) {
 
 int mkv_pool_set_slot_order(mkv_pool_t p, int32_t fmt, const int32_t* order, int32_t n) {
   if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
-  if (fmt != MKV_FMT_FP8 && fmt != MKV_FMT_TQ3) return fail(MKV_ERR_INVALID_ARG, "bad format");
-  Allocator& a = p->alloc[fmt];
+  if (fmt != MKV_FMT_FP8 && fmt != MKV_FMT_TQ3 && fmt != MKV_FMT_BF16)
+    return fail(MKV_ERR_INVALID_ARG, "bad format");
+  Allocator& a = p->alloc[slab_of(fmt)];
   if (n != a.n || (n > 0 && !order)) return fail(MKV_ERR_INVALID_ARG, "order must list all %d slots", a.n);
   std::vector<uint8_t> seen(n, 0);
   for (int32_t i = 0; i < n; ++i) {
@@ -517,6 +549,7 @@ int mkv_append_kv(mkv_pool_t p, const int32_t* seq_ids, const int32_t* n_new, in
     prm->slot_bytes = p->fp8_slot_bytes;
     prm->Hkv = p->cfg.num_kv_heads;
     prm->D = p->cfg.head_dim;
+    prm->bf16 = p->page_fmt == MKV_FMT_BF16 ? 1 : 0;
     for (size_t b = 0; b < descs.size() && rc == MKV_OK; b += kAppendMaxDesc) {
       const size_t m = std::min<size_t>(kAppendMaxDesc, descs.size() - b);
       prm->n_desc = static_cast<int32_t>(m);
@@ -536,7 +569,7 @@ int mkv_append_kv(mkv_pool_t p, const int32_t* seq_ids, const int32_t* n_new, in
     if (s.prot.size() < static_cast<size_t>(pages_after)) s.prot.resize(pages_after, 0);
     for (size_t k = first_new[i]; static_cast<int32_t>(s.table.size()) < pages_after; ++k) {
       s.fp8_pages.push_back(static_cast<int32_t>(s.table.size()));
-      s.table.push_back(entry_of(MKV_FMT_FP8, taken[k]));
+      s.table.push_back(entry_of(p->page_fmt, taken[k]));
     }
     s.ctx += n_new[i];
   }
@@ -562,7 +595,7 @@ int mkv_demote_pages(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, int32
   if (window < 0) return fail(MKV_ERR_INVALID_ARG, "window must be >= 0");
   struct Work { int32_t seq, page; };
   std::vector<Work> work;
-  for (int32_t i = 0; i < n_seqs; ++i) {
+  for (int32_t i = 0; i < n_seqs && p->page_fmt == MKV_FMT_FP8; ++i) {  // control: never
     const Seq& s = p->seqs[seq_ids[i]];
     const int64_t L = s.ctx;
     for (int32_t pg : s.fp8_pages) {
@@ -633,7 +666,7 @@ int mkv_demote_pages(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, int32
   for (int32_t i = 0; i < n_seqs; ++i) {
     Seq& s = p->seqs[seq_ids[i]];
     s.fp8_pages.erase(std::remove_if(s.fp8_pages.begin(), s.fp8_pages.end(),
-                                     [&](int32_t pg) { return fmt_of(s.table[pg]) != MKV_FMT_FP8; }),
+                                     [&](int32_t pg) { return fmt_of(s.table[pg]) != p->page_fmt; }),
                       s.fp8_pages.end());
   }
   for (const DemoteDesc& d : descs) p->alloc[0].give(d.src_slot);
@@ -661,7 +694,7 @@ int mkv_decode_plan(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, int32_
   const int64_t nu = static_cast<int64_t>(plan.unit.size());
   *n_units = static_cast<int32_t>(nu);
   if (ctas_per_wave)
-    *ctas_per_wave = p->sm_count * partial_ctas_per_sm(p->cfg.head_dim, plan.NC);
+    *ctas_per_wave = p->sm_count * partial_ctas_per_sm(p->cfg.head_dim, plan.NC, decode_mode(p));
   if (!units_out) return ok();  // count query
   if (nu > cap) return fail(MKV_ERR_INVALID_ARG, "%lld units do not fit in %d", (long long)nu, cap);
   const int64_t b[2] = {kFp8PageCost, kTq3PageCost};
@@ -723,7 +756,7 @@ int mkv_decode_attention(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, i
   // launches over groups of whole sequences, each within the parameter-block limits
   size_t u0 = 0;
   int32_t s0 = 0;
-  std::vector<size_t> order;
+  std::vector<int32_t> order;
   while (s0 < n_seqs && err == cudaSuccess) {
     int32_t s1 = s0;
     size_t u1 = u0;
@@ -741,15 +774,18 @@ int mkv_decode_attention(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, i
     if (err != cudaSuccess) break;
     for (int32_t i = s0; i < s1; ++i) prm->seq[i - s0] = plan.seq[i];
     order.resize(u1 - u0);
-    for (size_t k = 0; k < order.size(); ++k) order[k] = u0 + k;
-    std::stable_sort(order.begin(), order.end(),
-                     [&](size_t x, size_t y) { return plan.cost[x] > plan.cost[y]; });
+    prm->n_fp8 = order_units(
+        order.data(), static_cast<int32_t>(order.size()), p->fused_decode,
+        [&](int32_t k) { return static_cast<int>(plan.unit[u0 + k].fmt); },
+        [&](int32_t k) { return plan.cost[u0 + k]; });
     for (size_t k = 0; k < order.size(); ++k) {
-      prm->unit[k] = plan.unit[order[k]];
-      prm->unit[k].seq = static_cast<int16_t>(plan.pos[order[k]] - s0);
+      prm->unit[k] = plan.unit[u0 + order[k]];
+      prm->unit[k].seq = static_cast<int16_t>(plan.pos[u0 + order[k]] - s0);
     }
     prm->n_seqs = s1 - s0;
     prm->n_units = static_cast<int32_t>(order.size());
+    prm->fused = p->fused_decode ? 1 : 0;
+    prm->page_fmt = p->page_fmt;
     const bool last = s1 >= n_seqs;
     err = launch_partial(*prm, st);
     ++p->launches;
@@ -840,10 +876,11 @@ int mkv_decode_attention_noalloc(mkv_pool_t p, const int32_t* seq_ids, int32_t n
   if (bytes > cap)
     return fail(MKV_ERR_WORKSPACE_TOO_SMALL,
                 "call needs %zu bytes of partial-state scratch; the static scratch holds %zu", bytes, cap);
-  for (int32_t k = 0; k < nu; ++k) t.order[k] = k;
-  std::sort(t.order, t.order + nu, [&](int32_t x, int32_t y) {
-    return t.cost[x] != t.cost[y] ? t.cost[x] > t.cost[y] : x < y;
-  });
+  prm.n_fp8 = order_units(t.order, nu, p->fused_decode,
+                          [&](int32_t k) { return static_cast<int>(t.unit[k].fmt); },
+                          [&](int32_t k) { return t.cost[k]; });
+  prm.fused = p->fused_decode ? 1 : 0;
+  prm.page_fmt = p->page_fmt;
   for (int32_t k = 0; k < nu; ++k) prm.unit[k] = t.unit[t.order[k]];
   uint8_t* ws = static_cast<uint8_t*>(scratch);
   prm.fp8_slab = p->fp8_slab;
@@ -888,7 +925,7 @@ int mkv_seq_reset(mkv_pool_t p, int32_t seq, void* stream) {
     });
     if (rc != MKV_OK) return rc;
   }
-  for (int32_t e : s.table) p->alloc[fmt_of(e)].give(slot_of(e));
+  for (int32_t e : s.table) p->alloc[slab_of(fmt_of(e))].give(slot_of(e));
   s = Seq();
   return ok();
 }
@@ -931,8 +968,9 @@ int mkv_prefill_kv(mkv_pool_t p, const int32_t* seq_ids, const int32_t* n_tokens
   const int32_t MP = p->cfg.max_pages_per_seq, sink = p->cfg.sink_pages;
   // page p of a prefill of n tokens is packed to TQ3 at once iff the anchor policy would demote
   // it: p >= sink and 16p + 16 <= n - W (new pages carry no protection)
-  auto direct = [&](int64_t pg, int64_t n) {
-    return pg >= sink && kPageTokens * pg + kPageTokens <= n - anchor_window_tokens;
+  auto direct = [&](int64_t pg, int64_t n) {  // (a control pool writes every page as BF16)
+    return p->page_fmt == MKV_FMT_FP8 && pg >= sink &&
+           kPageTokens * pg + kPageTokens <= n - anchor_window_tokens;
   };
   int64_t need[2] = {0, 0}, rows = 0;
   for (int32_t i = 0; i < n_seqs; ++i) {
@@ -992,6 +1030,7 @@ int mkv_prefill_kv(mkv_pool_t p, const int32_t* seq_ids, const int32_t* n_tokens
     ap->slot_bytes = p->fp8_slot_bytes;
     ap->Hkv = p->cfg.num_kv_heads;
     ap->D = p->cfg.head_dim;
+    ap->bf16 = p->page_fmt == MKV_FMT_BF16 ? 1 : 0;
     for (size_t b = 0; b < fp8_descs.size() && rc == MKV_OK; b += kAppendMaxDesc) {
       const size_t m = std::min<size_t>(kAppendMaxDesc, fp8_descs.size() - b);
       ap->n_desc = static_cast<int32_t>(m);
@@ -1009,6 +1048,7 @@ int mkv_prefill_kv(mkv_pool_t p, const int32_t* seq_ids, const int32_t* n_tokens
     pp->tq3_slot_bytes = p->tq3_slot_bytes;
     pp->Hkv = p->cfg.num_kv_heads;
     pp->D = p->cfg.head_dim;
+    pp->vec16 = ((reinterpret_cast<uintptr_t>(k_bf16) | reinterpret_cast<uintptr_t>(v_bf16)) & 15) ? 0 : 1;
     for (size_t b = 0; b < tq3_descs.size() && rc == MKV_OK; b += kPackMaxDesc) {
       const size_t m = std::min<size_t>(kPackMaxDesc, tq3_descs.size() - b);
       pp->n_desc = static_cast<int32_t>(m);
@@ -1030,7 +1070,7 @@ int mkv_prefill_kv(mkv_pool_t p, const int32_t* seq_ids, const int32_t* n_tokens
     s.prot.assign(pages, 0);
     for (int32_t pg = 0; pg < pages; ++pg) {
       const int f = direct(pg, n) ? 1 : 0;
-      s.table.push_back(entry_of(f, taken[f][next[f]++]));
+      s.table.push_back(entry_of(f == 1 ? MKV_FMT_TQ3 : p->page_fmt, taken[f][next[f]++]));
       if (f == 1) ++s.n3;
       else s.fp8_pages.push_back(pg);
     }
@@ -1064,6 +1104,7 @@ int mkv_materialise_kv(mkv_pool_t p, int32_t seq, float* k_out, float* v_out,
   prm.ctx = s.ctx;
   prm.fp8_slots = p->cfg.fp8_slots;
   prm.tq3_slots = p->cfg.tq3_slots;
+  prm.page_fmt = p->page_fmt;
   cudaError_t e = launch_materialise(prm, as_stream(stream));
   ++p->launches;
   if (e != cudaSuccess) return cuda_fail(e, "materialise launch");
@@ -1078,7 +1119,7 @@ int mkv_seq_copy(mkv_pool_t p, int32_t src, int32_t dst, void* stream) {
     return fail(MKV_ERR_INVALID_ARG, "destination must be a different, empty sequence");
   const Seq& s = p->seqs[src];
   int64_t need[2] = {0, 0};
-  for (int32_t e : s.table) need[fmt_of(e)]++;
+  for (int32_t e : s.table) need[slab_of(fmt_of(e))]++;
   for (int f = 0; f < 2; ++f)
     if (need[f] > p->alloc[f].n_free) return fail(MKV_ERR_OUT_OF_PAGES, "slab %d exhausted", f);
   // ---- stage: a slot of the same format per page, pages ascending
@@ -1090,7 +1131,7 @@ int mkv_seq_copy(mkv_pool_t p, int32_t src, int32_t dst, void* stream) {
   std::vector<CopyDesc> descs;
   for (size_t pg = 0; pg < s.table.size(); ++pg) {
     const int f = fmt_of(s.table[pg]);
-    const int32_t ns = p->alloc[f].take();
+    const int32_t ns = p->alloc[slab_of(f)].take();
     d.table.push_back(entry_of(f, ns));
     descs.push_back({slot_of(s.table[pg]), ns, f, dst * p->cfg.max_pages_per_seq + static_cast<int32_t>(pg)});
   }
@@ -1112,7 +1153,8 @@ int mkv_seq_copy(mkv_pool_t p, int32_t src, int32_t dst, void* stream) {
     delete prm;
   }
   if (rc != MKV_OK) {
-    for (auto it = descs.rbegin(); it != descs.rend(); ++it) p->alloc[it->fmt].give(it->dst_slot);
+    for (auto it = descs.rbegin(); it != descs.rend(); ++it)
+      p->alloc[slab_of(it->fmt)].give(it->dst_slot);
     return rc;
   }
   p->seqs[dst] = std::move(d);
@@ -1134,7 +1176,7 @@ int mkv_get_block_table(mkv_pool_t p, int32_t seq, int32_t* host_out, int32_t ca
 
 int mkv_slot_bytes(mkv_pool_t p, int32_t fmt, size_t* bytes) {
   if (!valid_pool(p) || !bytes) return fail(MKV_ERR_INVALID_ARG, "NULL argument");
-  if (fmt == MKV_FMT_FP8) *bytes = p->fp8_slot_bytes;
+  if (fmt == p->page_fmt) *bytes = p->fp8_slot_bytes;
   else if (fmt == MKV_FMT_TQ3) *bytes = p->tq3_slot_bytes;
   else return fail(MKV_ERR_INVALID_ARG, "bad format");
   return ok();
@@ -1143,14 +1185,14 @@ int mkv_slot_bytes(mkv_pool_t p, int32_t fmt, size_t* bytes) {
 int mkv_read_slot(mkv_pool_t p, int32_t entry, void* host_out, size_t cap, void* stream) {
   if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
   if (p->host_only) return fail(MKV_ERR_INVALID_ARG, "host-only pool has no slabs");
-  if (entry < 0) return fail(MKV_ERR_INVALID_ARG, "unmapped entry");
+  if (entry == MKV_ENTRY_UNMAPPED) return fail(MKV_ERR_INVALID_ARG, "unmapped entry");
   const int f = fmt_of(entry);
   const int32_t slot = slot_of(entry);
-  if (f > 1 || slot >= (f == 0 ? p->cfg.fp8_slots : p->cfg.tq3_slots))
+  if ((f != MKV_FMT_TQ3 && f != p->page_fmt) || slot >= (f == MKV_FMT_TQ3 ? p->cfg.tq3_slots : p->cfg.fp8_slots))
     return fail(MKV_ERR_INVALID_ARG, "entry 0x%x names no slot", entry);
-  const int64_t b = f == 0 ? p->fp8_slot_bytes : p->tq3_slot_bytes;
+  const int64_t b = f == MKV_FMT_TQ3 ? p->tq3_slot_bytes : p->fp8_slot_bytes;
   if (!host_out || cap < static_cast<size_t>(b)) return fail(MKV_ERR_INVALID_ARG, "output buffer too small");
-  const uint8_t* src = (f == 0 ? p->fp8_slab : p->tq3_slab) + slot * b;
+  const uint8_t* src = (f == MKV_FMT_TQ3 ? p->tq3_slab : p->fp8_slab) + slot * b;
   cudaStream_t st = as_stream(stream);
   cudaError_t e = cudaMemcpyAsync(host_out, src, b, cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
@@ -1213,6 +1255,14 @@ int mkv_timing_read(mkv_pool_t p, double* ms_partial, double* ms_merge, int64_t*
   if (ms_partial) *ms_partial = a;
   if (ms_merge) *ms_merge = b;
   if (calls) *calls = n;
+  return ok();
+}
+
+int mkv_set_decode_kernels(mkv_pool_t p, int32_t mode) {
+  if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
+  if (mode != MKV_DECODE_SPLIT && mode != MKV_DECODE_FUSED)
+    return fail(MKV_ERR_INVALID_ARG, "unknown decode kernel mode %d", mode);
+  p->fused_decode = mode == MKV_DECODE_FUSED;
   return ok();
 }
 

@@ -12,6 +12,9 @@ Recipe (all values bf16 from fp32 N(0,1) draws rounded to nearest even):
   K        N(0,1); with ``outliers`` 4 distinct channels per (layer, KV head) are scaled x8
            before rounding (the same channels for every token and sequence).
   V, Q     N(0,1).
+  scales   optional value-range variants multiply the fp32 draws before rounding: K by
+           ``k_scale``, V by ``v_scale``, and with ``scale_mix`` every (token, KV head,
+           32-channel group) of K and of V by a level drawn from ``MIX_LEVELS`` (stream 8).
   cache    per sequence, in order: append all L tokens as FP8 in one call, mark protected
            pages, demote with the anchor window W; then decode the last q_len tokens.
 
@@ -34,7 +37,9 @@ from dataclasses import dataclass
 import numpy as np
 
 PAGE = 16
-S_Q, S_K, S_V, S_SLOT, S_OUTLIER, S_PROTECT, S_CTX, S_STEP = range(8)
+S_Q, S_K, S_V, S_SLOT, S_OUTLIER, S_PROTECT, S_CTX, S_STEP, S_MIX = range(9)
+# multipliers of the mixed-scale variant: from far below to far above N(0,1)
+MIX_LEVELS = np.array([1e-4, 1e-2, 1.0, 1e3, 3e4], dtype=np.float32)
 
 
 def bf16_bits(x) -> np.ndarray:
@@ -62,6 +67,9 @@ class Workload:
     layers: int = 1
     slot_order: bool = True          # random slot order (permuted block tables)
     pool_slots: int = 0              # fixed slots per format (0 -> sized from the workload)
+    k_scale: float = 1.0             # multiplier of every K draw (value-range variants)
+    v_scale: float = 1.0             # multiplier of every V draw
+    scale_mix: bool = False          # per-(token, KV head, group) levels from MIX_LEVELS
 
     # ------------------------------------------------------------------ derived
     @property
@@ -110,6 +118,7 @@ class Workload:
                 oc = self.outlier_channels(layer)
                 for h in range(self.Hkv):
                     k[:, h, oc[h]] *= np.float32(8.0)
+            k, v = self._rescale(k, v, self.rng(S_MIX, layer, seq, b0 // blk))
             a, b = max(lo, b0) - b0, min(hi, b0 + n) - b0
             ks.append(bf16_bits(k[a:b]))
             vs.append(bf16_bits(v[a:b]))
@@ -132,7 +141,25 @@ class Workload:
             oc = self.outlier_channels(layer)
             for h in range(self.Hkv):
                 k[:, h, oc[h]] *= np.float32(8.0)
+        k, v = self._rescale(k, v, self.rng(S_MIX, layer, 1 << 20, step))
         return bf16_bits(k), bf16_bits(v), bf16_bits(q)
+
+    def _rescale(self, k, v, r):
+        """Value-range variants: scale fp32 K, V [n, Hkv, D] draws before rounding."""
+        if self.k_scale != 1.0:
+            k = k * np.float32(self.k_scale)
+        if self.v_scale != 1.0:
+            v = v * np.float32(self.v_scale)
+        if self.scale_mix:
+            n, G = k.shape[0], self.D // 32
+            for which in (0, 1):
+                lv = MIX_LEVELS[r.integers(0, MIX_LEVELS.size, size=(n, self.Hkv, G))]
+                m = np.repeat(lv, 32, axis=2)
+                if which == 0:
+                    k = k * m
+                else:
+                    v = v * m
+        return k, v
 
     def protected(self, seq: int) -> list:
         """Logical pages the caller marks protected (sorted).  Candidates are the full pages

@@ -224,6 +224,43 @@ def tq3_slot_bytes(kq, ks, vq, vs):
     return np.concatenate(out)
 
 
+# --------------------------------------------------------------------------- BF16 control pages
+# The control format the pages compare against ("Memória e compressão": KV bytes versus BF16):
+# the bf16 values stored as they are.  Slot per KV head: K rows [16 tokens][D] then V rows
+# [16][D], bf16 little-endian; rows of tokens not yet written are zero.
+def bf16_head_bytes(D: int) -> int:
+    return 2 * PAGE_TOKENS * D * 2
+
+
+def f64_to_bf16_bits(x):
+    """float64 values that bf16 holds exactly -> their uint16 bit patterns."""
+    x = np.asarray(x, dtype=np.float64)
+    f = x.astype(np.float32)
+    if not np.array_equal(f.astype(np.float64), x, equal_nan=True):
+        raise ValueError("value not representable in fp32")
+    u = f.view(np.uint32)
+    if np.any(u & np.uint32(0xFFFF)):
+        raise ValueError("value not representable in bf16")
+    return (u >> np.uint32(16)).astype(np.uint16)
+
+
+def bf16_slot_bytes(kbits, vbits):
+    """Raw bytes of a BF16 slot: kbits, vbits uint16 [Hkv, 16, D]; per KV head K rows then V
+    rows, each element little-endian."""
+    out = []
+    for h in range(kbits.shape[0]):
+        out.append(np.asarray(kbits[h], dtype="<u2").reshape(-1).view(np.uint8))
+        out.append(np.asarray(vbits[h], dtype="<u2").reshape(-1).view(np.uint8))
+    return np.concatenate(out)
+
+
+def parse_bf16_slot(raw, Hkv, D):
+    """Inverse of bf16_slot_bytes: -> (kbits, vbits) uint16 [Hkv, 16, D]."""
+    raw = np.asarray(raw, dtype=np.uint8)
+    b = raw[:Hkv * bf16_head_bytes(D)].view("<u2").reshape(Hkv, 2, PAGE_TOKENS, D)
+    return b[:, 0].astype(np.uint16), b[:, 1].astype(np.uint16)
+
+
 def parse_fp8_slot(raw, Hkv, D):
     """Inverse of fp8_slot_bytes: -> (kcodes, vcodes [Hkv,16,D], kscale, vscale [Hkv])."""
     raw = np.asarray(raw, dtype=np.uint8)

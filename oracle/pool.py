@@ -15,8 +15,14 @@ are converted to packed TQ3.  Readings of what the pages leave open:
 * Slots are handed out lowest rank first (rank = position in a per-format slot order,
   identity unless set), sequences in the order the call lists them, pages ascending.
   Slots freed by a call return to the free list at the end of that call.
-* Block-table entry: -1 unmapped, else (format << 30) | slot with format 0 = FP8, 1 = TQ3.
+* Block-table entry: -1 unmapped, else (format << 30) | slot with format 0 = FP8, 1 = TQ3,
+  2 = BF16.
 * A call that fails changes nothing.
+
+A control pool (``bf16_control=True``) models the comparator the pages measure the method
+against ("Memória e compressão", "Verificação canário"): every page holds its bf16 values as
+they are (format BF16, taken from the first slab), no page is ever demoted, and attention runs
+over those values.
 """
 from __future__ import annotations
 
@@ -26,8 +32,13 @@ import numpy as np
 
 from . import formats as F
 
-FP8, TQ3 = 0, 1
+FP8, TQ3, BF16 = 0, 1, 2
 PAGE = F.PAGE_TOKENS
+
+
+def _slab(fmt):
+    """Slab (and allocator) of a format: BF16 control pages use the first slab, as FP8."""
+    return 1 if fmt == TQ3 else 0
 
 
 class PoolError(Exception):
@@ -70,7 +81,7 @@ class RefPool:
     """The pool's whole observable state: tables, lengths, flags and every slot's contents."""
 
     def __init__(self, Hkv, D, max_seqs, max_pages_per_seq, fp8_slots, tq3_slots,
-                 sink_pages=1):
+                 sink_pages=1, bf16_control=False):
         if D % F.TQ3_GROUP:
             raise PoolError("INVALID_ARG", "head_dim must be a multiple of 32")
         self.Hkv, self.D, self.G = Hkv, D, D // F.TQ3_GROUP
@@ -82,6 +93,9 @@ class RefPool:
         self.protected = [set() for _ in range(max_seqs)]
         self.fp8 = {}   # slot -> [kcodes [Hkv,16,D], vcodes, kscale [Hkv], vscale [Hkv]]
         self.tq3 = {}   # slot -> [kq [Hkv,16,D], ks [Hkv,16,G], vq, vs]
+        self.bf16_control = bf16_control
+        self.bf16 = {}  # slot -> [kbits [Hkv,16,D] uint16, vbits]  (control pools)
+        self.page_fmt = BF16 if bf16_control else FP8   # format of written (unconverted) pages
 
     # ------------------------------------------------------------------ helpers
     def _check_seq(self, s):
@@ -89,11 +103,43 @@ class RefPool:
             raise PoolError("BAD_SEQ", f"sequence {s}")
 
     def set_slot_order(self, fmt, order):
-        self.alloc[fmt].set_order(order)
+        self.alloc[_slab(fmt)].set_order(order)
+
+    def _store(self, fmt):
+        return {FP8: self.fp8, TQ3: self.tq3, BF16: self.bf16}[fmt]
+
+    def _new_page(self, seq):
+        """Take a slot for a fresh written page (FP8, or BF16 in a control pool)."""
+        slot = self.alloc[0].take()
+        z = np.zeros((self.Hkv, PAGE, self.D), np.uint8)
+        if self.bf16_control:
+            zb = np.zeros((self.Hkv, PAGE, self.D), np.uint16)
+            self.bf16[slot] = [zb, zb.copy()]
+        else:
+            self.fp8[slot] = [z, z.copy(), np.zeros(self.Hkv), np.zeros(self.Hkv)]
+        self.table[seq].append((self.page_fmt, slot))
+        return slot
+
+    def _write_rows(self, slot, off, k, v):
+        """Write rows [off, off + n) of a written page from k, v float64 [n, Hkv, D]."""
+        if self.bf16_control:
+            st = self.bf16[slot]
+            for which, src in ((0, k), (1, v)):
+                st[which][:, off:off + src.shape[0], :] = F.f64_to_bf16_bits(
+                    np.transpose(src, (1, 0, 2)))
+            return
+        st = self.fp8[slot]
+        for h in range(self.Hkv):
+            for which, src in ((0, k), (1, v)):
+                codes, sc = F.fp8_write(st[which][h], st[2 + which][h], off, src[:, h, :])
+                st[which][h] = codes
+                st[2 + which][h] = sc
 
     def entry(self, seq, page) -> int:
+        """The int32 table entry (format 2 sets the sign bit)."""
         fmt, slot = self.table[seq][page]
-        return (fmt << 30) | slot
+        e = (fmt << 30) | slot
+        return e - (1 << 32) if e >= 1 << 31 else e
 
     def block_table(self, seq):
         return [self.entry(seq, p) for p in range(len(self.table[seq]))]
@@ -121,24 +167,15 @@ class RefPool:
             L0 = self.ctx[s]
             pages_after = -(-(L0 + n) // PAGE)
             for _ in range(len(self.table[s]), pages_after):
-                slot = self.alloc[FP8].take()
-                self.table[s].append((FP8, slot))
-                z = np.zeros((self.Hkv, PAGE, self.D), np.uint8)
-                self.fp8[slot] = [z, z.copy(), np.zeros(self.Hkv), np.zeros(self.Hkv)]
+                self._new_page(s)
             t = 0
             while t < n:
                 pos = L0 + t
                 page, off = divmod(pos, PAGE)
                 cnt = min(PAGE - off, n - t)
                 fmt, slot = self.table[s][page]
-                assert fmt == FP8
-                st = self.fp8[slot]
-                for h in range(self.Hkv):
-                    for which, src in ((0, k), (1, v)):
-                        x = src[row + t:row + t + cnt, h, :]
-                        codes, sc = F.fp8_write(st[which][h], st[2 + which][h], off, x)
-                        st[which][h] = codes
-                        st[2 + which][h] = sc
+                assert fmt == self.page_fmt
+                self._write_rows(slot, off, k[row + t:row + t + cnt], v[row + t:row + t + cnt])
                 t += cnt
             self.ctx[s] = L0 + n
             row += n
@@ -167,8 +204,8 @@ class RefPool:
             pages = -(-n // PAGE)
             if pages > self.max_pages:
                 raise PoolError("OUT_OF_PAGES", f"sequence {s} exceeds max pages")
-            d = [p >= self.sink_pages and PAGE * p + PAGE <= n - window_tokens
-                 for p in range(pages)]
+            d = [not self.bf16_control and p >= self.sink_pages
+                 and PAGE * p + PAGE <= n - window_tokens for p in range(pages)]
             direct.append(d)
             need[TQ3] += sum(d)
             need[FP8] += pages - sum(d)
@@ -189,17 +226,8 @@ class RefPool:
                     self.tq3[slot] = res
                     self.table[s].append((TQ3, slot))
                 else:
-                    slot = self.alloc[FP8].take()
-                    z = np.zeros((self.Hkv, PAGE, self.D), np.uint8)
-                    st = [z, z.copy(), np.zeros(self.Hkv), np.zeros(self.Hkv)]
-                    for h in range(self.Hkv):
-                        for which, src in ((0, k), (1, v)):
-                            codes, sc = F.fp8_write(st[which][h], st[2 + which][h], 0,
-                                                    src[r0:r0 + cnt, h, :])
-                            st[which][h] = codes
-                            st[2 + which][h] = sc
-                    self.fp8[slot] = st
-                    self.table[s].append((FP8, slot))
+                    slot = self._new_page(s)
+                    self._write_rows(slot, 0, k[r0:r0 + cnt], v[r0:r0 + cnt])
             self.ctx[s] = n
             row += n
 
@@ -234,7 +262,8 @@ class RefPool:
             self._check_seq(s)
         if len(set(seq_ids)) != len(seq_ids) or window_tokens < 0:
             raise PoolError("INVALID_ARG", "repeated sequence or negative window")
-        work = [(s, p) for s in seq_ids for p in self.demote_candidates(s, window_tokens)]
+        work = [] if self.bf16_control else [
+            (s, p) for s in seq_ids for p in self.demote_candidates(s, window_tokens)]
         if len(work) > len(self.alloc[TQ3].free):
             raise PoolError("OUT_OF_PAGES", "TQ3 pool exhausted")
         done, freed = [], []
@@ -264,13 +293,9 @@ class RefPool:
     # ------------------------------------------------------------------ lifecycle
     def seq_reset(self, seq):
         self._check_seq(seq)
-        freed = [[], []]
         for fmt, slot in self.table[seq]:
-            freed[fmt].append(slot)
-        for fmt in (FP8, TQ3):
-            for slot in freed[fmt]:
-                (self.fp8 if fmt == FP8 else self.tq3).pop(slot)
-                self.alloc[fmt].give(slot)
+            self._store(fmt).pop(slot)
+            self.alloc[_slab(fmt)].give(slot)
         self.table[seq] = []
         self.ctx[seq] = 0
         self.protected[seq] = set()
@@ -283,13 +308,13 @@ class RefPool:
             raise PoolError("INVALID_ARG", "destination must be a different, empty sequence")
         need = [0, 0]
         for fmt, _ in self.table[src]:
-            need[fmt] += 1
-        for fmt in (FP8, TQ3):
-            if need[fmt] > len(self.alloc[fmt].free):
+            need[_slab(fmt)] += 1
+        for slab in (0, 1):
+            if need[slab] > len(self.alloc[slab].free):
                 raise PoolError("OUT_OF_PAGES", "pool exhausted")
         for fmt, slot in self.table[src]:
-            new = self.alloc[fmt].take()
-            store = self.fp8 if fmt == FP8 else self.tq3
+            new = self.alloc[_slab(fmt)].take()
+            store = self._store(fmt)
             store[new] = [np.array(a, copy=True) for a in store[slot]]
             self.table[dst].append((fmt, new))
         self.ctx[dst] = self.ctx[src]
@@ -297,10 +322,13 @@ class RefPool:
 
     # ------------------------------------------------------------------ views
     def slot_bytes(self, entry: int):
-        fmt, slot = entry >> 30, entry & ((1 << 30) - 1)
+        fmt, slot = (entry >> 30) & 3, entry & ((1 << 30) - 1)
         if fmt == FP8:
             kc, vc, ks, vs = self.fp8[slot]
             return F.fp8_slot_bytes(kc, vc, ks, vs)
+        if fmt == BF16:
+            kb, vb = self.bf16[slot]
+            return F.bf16_slot_bytes(kb, vb)
         kq, ks, vq, vs = self.tq3[slot]
         return F.tq3_slot_bytes(kq, ks, vq, vs)
 
@@ -318,6 +346,10 @@ class RefPool:
                     kc, vc, ks, vs = self.fp8[slot]
                     K[rows, j] = F.fp8_dequant(kc[h], ks[h])
                     V[rows, j] = F.fp8_dequant(vc[h], vs[h])
+                elif fmt == BF16:
+                    kb, vb = self.bf16[slot]
+                    K[rows, j] = F.bf16_bits_to_f64(kb[h])
+                    V[rows, j] = F.bf16_bits_to_f64(vb[h])
                 else:
                     kq, kscale, vq, vscale = self.tq3[slot]
                     K[rows, j] = F.tq3_dequant(kq[h].reshape(PAGE, self.G, F.TQ3_GROUP),
@@ -328,7 +360,8 @@ class RefPool:
 
     def stats(self):
         live = sum(self.ctx)
-        n8 = sum(1 for t in self.table for f, _ in t if f == FP8)
+        n8 = sum(1 for t in self.table for f, _ in t if f == self.page_fmt)
         n3 = sum(1 for t in self.table for f, _ in t if f == TQ3)
-        kv_bytes = n8 * self.Hkv * F.fp8_head_bytes(self.D) + n3 * self.Hkv * F.tq3_head_bytes(self.D)
+        head = F.bf16_head_bytes(self.D) if self.bf16_control else F.fp8_head_bytes(self.D)
+        kv_bytes = n8 * self.Hkv * head + n3 * self.Hkv * F.tq3_head_bytes(self.D)
         return live, n8, n3, (kv_bytes / live if live else 0.0)

@@ -13,14 +13,16 @@ ATOL = 2e-3
 REL_L2 = 1e-3
 
 
-def oracle_pool(w: Workload, layer: int = 0, shape: dict | None = None, seqs=None, heads=None):
+def oracle_pool(w: Workload, layer: int = 0, shape: dict | None = None, seqs=None, heads=None,
+                bf16_control: bool = False):
     """Oracle pool after the workload's build calls.  ``seqs`` restricts the build to some
     sequences (their contents do not depend on the others); ``heads`` keeps only some KV
-    heads (pages of one head depend only on that head's inputs)."""
+    heads (pages of one head depend only on that head's inputs).  ``bf16_control`` builds the
+    BF16 control pool instead (pages keep their bf16 values, nothing is demoted)."""
     shape = shape or w.pool_shape()
     Hkv = shape["num_kv_heads"] if heads is None else len(heads)
     pool = P.RefPool(Hkv, shape["head_dim"], shape["max_seqs"], shape["max_pages_per_seq"],
-                     shape["fp8_slots"], shape["tq3_slots"])
+                     shape["fp8_slots"], shape["tq3_slots"], bf16_control=bf16_control)
     if seqs is None and heads is None:
         for fmt, key in ((P.FP8, "fp8_slots"), (P.TQ3, "tq3_slots")):
             order = w.slot_permutation(fmt, shape[key])
@@ -48,11 +50,12 @@ def to_bf16_tensor(bits, device="cuda"):
     return t.to(device)
 
 
-def lib_pool(w: Workload, layer: int = 0, shape: dict | None = None, host_only: bool = False):
+def lib_pool(w: Workload, layer: int = 0, shape: dict | None = None, host_only: bool = False,
+             bf16_control: bool = False):
     """Library pool after the same build calls (inputs copied to the device per call)."""
     from mixed_format_paged_mkv_b200 import Pool
     shape = shape or w.pool_shape()
-    pool = Pool(**shape, host_only=host_only)
+    pool = Pool(**shape, host_only=host_only, bf16_control=bf16_control)
     for fmt, key in ((0, "fp8_slots"), (1, "tq3_slots")):
         order = w.slot_permutation(fmt, shape[key])
         if order is not None:

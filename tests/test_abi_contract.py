@@ -85,10 +85,13 @@ def test_config_validation_and_required_bytes():
     assert [s.value for s in sizes] == [8 * 2 * (32 * 64 + 16), 8 * 2 * 14 * 64, 4 * 8 * 4, 256]
     assert L.mkv_pool_required_bytes(ctypes.byref(c), None, None, None, None) == OK
     assert L.mkv_pool_required_bytes(None, None, None, None, None) == INVALID_ARG
+    ctl = cfg(flags=2)      # BF16 control pool: the first slab holds 64*D bytes per head
+    assert L.mkv_pool_required_bytes(ctypes.byref(ctl), *[ctypes.byref(s) for s in sizes]) == OK
+    assert sizes[0].value == 8 * 2 * 64 * 64
     for bad, code in ((dict(head_dim=96), UNSUPPORTED), (dict(page_size=32), INVALID_ARG),
                       (dict(num_kv_heads=0), INVALID_ARG), (dict(max_seqs=0), INVALID_ARG),
                       (dict(fp8_slots=0), INVALID_ARG), (dict(tq3_slots=-1), INVALID_ARG),
-                      (dict(sink_pages=-1), INVALID_ARG), (dict(flags=2), INVALID_ARG),
+                      (dict(sink_pages=-1), INVALID_ARG), (dict(flags=4), INVALID_ARG),
                       (dict(max_seqs=1 << 16, max_pages_per_seq=1 << 16), INVALID_ARG)):
         c = cfg(**bad)
         assert L.mkv_pool_required_bytes(ctypes.byref(c), None, None, None, None) == code, bad

@@ -43,6 +43,21 @@ def test_workloads_scaled(cfg, kw):
     run_and_check(WORKLOADS[cfg].scaled(**kw))
 
 
+@pytest.mark.parametrize("fused", [False, True])
+@pytest.mark.parametrize("w", [
+    WORKLOADS[2].scaled(B=3, ctx=(800, 2048, 1500)),
+    WORKLOADS[3].scaled(B=4, ctx_range=(200, 3000), window=256, protect_frac=0.3),
+    Workload("fp8heavy", 17, B=2, Hq=8, Hkv=2, D=256, q_len=1, window=2000, ctx=(2500, 900)),
+    Workload("multitok", 18, B=2, Hq=12, Hkv=2, D=128, q_len=3, window=48, ctx=(1200, 77)),
+], ids=["batch", "ragged", "fp8heavy", "multitok"])
+def test_split_and_fused_partial_kernels(w, fused):
+    """The per-format grids (TQ3 grid, then the FP8 grid as its programmatic dependent) and the
+    fused grid both match the oracle."""
+    lp = lib_pool(w)
+    lp.set_decode_kernels(fused)
+    run_and_check(w, lp=lp)
+
+
 def test_long_qlen4_scaled():
     run_and_check(long_qlen4().scaled(B=2, ctx=(3001, 1200), layers=1))
 
