@@ -467,10 +467,10 @@ def run_gpu(args, rank, world, local_rank):
                    "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2: each decode reads ~494 MB of pages; 48 layers cycle",
                    "decode_bytes_per_layer_call": int(per_call_total)},
-        "roofline": {"bound": "hbm", "kernel": "decode_kernel (FP8 + TQ3 partial attention)",
+        "roofline": {"bound": "hbm", "kernel": "partial_kernel: the FP8 and TQ3 grids of a call",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_source": peak_src,
-                     "traffic": ncu_traffic("decode_kernel"),
+                     "traffic": ncu_traffic("partial_grids"),
                      "bytes_per_launch": int(per_call_partial),
                      "launch_ms": round(partial_ms, 5),
                      "merge_ms": round(tm["merge_ms"] / max(tm["calls"], 1), 5),

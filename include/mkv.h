@@ -229,15 +229,19 @@ MKV_API int mkv_decode_attention_noalloc(mkv_pool_t pool, const int32_t* seq_ids
                                          int32_t q_len, const void* q_bf16, int32_t num_q_heads,
                                          float sm_scale, float* out, void* stream);
 
-/* Which partial-attention kernels decode uses (both compute the same partial states, so the
- * results are identical; this exists to compare the two designs):
- *   MKV_DECODE_SPLIT (default) -- a separate kernel per page format, as the pages describe
- *     (section "Como os resultados parciais são combinados"): the TQ3 grid, then the FP8 grid
- *     launched as its programmatic dependent so that FP8 CTAs take SM room as TQ3 CTAs retire;
- *   MKV_DECODE_FUSED -- one grid whose CTAs branch on their unit's format.
+/* Which partial-attention kernels decode uses (both compute the same partial states; results
+ * agree within the attention tolerance, the work cut differing):
+ *   MKV_DECODE_SPLIT -- a separate kernel per page format, as the pages describe (section "Como
+ *     os resultados parciais são combinados"): the FP8 grid, then the TQ3 grid launched as its
+ *     programmatic dependent, so both share one wave;
+ *   MKV_DECODE_FUSED -- one grid whose CTAs branch on their unit's format;
+ *   MKV_DECODE_AUTO (default) -- per call: FUSED when FP8 pages carry more than 15% of the
+ *     call's planned time, else SPLIT (FP8 CTAs need more shared memory than TQ3 CTAs, so many
+ *     of them no longer fit one wave of per-format grids).
  * Host only; applies to later decode calls on this pool.  Errors: INVALID_ARG. */
 #define MKV_DECODE_SPLIT 0
 #define MKV_DECODE_FUSED 1
+#define MKV_DECODE_AUTO 2
 MKV_API int mkv_set_decode_kernels(mkv_pool_t pool, int32_t mode);
 
 /* Free every page of a sequence and clear its table row and flags. */

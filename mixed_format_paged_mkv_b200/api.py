@@ -353,9 +353,10 @@ class Pool:
         return dict(partial_ms=v[0].value, merge_ms=v[1].value, calls=n.value)
 
     def set_decode_kernels(self, fused):
-        """Decode with one fused partial grid (True) or a grid per page format (False)."""
-        _check(lib().mkv_set_decode_kernels(self.handle, 1 if fused else 0),
-               "mkv_set_decode_kernels")
+        """Decode with one fused partial grid (True), a grid per page format (False) or the
+        automatic per-call choice (None, the default)."""
+        mode = 2 if fused is None else (1 if fused else 0)
+        _check(lib().mkv_set_decode_kernels(self.handle, mode), "mkv_set_decode_kernels")
 
     def test_fail_launch(self, after):
         """Make the device operation after the next ``after`` ones fail (test hook; -1: off)."""

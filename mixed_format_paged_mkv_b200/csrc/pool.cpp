@@ -121,7 +121,7 @@ struct mkv_pool {
   Allocator alloc[2];
   int64_t launches = 0;
   int64_t fail_after = -1;  // test hook: device operations that still succeed before one fails
-  bool fused_decode = false;  // decode kernels: per-format grids (default) or one fused grid
+  int decode_kernels = MKV_DECODE_AUTO;  // per-format grids, one fused grid, or chosen per call
   int page_fmt = MKV_FMT_FP8;  // format of written pages: FP8, or BF16 in a control pool
   bool timing = false;
   std::vector<TimingRec> timing_recs;
@@ -132,8 +132,31 @@ namespace {
 
 bool valid_pool(mkv_pool_t p) { return p != nullptr; }
 
-int decode_mode(const mkv_pool* p) {
-  return p->page_fmt == MKV_FMT_BF16 ? kDecodeBf16 : (p->fused_decode ? kDecodeFused : kDecodeSplit);
+// Relative time of one page of each format in a CTA (measured with device timestamps on the
+// long-context workload: 0.45 us per TQ3 page and 0.48-0.53 us per FP8 page per CTA).  Units are
+// balanced by time, not bytes: an FP8 page carries 2.3x the bytes of a TQ3 page but costs less
+// arithmetic per byte.
+constexpr int64_t kFp8PageCost = 11;
+constexpr int64_t kTq3PageCost = 10;
+// Automatic choice of partial kernels: one fused grid when FP8 pages carry more than this share
+// of the call's planned time.  Measured on the long-context workload: at 4% FP8 pages the
+// per-format grids are faster (150.8 against 156.3 us), at 25% the fused grid (170.0 against
+// 198.8 us): FP8 CTAs need more shared memory than TQ3 CTAs, so beyond one FP8 CTA per SM the
+// per-format grids no longer fit one wave.
+constexpr double kFusedAboveFp8Share = 0.15;
+
+// Decode kernels of a call over these sequences (kDecodeSplit, kDecodeFused or kDecodeBf16).
+int decode_mode(const mkv_pool* p, const int32_t* seq_ids, int32_t n) {
+  if (p->page_fmt == MKV_FMT_BF16) return kDecodeBf16;
+  if (p->decode_kernels != MKV_DECODE_AUTO)
+    return p->decode_kernels == MKV_DECODE_FUSED ? kDecodeFused : kDecodeSplit;
+  int64_t c8 = 0, c3 = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    const Seq& s = p->seqs[seq_ids[i]];
+    c8 += static_cast<int64_t>(s.fp8_pages.size()) * kFp8PageCost;
+    c3 += static_cast<int64_t>(s.n3) * kTq3PageCost;
+  }
+  return c8 > kFusedAboveFp8Share * static_cast<double>(c8 + c3) ? kDecodeFused : kDecodeSplit;
 }
 
 int64_t page_head_bytes(const mkv_pool_config& c) {
@@ -189,6 +212,7 @@ size_t status_bytes(const mkv_pool_config&) { return 256; }
 
 struct DecodePlan {
   int32_t NC = 0, g = 0;
+  int mode = kDecodeSplit;     // partial kernels of the call
   std::vector<SeqDesc> seq;    // per call position
   std::vector<UnitDesc> unit;  // per sequence, in order
   std::vector<int32_t> pos;    // call position of each unit's sequence
@@ -212,15 +236,9 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 // `emit` returns false.
 constexpr int kMinTq3PagesPerUnit = 8;
 constexpr int kMinFp8PagesPerUnit = 4;
-// Relative time of one page of each format in a CTA (measured with device timestamps on the
-// long-context workload: 0.45 us per TQ3 page and 0.48-0.53 us per FP8 page per CTA).  Units are
-// balanced by time, not bytes: an FP8 page carries 2.3x the bytes of a TQ3 page but costs less
-// arithmetic per byte.
-constexpr int64_t kFp8PageCost = 11;
-constexpr int64_t kTq3PageCost = 10;
 
 template <class Emit>
-int64_t cut_units(const mkv_pool* p, const int32_t* seq_ids, int32_t n, int32_t NC,
+int64_t cut_units(const mkv_pool* p, const int32_t* seq_ids, int32_t n, int32_t NC, int mode,
                   int32_t* n_parts, Emit&& emit) {
   const int64_t b8 = kFp8PageCost, b3 = kTq3PageCost;
   const int Hkv = p->cfg.num_kv_heads;
@@ -230,7 +248,7 @@ int64_t cut_units(const mkv_pool* p, const int32_t* seq_ids, int32_t n, int32_t 
     total += static_cast<int64_t>(s.fp8_pages.size()) * b8 + static_cast<int64_t>(s.n3) * b3;
   }
   const int64_t slots =
-      static_cast<int64_t>(p->sm_count) * partial_ctas_per_sm(p->cfg.head_dim, NC, decode_mode(p));
+      static_cast<int64_t>(p->sm_count) * partial_ctas_per_sm(p->cfg.head_dim, NC, mode);
   const int64_t U = std::max<int64_t>(1, slots / Hkv);
   // units of a group at unit cost c: as many as its cost needs, clamped to the page limits
   auto units_at = [](double c, int64_t cost, int64_t pages, int min_pages) -> int64_t {
@@ -328,7 +346,9 @@ int plan_decode(mkv_pool_t p, const int32_t* seq_ids, int32_t n, int32_t q_len, 
   plan->pos.clear();
   plan->cost.clear();
   std::vector<int32_t> np(n);
-  cut_units(p, seq_ids, n, plan->NC, np.data(), [&](const UnitDesc& u, int64_t cost, int32_t i) {
+  plan->mode = decode_mode(p, seq_ids, n);
+  cut_units(p, seq_ids, n, plan->NC, plan->mode, np.data(),
+            [&](const UnitDesc& u, int64_t cost, int32_t i) {
     plan->unit.push_back(u);
     plan->pos.push_back(i);
     plan->cost.push_back(cost);
@@ -694,7 +714,7 @@ int mkv_decode_plan(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, int32_
   const int64_t nu = static_cast<int64_t>(plan.unit.size());
   *n_units = static_cast<int32_t>(nu);
   if (ctas_per_wave)
-    *ctas_per_wave = p->sm_count * partial_ctas_per_sm(p->cfg.head_dim, plan.NC, decode_mode(p));
+    *ctas_per_wave = p->sm_count * partial_ctas_per_sm(p->cfg.head_dim, plan.NC, plan.mode);
   if (!units_out) return ok();  // count query
   if (nu > cap) return fail(MKV_ERR_INVALID_ARG, "%lld units do not fit in %d", (long long)nu, cap);
   const int64_t b[2] = {kFp8PageCost, kTq3PageCost};
@@ -775,7 +795,7 @@ int mkv_decode_attention(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, i
     for (int32_t i = s0; i < s1; ++i) prm->seq[i - s0] = plan.seq[i];
     order.resize(u1 - u0);
     prm->n_fp8 = order_units(
-        order.data(), static_cast<int32_t>(order.size()), p->fused_decode,
+        order.data(), static_cast<int32_t>(order.size()), plan.mode != kDecodeSplit,
         [&](int32_t k) { return static_cast<int>(plan.unit[u0 + k].fmt); },
         [&](int32_t k) { return plan.cost[u0 + k]; });
     for (size_t k = 0; k < order.size(); ++k) {
@@ -784,7 +804,7 @@ int mkv_decode_attention(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, i
     }
     prm->n_seqs = s1 - s0;
     prm->n_units = static_cast<int32_t>(order.size());
-    prm->fused = p->fused_decode ? 1 : 0;
+    prm->fused = plan.mode == kDecodeFused ? 1 : 0;
     prm->page_fmt = p->page_fmt;
     const bool last = s1 >= n_seqs;
     err = launch_partial(*prm, st);
@@ -852,7 +872,8 @@ int mkv_decode_attention_noalloc(mkv_pool_t p, const int32_t* seq_ids, int32_t n
     t.cost[nu++] = cost;
     return true;
   };
-  const int64_t cut = cut_units(p, seq_ids, n_seqs, NC, np, keep);
+  const int mode = decode_mode(p, seq_ids, n_seqs);
+  const int64_t cut = cut_units(p, seq_ids, n_seqs, NC, mode, np, keep);
   if (cut < 0)
     return fail(MKV_ERR_UNSUPPORTED, "the no-allocation decode takes at most %d work units per call", kDecodeMaxUnits);
   int32_t parts = 0;
@@ -876,10 +897,10 @@ int mkv_decode_attention_noalloc(mkv_pool_t p, const int32_t* seq_ids, int32_t n
   if (bytes > cap)
     return fail(MKV_ERR_WORKSPACE_TOO_SMALL,
                 "call needs %zu bytes of partial-state scratch; the static scratch holds %zu", bytes, cap);
-  prm.n_fp8 = order_units(t.order, nu, p->fused_decode,
+  prm.n_fp8 = order_units(t.order, nu, mode != kDecodeSplit,
                           [&](int32_t k) { return static_cast<int>(t.unit[k].fmt); },
                           [&](int32_t k) { return t.cost[k]; });
-  prm.fused = p->fused_decode ? 1 : 0;
+  prm.fused = mode == kDecodeFused ? 1 : 0;
   prm.page_fmt = p->page_fmt;
   for (int32_t k = 0; k < nu; ++k) prm.unit[k] = t.unit[t.order[k]];
   uint8_t* ws = static_cast<uint8_t*>(scratch);
@@ -1260,9 +1281,9 @@ int mkv_timing_read(mkv_pool_t p, double* ms_partial, double* ms_merge, int64_t*
 
 int mkv_set_decode_kernels(mkv_pool_t p, int32_t mode) {
   if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
-  if (mode != MKV_DECODE_SPLIT && mode != MKV_DECODE_FUSED)
+  if (mode != MKV_DECODE_SPLIT && mode != MKV_DECODE_FUSED && mode != MKV_DECODE_AUTO)
     return fail(MKV_ERR_INVALID_ARG, "unknown decode kernel mode %d", mode);
-  p->fused_decode = mode == MKV_DECODE_FUSED;
+  p->decode_kernels = mode;
   return ok();
 }
 
