@@ -792,65 +792,82 @@ __device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDes
 }
 
 // Merge of the partial states of one (sequence, KV head, query column): the globally
-// normalised combination M = max m, L = sum l 2^(m-M), O = sum acc 2^(m-M) / L.  The maximum and
-// the weights are computed once in shared memory; the accumulation over partials is then a
-// branch-free sum of independent float4 loads, split over thread groups and reduced at the end.
-constexpr int kMergeThreads = 256;
+// normalised combination M = max m, L = sum l 2^(m-M), O = sum acc 2^(m-M) / L.  One pass: a
+// thread owns 4 channels of a subset of the partials (every nsub-th one) and keeps a running
+// (m, l, acc) over them, loading eight partials at a time so that their loads are in flight
+// together; the subsets are combined in shared memory at the end.  Two dependent rounds of
+// memory access in all (the partial states, then the output) for up to 8 x nsub partials.
+constexpr int kMergeThreads = 512;
+constexpr int kMergeBatch = 8;
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_constant__ DecodeParams p) {
-  __shared__ float w[kDecodeMaxUnits];
-  __shared__ float red[kMergeThreads / 32];
-  __shared__ float4 part[kMergeThreads];
+  __shared__ float4 part_o[kMergeThreads];
+  __shared__ float2 part_ml[kMergeThreads];
   // launched as a programmatic dependent of the partial kernels: resident early, it reads the
   // partial states only once they are complete and visible
   pdl_wait();
   const int pair = blockIdx.x / p.NC, n = blockIdx.x % p.NC;
   const SeqDesc& sd = p.seq[pair / p.Hkv];
   const int h = pair % p.Hkv;
-  const int S = sd.n_parts, D = p.D, tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+  const int S = sd.n_parts, D = p.D, tid = threadIdx.x;
+  const int groups = D / 4, nsub = kMergeThreads / groups;
+  const int c4 = tid % groups, k = tid / groups;
   const int64_t base0 = (static_cast<int64_t>(sd.part0) * p.Hkv + h) * p.NC + n;
   const int64_t stride = static_cast<int64_t>(p.Hkv) * p.NC;
   const float2* ml = reinterpret_cast<const float2*>(p.part_ml);
-  float mloc = -INFINITY;
-  for (int j = tid; j < S; j += kMergeThreads) mloc = fmaxf(mloc, ml[base0 + j * stride].x);
-  for (int o = 16; o > 0; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
-  if (lane == 0) red[wp] = mloc;
-  __syncthreads();
-  float M = -INFINITY;
-  for (int i = 0; i < kMergeThreads / 32; ++i) M = fmaxf(M, red[i]);
-  __syncthreads();
-  float lloc = 0.f;
-  for (int j = tid; j < S; j += kMergeThreads) {
-    const float2 v = ml[base0 + j * stride];
-    const float wj = (v.x == -INFINITY || M == -INFINITY) ? 0.f : exp2f(v.x - M);
-    w[j] = wj;
-    lloc = fmaf(wj, v.y, lloc);
-  }
-  for (int o = 16; o > 0; o >>= 1) lloc += __shfl_xor_sync(0xffffffffu, lloc, o);
-  if (lane == 0) red[wp] = lloc;
-  __syncthreads();
-  float L = 0.f;
-  for (int i = 0; i < kMergeThreads / 32; ++i) L += red[i];
-  // accumulation: thread = (subset k of the partials, group c4 of 4 channels)
-  const int groups = D / 4, nsub = kMergeThreads / groups;
-  const int c4 = tid % groups, k = tid / groups;
-  float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
   const float4* acc = reinterpret_cast<const float4*>(p.part_acc);
-#pragma unroll 8
-  for (int j = k; j < S; j += nsub) {
-    const float4 a = acc[(base0 + j * stride) * groups + c4];
-    const float wj = w[j];
-    O.x = fmaf(wj, a.x, O.x);
-    O.y = fmaf(wj, a.y, O.y);
-    O.z = fmaf(wj, a.z, O.z);
-    O.w = fmaf(wj, a.w, O.w);
+  float m = -INFINITY, l = 0.f;
+  float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j0 = k; j0 < S; j0 += kMergeBatch * nsub) {
+    float2 v[kMergeBatch];
+    float4 a[kMergeBatch];
+#pragma unroll
+    for (int i = 0; i < kMergeBatch; ++i) {
+      const int j = j0 + i * nsub;
+      v[i] = make_float2(-INFINITY, 0.f);
+      a[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j < S) {
+        v[i] = ml[base0 + j * stride];
+        a[i] = acc[(base0 + j * stride) * groups + c4];
+      }
+    }
+    float mb = m;
+#pragma unroll
+    for (int i = 0; i < kMergeBatch; ++i) mb = fmaxf(mb, v[i].x);
+    if (mb == -INFINITY) continue;  // nothing attended so far
+    const float r = exp2f(m - mb);  // 0 while m is still -inf
+    l *= r;
+    o.x *= r; o.y *= r; o.z *= r; o.w *= r;
+#pragma unroll
+    for (int i = 0; i < kMergeBatch; ++i) {
+      const float wi = exp2f(v[i].x - mb);  // 0 for an empty partial
+      l = fmaf(wi, v[i].y, l);
+      o.x = fmaf(wi, a[i].x, o.x);
+      o.y = fmaf(wi, a[i].y, o.y);
+      o.z = fmaf(wi, a[i].z, o.z);
+      o.w = fmaf(wi, a[i].w, o.w);
+    }
+    m = mb;
   }
-  part[tid] = O;
+  part_o[tid] = o;
+  if (c4 == 0) part_ml[k] = make_float2(m, l);
   __syncthreads();
   if (tid < groups) {
-    float4 t = part[tid];
-    for (int i = 1; i < nsub; ++i) {
-      const float4 u = part[tid + i * groups];
-      t.x += u.x; t.y += u.y; t.z += u.z; t.w += u.w;
+    float M = -INFINITY;
+    for (int i = 0; i < nsub; ++i) M = fmaxf(M, part_ml[i].x);
+    float L = 0.f;
+    float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (M != -INFINITY) {
+      for (int i = 0; i < nsub; ++i) {
+        const float2 q = part_ml[i];
+        if (q.x == -INFINITY) continue;
+        const float wi = exp2f(q.x - M);
+        const float4 u = part_o[tid + i * groups];
+        L = fmaf(wi, q.y, L);
+        t.x = fmaf(wi, u.x, t.x);
+        t.y = fmaf(wi, u.y, t.y);
+        t.z = fmaf(wi, u.z, t.z);
+        t.w = fmaf(wi, u.w, t.w);
+      }
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
     const int qi = n / p.g, hq = h * p.g + n % p.g;
