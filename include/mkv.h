@@ -244,6 +244,12 @@ MKV_API int mkv_decode_attention_noalloc(mkv_pool_t pool, const int32_t* seq_ids
 #define MKV_DECODE_AUTO 2
 MKV_API int mkv_set_decode_kernels(mkv_pool_t pool, int32_t mode);
 
+/* Plan later decode calls on this pool for at most `sms` SMs (0, the default: all of the
+ * device's): the work cut then fills one wave of that many SMs, leaving room for work the
+ * caller runs beside decode on other streams.  It sizes the grid only: the hardware may still
+ * place CTAs on any SM.  Host only.  Errors: INVALID_ARG (sms < 0). */
+MKV_API int mkv_set_decode_sms(mkv_pool_t pool, int32_t sms);
+
 /* Free every page of a sequence and clear its table row and flags. */
 MKV_API int mkv_seq_reset(mkv_pool_t pool, int32_t seq, void* stream);
 

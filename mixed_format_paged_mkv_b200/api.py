@@ -70,6 +70,7 @@ SIGNATURES = {
     "mkv_launch_count": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int64)]),
     "mkv_test_fail_launch": (ctypes.c_int, [_P, _I32]),
     "mkv_set_decode_kernels": (ctypes.c_int, [_P, _I32]),
+    "mkv_set_decode_sms": (ctypes.c_int, [_P, _I32]),
     "mkv_last_error": (ctypes.c_char_p, []),
 }
 
@@ -357,6 +358,10 @@ class Pool:
         automatic per-call choice (None, the default)."""
         mode = 2 if fused is None else (1 if fused else 0)
         _check(lib().mkv_set_decode_kernels(self.handle, mode), "mkv_set_decode_kernels")
+
+    def set_decode_sms(self, sms):
+        """Plan later decode calls for at most ``sms`` SMs (0: all of the device's)."""
+        _check(lib().mkv_set_decode_sms(self.handle, int(sms)), "mkv_set_decode_sms")
 
     def test_fail_launch(self, after):
         """Make the device operation after the next ``after`` ones fail (test hook; -1: off)."""

@@ -117,6 +117,7 @@ struct mkv_pool {
   int32_t* d_status = nullptr;
   int64_t fp8_slot_bytes = 0, tq3_slot_bytes = 0;
   int sm_count = 148;
+  int decode_sms = 0;  // SMs decode plans for (0: all of the device's)
   std::vector<Seq> seqs;
   Allocator alloc[2];
   int64_t launches = 0;
@@ -157,6 +158,11 @@ int decode_mode(const mkv_pool* p, const int32_t* seq_ids, int32_t n) {
     c3 += static_cast<int64_t>(s.n3) * kTq3PageCost;
   }
   return c8 > kFusedAboveFp8Share * static_cast<double>(c8 + c3) ? kDecodeFused : kDecodeSplit;
+}
+
+// SMs a decode call's cut is planned for: the device's, or fewer when the caller asked so.
+int plan_sms(const mkv_pool* p) {
+  return p->decode_sms > 0 && p->decode_sms < p->sm_count ? p->decode_sms : p->sm_count;
 }
 
 int64_t page_head_bytes(const mkv_pool_config& c) {
@@ -248,7 +254,7 @@ int64_t cut_units(const mkv_pool* p, const int32_t* seq_ids, int32_t n, int32_t 
     total += static_cast<int64_t>(s.fp8_pages.size()) * b8 + static_cast<int64_t>(s.n3) * b3;
   }
   const int64_t slots =
-      static_cast<int64_t>(p->sm_count) * partial_ctas_per_sm(p->cfg.head_dim, NC, mode);
+      static_cast<int64_t>(plan_sms(p)) * partial_ctas_per_sm(p->cfg.head_dim, NC, mode);
   const int64_t U = std::max<int64_t>(1, slots / Hkv);
   // units of a group at unit cost c: as many as its cost needs, clamped to the page limits
   auto units_at = [](double c, int64_t cost, int64_t pages, int min_pages) -> int64_t {
@@ -714,7 +720,7 @@ int mkv_decode_plan(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, int32_
   const int64_t nu = static_cast<int64_t>(plan.unit.size());
   *n_units = static_cast<int32_t>(nu);
   if (ctas_per_wave)
-    *ctas_per_wave = p->sm_count * partial_ctas_per_sm(p->cfg.head_dim, plan.NC, plan.mode);
+    *ctas_per_wave = plan_sms(p) * partial_ctas_per_sm(p->cfg.head_dim, plan.NC, plan.mode);
   if (!units_out) return ok();  // count query
   if (nu > cap) return fail(MKV_ERR_INVALID_ARG, "%lld units do not fit in %d", (long long)nu, cap);
   const int64_t b[2] = {kFp8PageCost, kTq3PageCost};
@@ -1284,6 +1290,13 @@ int mkv_set_decode_kernels(mkv_pool_t p, int32_t mode) {
   if (mode != MKV_DECODE_SPLIT && mode != MKV_DECODE_FUSED && mode != MKV_DECODE_AUTO)
     return fail(MKV_ERR_INVALID_ARG, "unknown decode kernel mode %d", mode);
   p->decode_kernels = mode;
+  return ok();
+}
+
+int mkv_set_decode_sms(mkv_pool_t p, int32_t sms) {
+  if (!valid_pool(p)) return fail(MKV_ERR_INVALID_ARG, "pool is NULL");
+  if (sms < 0) return fail(MKV_ERR_INVALID_ARG, "sms must be >= 0");
+  p->decode_sms = sms;
   return ok();
 }
 

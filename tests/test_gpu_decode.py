@@ -58,6 +58,18 @@ def test_split_and_fused_partial_kernels(w, fused):
     run_and_check(w, lp=lp)
 
 
+def test_decode_planned_for_fewer_sms():
+    """A cut planned for 8 SMs (longer units, full page lists) matches the oracle too."""
+    w = Workload("fewsms", 19, B=2, Hq=8, Hkv=2, D=128, q_len=1, window=64, ctx=(12000, 900),
+                 outliers=True)
+    lp = lib_pool(w)
+    full, _ = lp.decode_plan([0, 1], 1, 8)
+    lp.set_decode_sms(8)
+    units, _ = lp.decode_plan([0, 1], 1, 8)
+    assert units[:, 4].max() > full[:, 4].max()
+    run_and_check(w, lp=lp)
+
+
 def test_long_qlen4_scaled():
     run_and_check(long_qlen4().scaled(B=2, ctx=(3001, 1200), layers=1))
 

@@ -188,3 +188,21 @@ def test_a_sequence_beyond_one_launch_is_rejected():
     pool.append([0], [16 * (pages - 1)])
     units, _ = pool.decode_plan([0], 1, 1)
     assert len(units) == 1536 and units[:, 4].max() == 512
+
+
+
+def test_decode_sms_caps_the_wave():
+    """set_decode_sms plans the cut for fewer SMs: the CTA budget of the wave shrinks with it and
+    the cut still covers every page once."""
+    pool, seqs = mixed_pool((16 * 8192, 5000), Hkv=2, window=64)
+    units, wave = pool.decode_plan(seqs, 1, 2)
+    pool.set_decode_sms(8)
+    small, small_wave = pool.decode_plan(seqs, 1, 2)
+    assert small_wave <= wave and small_wave <= 8 * 8
+    check_cut(pool, seqs, small, small_wave, 2)
+    assert len(small) <= len(units)
+    pool.set_decode_sms(0)
+    assert pool.decode_plan(seqs, 1, 2)[1] == wave
+    from mixed_format_paged_mkv_b200.api import MkvError
+    with pytest.raises(MkvError):
+        pool.set_decode_sms(-1)
