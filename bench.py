@@ -621,7 +621,8 @@ def run_extra(args):
             torch.cuda.empty_cache()
     elif args.mode == "profile":
         # a small target for ncu: one layer of the long-context workload, a few decode calls
-        w = WORKLOADS[4].scaled(layers=1)
+        w = WORKLOADS[4].scaled(layers=1, q_len=args.q_len,
+                                name=WORKLOADS[4].name + ("" if args.q_len == 1 else f"_q{args.q_len}"))
         pool = build_pool(w, 1, 3, device)
         pool.set_decode_kernels(args.fused)
         seqs = list(range(w.B))
@@ -879,6 +880,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--fused", action="store_true", help="--mode profile: the fused kernel")
+    ap.add_argument("--q-len", type=int, default=1, help="--mode profile: new tokens per sequence")
     ap.add_argument("--mode", choices=["bench", "sweep", "canary", "pack", "prefill", "materialise",
                                        "configs", "ablation", "profile"],
                     default="bench",

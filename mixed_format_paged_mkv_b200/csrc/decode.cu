@@ -58,8 +58,15 @@ enum Fmt { kFp8 = 0, kTq3 = 1, kBf16 = 2 };
 
 template <int D, int NT, int K>
 struct Cfg {
-  static constexpr int PW = NT == 1 ? 4 : (NT == 2 ? 2 : 1);  // page-parallel warp groups
-  static constexpr int WARPS = NT * PW;                        // warp nt of group pw: nt + NT*pw
+  // Team layout (more than 8 query columns, FP8/TQ3 pages): TW warps; each decodes the K of
+  // one page of a batch of TW pages for all NT n-tiles and shares its probabilities through
+  // shared memory, then every warp multiplies the whole batch by the V of its own GW channel
+  // groups.  Otherwise (one n-tile, or the BF16 control) warp nt of group pw takes n-tile nt of
+  // the group's pages.
+  static constexpr bool TEAM = NT > 1 && K != kKindBf16;
+  static constexpr int TW = D == 64 ? 2 : 4;
+  static constexpr int PW = TEAM ? 1 : (NT == 1 ? 4 : (NT == 2 ? 2 : 1));  // page-parallel groups
+  static constexpr int WARPS = TEAM ? TW : NT * PW;  // warp nt of group pw: nt + NT*pw
   static constexpr int THREADS = 32 * WARPS;
   static constexpr int FP8_STAGE = 32 * D + 16;
   static constexpr int TQ3_STAGE = 14 * D;
@@ -76,8 +83,15 @@ struct Cfg {
   static constexpr int RING_FP8 = (K == kKindFp8 || K == kKindFused) ? FP8_NST * FP8_STAGE : 0;
   static constexpr int RING_TQ3 = (K == kKindTq3 || K == kKindFused) ? TQ3_NST * TQ3_STAGE
                                   : (K == kKindBf16 ? BF16_NST * BF16_STAGE : 0);
-  // end-of-unit combine: (m, l) and acc of every warp
-  static constexpr int COMBINE = PW * NT * 8 * (D + 2) * 4;
+  // end-of-unit combine: (m, l) and acc of every warp (team: of every n-tile, then the warps'
+  // denominators)
+  static constexpr int COMBINE = TEAM ? NT * 8 * (D + 2) * 4 + TW * NT * 8 * 4
+                                      : PW * NT * 8 * (D + 2) * 4;
+  // team exchange, two batches: P fragments [batch][page][n-tile][lane] (uint2), then the
+  // page references and sums [batch][page][n-tile][column] (float2)
+  static constexpr int XCH_P = TEAM ? 2 * TW * NT * 32 * 8 : 0;
+  static constexpr int XCH = TEAM ? XCH_P + 2 * TW * NT * 8 * 4 : 0;
+
   static constexpr int RING = RING_FP8 > RING_TQ3 ? (RING_FP8 > COMBINE ? RING_FP8 : COMBINE)
                                                   : (RING_TQ3 > COMBINE ? RING_TQ3 : COMBINE);
   // header: full[16] mbarriers | release counters | fills issued | misc | page list |
@@ -89,21 +103,26 @@ struct Cfg {
   static constexpr int OFF_QF = (OFF_LIST + kMaxPagesPerUnit * 8 + 127) / 128 * 128;
   static constexpr int QF = NT * D * 16;
   static constexpr int OFF_CORR = OFF_QF + QF;
-  static constexpr int OFF_RING = (OFF_CORR + NT * (D / 32) * 32 + 127) / 128 * 128;
+  static constexpr int OFF_XCH = (OFF_CORR + NT * (D / 32) * 32 + 127) / 128 * 128;
+  static constexpr int OFF_RING = (OFF_XCH + XCH + 127) / 128 * 128;
   static constexpr int SMEM = OFF_RING + RING;
   // CTAs per SM the launch bounds aim at (registers: 65536 / (THREADS * that))
   // (an FP8 CTA fits beside three TQ3 CTAs: both kernels at 4 for D 256)
-  static constexpr int MINB = K == kKindBf16 ? 1 : D == 256 ? (K == kKindFused ? 3 : 4) : (D == 128 ? 5 : 6);
+  static constexpr int MINB = TEAM ? (D == 64 ? 8 : (D == 256 ? 3 : 4))
+                             : K == kKindBf16 ? 1 : D == 256 ? (K == kKindFused ? 3 : 4)
+                                                             : (D == 128 ? 5 : 6);
 };
 
 struct Smem {
   uint64_t* full;   // [stage]: the stage's page landed (arrive + bulk-copy bytes)
-  int32_t* cnt;     // [stage]: warps done with the stage's page (several n-tiles per page)
+  int32_t* cnt;     // [stage]: warps done with the stage's page (several n-tiles per page);
+                    // team layout: then [2][TW] flags of pages that raised a reference
   int32_t* fills;   // [stage]: copies issued into the stage
   int32_t* misc;    // [0] page count, [1] abort flag, [4..7] logit scales per n-tile
   int2* list;       // {slot, logical page} of the unit's pages
   uint4* qf;        // Q fragments [NT][D/32][32 lanes]
   float2* corr;     // TQ3 K corrections [NT][D/32][4 column pairs]
+  uint8_t* xch;     // team exchange (P fragments, page references and sums)
   uint8_t* ring;
 };
 
@@ -118,6 +137,7 @@ __device__ __forceinline__ Smem carve(uint8_t* base) {
   s.list = reinterpret_cast<int2*>(base + C::OFF_LIST);
   s.qf = reinterpret_cast<uint4*>(base + C::OFF_QF);
   s.corr = reinterpret_cast<float2*>(base + C::OFF_CORR);
+  s.xch = base + C::OFF_XCH;
   s.ring = base + C::OFF_RING;
   return s;
 }
@@ -172,6 +192,12 @@ __device__ __forceinline__ void softmax_k(KState& st, float (&x)[4], float (&pr)
   pr[3] = fast_exp2(x[3] - r1);
   st.l[0] += pr[0] + pr[2];
   st.l[1] += pr[1] + pr[3];
+}
+
+// 2^d for an integer-valued d <= 127, built from its exponent bits (exact); 0 for d < -126,
+// -inf included.
+__device__ __forceinline__ float pow2i(float d) {
+  return d < -126.f ? 0.f : __int_as_float((static_cast<int>(d) + 127) << 23);
 }
 
 __device__ __forceinline__ void mask_page(float (&x)[4], int tok0, int r, int lim0, int lim1) {
@@ -367,6 +393,176 @@ __device__ __forceinline__ void fp8_pv(VState<D>& st, const uint8_t* pg, int lan
     for (int e = 0; e < 4; ++e) {
       st.acc[2 * g][e] = fmaf(sv, t0[e], st.acc[2 * g][e]);
       st.acc[2 * g + 1][e] = fmaf(sv, t1[e], st.acc[2 * g + 1][e]);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ team kernels: NT n-tiles
+// The same page arithmetic with the codes of a page decoded once for all NT n-tiles of the KV
+// head (more than 8 query columns).  Q fragments and TQ3 corrections of n-tile nt sit at
+// qf + nt*(D/32)*32 and corr + nt*(D/32)*4.
+template <int D, int NT>
+__device__ __forceinline__ void tq3_logits_nt(const uint8_t* pg, const uint4* qf,
+                                              const float2* corr, int lane, int kw, int ks,
+                                              float (&x)[NT][4]) {
+  constexpr int G = D / 32;
+  const int r = lane >> 2, c = lane & 3;
+  const uint8_t* krec = pg;
+  const __half* kscale = reinterpret_cast<const __half*>(pg + G * 16 * 12);
+  uint32_t kMask = 0x00380380u, kMagic = 0x58004800u;
+  opaque(kMask, kMagic);
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) x[nt][0] = x[nt][1] = x[nt][2] = x[nt][3] = 0.f;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const uint32_t* ra = reinterpret_cast<const uint32_t*>(krec + 12 * (16 * g + r));
+    const uint32_t* rb = ra + 24;  // token r + 8
+    const uint32_t xa = __funnelshift_r(ra[kw], ra[kw + 1], ks);
+    const uint32_t xb = __funnelshift_r(rb[kw], rb[kw + 1], ks);
+    const uint32_t a0 = and_or(xa, kMask, kMagic), b0 = and_or(xb, kMask, kMagic);
+    const uint32_t a1 = and_or(xa >> 3, kMask, kMagic), b1 = and_or(xb >> 3, kMask, kMagic);
+    const uint32_t a2 = and_or(xa >> 6, kMask, kMagic), b2 = and_or(xb >> 6, kMask, kMagic);
+    const uint32_t a3 = and_or(xa >> 9, kMask, kMagic), b3 = and_or(xb >> 9, kMask, kMagic);
+    const float sa = __half2float(kscale[16 * g + r]);
+    const float sb = __half2float(kscale[16 * g + r + 8]);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const uint4 qb = qf[nt * G * 32 + 32 * g + lane];
+      const float2 cr = corr[nt * G * 4 + 4 * g + c];
+      float cg[4];
+      mma_f16_16816(cg, a0, b0, a1, b1, qb.x, qb.y, {cr.x, cr.y, cr.x, cr.y});
+      mma_f16_16816(cg, a2, b2, a3, b3, qb.z, qb.w, cg);
+      x[nt][0] = fmaf(sa, cg[0], x[nt][0]);
+      x[nt][1] = fmaf(sa, cg[1], x[nt][1]);
+      x[nt][2] = fmaf(sb, cg[2], x[nt][2]);
+      x[nt][3] = fmaf(sb, cg[3], x[nt][3]);
+    }
+  }
+}
+
+template <int D, int NT>
+__device__ __forceinline__ void fp8_logits_nt(const uint8_t* pg, const uint4* qf, int lane,
+                                              float (&x)[NT][4]) {
+  const int r = lane >> 2, c = lane & 3;
+  const float sk = *reinterpret_cast<const float*>(pg + 32 * D);
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) x[nt][0] = x[nt][1] = x[nt][2] = x[nt][3] = 0.f;
+#pragma unroll
+  for (int j = 0; j < D / 64; ++j) {
+    const uint4 wa = *reinterpret_cast<const uint4*>(pg + r * D + 64 * j + 16 * c);
+    const uint4 wb = *reinterpret_cast<const uint4*>(pg + (r + 8) * D + 64 * j + 16 * c);
+    const uint32_t va[4] = {wa.x, wa.y, wa.z, wa.w};
+    const uint32_t vb[4] = {wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t a0 = e4m3x2_to_f16x2(va[i]), a1 = e4m3x2_to_f16x2(vb[i]);
+      const uint32_t a2 = e4m3x2_to_f16x2(va[i] >> 16), a3 = e4m3x2_to_f16x2(vb[i] >> 16);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const uint4 q = qf[nt * (D / 32) * 32 + 32 * (2 * j + (i >> 1)) + lane];
+        mma_f16_16816(x[nt], a0, a1, a2, a3, (i & 1) ? q.z : q.x, (i & 1) ? q.w : q.y, x[nt]);
+      }
+    }
+  }
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x[nt][e] *= sk;
+}
+
+// P.V of the channel groups [g0, g0 + GW) for all n-tiles: acc[2 lg + j][nt] is channel tile
+// 2 (g0 + lg) + j (channel order as for one n-tile); pb[nt] the n-tile's P^T fragments.
+template <int D, int NT, int GW, bool WIDE>
+__device__ __forceinline__ void tq3_pv_nt(float (&acc)[2 * GW][NT][4], const uint8_t* pg,
+                                          int lane, int vw, int vs1, int g0,
+                                          const uint2 (&pb)[NT]) {
+  constexpr int G = D / 32;
+  const int c = lane & 3;
+  const uint8_t* vrec = pg + G * 16 * 14;
+  const __half* vscale = reinterpret_cast<const __half*>(vrec + G * 16 * 12);
+  uint32_t m0 = 0x000E000Eu, g0m = 0x60006000u, m1 = 0x00700070u, g1 = 0x54005400u;
+  uint32_t m2 = 0x03800380u, g2 = 0x48004800u;
+  opaque(m0, g0m, m1, g1, m2, g2);
+  const uint32_t s0 = f16x2_const(515.5f, 515.5f), s1 = f16x2_const(67.5f, 67.5f);
+  const uint32_t s2 = f16x2_const(11.5f, 11.5f);
+#pragma unroll
+  for (int lg = 0; lg < GW; ++lg) {
+    const int g = g0 + lg;
+    const uint32_t* rc = reinterpret_cast<const uint32_t*>(vrec + 12 * (16 * g + 2 * c));
+    const uint32_t f0 = __funnelshift_r(rc[vw], rc[vw + 1], vs1);        // token 2c
+    const uint32_t f1 = __funnelshift_r(rc[vw + 3], rc[vw + 4], vs1);    // token 2c+1
+    const uint32_t f8 = __funnelshift_r(rc[vw + 24], rc[vw + 25], vs1);  // token 2c+8
+    const uint32_t f9 = __funnelshift_r(rc[vw + 27], rc[vw + 28], vs1);  // token 2c+9
+    const uint32_t z01 = __byte_perm(f0, f1, 0x5410);
+    const uint32_t z89 = __byte_perm(f8, f9, 0x5410);
+    const uint32_t a0 = hsub2_u32(and_or(z01, m0, g0m), s0), b0 = hsub2_u32(and_or(z89, m0, g0m), s0);
+    const uint32_t a1 = hsub2_u32(and_or(z01, m1, g1), s1), b1 = hsub2_u32(and_or(z89, m1, g1), s1);
+    const uint32_t a2 = hsub2_u32(and_or(z01, m2, g2), s2), b2 = hsub2_u32(and_or(z89, m2, g2), s2);
+    const uint32_t a3 = hsub2_u32(and_or(z01 >> 3, m2, g2), s2);
+    const uint32_t b3 = hsub2_u32(and_or(z89 >> 3, m2, g2), s2);
+    uint32_t sv0 = *reinterpret_cast<const uint32_t*>(vscale + 16 * g + 2 * c);
+    uint32_t sv8 = *reinterpret_cast<const uint32_t*>(vscale + 16 * g + 2 * c + 8);
+    if constexpr (!WIDE) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const uint32_t q0 = hmul2_u32(pb[nt].x, sv0), q1 = hmul2_u32(pb[nt].y, sv8);
+        mma_f16_16816(acc[2 * lg][nt], a0, a1, b0, b1, q0, q1, acc[2 * lg][nt]);
+        mma_f16_16816(acc[2 * lg + 1][nt], a2, a3, b2, b3, q0, q1, acc[2 * lg + 1][nt]);
+      }
+    } else {
+      uint32_t m = hmax2_u32(sv0, sv8);
+      m = hmax2_u32(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = hmax2_u32(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      const int e = max(static_cast<int>(max(m & 0xffffu, m >> 16) >> 10), 1);
+      const uint32_t down = static_cast<uint32_t>(31 - e) * 0x04000400u;  // f16x2 2^(16-e)
+      const float up = __int_as_float((e + 111) << 23);                   // fp32 2^(e-16)
+      sv0 = hmul2_u32(sv0, down);
+      sv8 = hmul2_u32(sv8, down);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const uint32_t q0 = hmul2_u32(pb[nt].x, sv0), q1 = hmul2_u32(pb[nt].y, sv8);
+        float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_f16_16816(t0, a0, a1, b0, b1, q0, q1, t0);
+        mma_f16_16816(t1, a2, a3, b2, b3, q0, q1, t1);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          acc[2 * lg][nt][j] = fmaf(up, t0[j], acc[2 * lg][nt][j]);
+          acc[2 * lg + 1][nt][j] = fmaf(up, t1[j], acc[2 * lg + 1][nt][j]);
+        }
+      }
+    }
+  }
+}
+
+template <int D, int NT, int GW>
+__device__ __forceinline__ void fp8_pv_nt(float (&acc)[2 * GW][NT][4], const uint8_t* pg,
+                                          int lane, int g0, const uint2 (&pb)[NT]) {
+  const int r = lane >> 2, c = lane & 3;
+  const float sv = *reinterpret_cast<const float*>(pg + 32 * D + 4);
+  const uint8_t* vrows = pg + 16 * D;
+#pragma unroll
+  for (int lg = 0; lg < GW; ++lg) {
+    const int off = 32 * (g0 + lg) + 4 * r;
+    const uint32_t w0 = *reinterpret_cast<const uint32_t*>(vrows + (2 * c) * D + off);
+    const uint32_t w1 = *reinterpret_cast<const uint32_t*>(vrows + (2 * c + 1) * D + off);
+    const uint32_t w8 = *reinterpret_cast<const uint32_t*>(vrows + (2 * c + 8) * D + off);
+    const uint32_t w9 = *reinterpret_cast<const uint32_t*>(vrows + (2 * c + 9) * D + off);
+    const uint32_t lo01 = __byte_perm(w0, w1, 0x5140), hi01 = __byte_perm(w0, w1, 0x7362);
+    const uint32_t lo89 = __byte_perm(w8, w9, 0x5140), hi89 = __byte_perm(w8, w9, 0x7362);
+    const uint32_t a0 = e4m3x2_to_f16x2(lo01), a1 = e4m3x2_to_f16x2(lo01 >> 16);
+    const uint32_t a2 = e4m3x2_to_f16x2(lo89), a3 = e4m3x2_to_f16x2(lo89 >> 16);
+    const uint32_t b0 = e4m3x2_to_f16x2(hi01), b1 = e4m3x2_to_f16x2(hi01 >> 16);
+    const uint32_t b2 = e4m3x2_to_f16x2(hi89), b3 = e4m3x2_to_f16x2(hi89 >> 16);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
+      mma_f16_16816(t0, a0, a1, a2, a3, pb[nt].x, pb[nt].y, t0);
+      mma_f16_16816(t1, b0, b1, b2, b3, pb[nt].x, pb[nt].y, t1);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc[2 * lg][nt][e] = fmaf(sv, t0[e], acc[2 * lg][nt][e]);
+        acc[2 * lg + 1][nt][e] = fmaf(sv, t1[e], acc[2 * lg + 1][nt][e]);
+      }
     }
   }
 }
@@ -791,6 +987,315 @@ __device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDes
   }
 }
 
+// Team layout (more than 8 query columns; FP8 or TQ3 pages).  The unit's pages are taken in
+// batches of TW: warp w decodes the K of page b + w once for all NT n-tiles, computes the
+// page's logits and probabilities against the common reference of each column (identical on
+// every warp), and publishes their P^T fragments; after one team barrier every warp multiplies
+// the whole batch by the V of its own channel groups.  Every page's codes are decoded once.
+// The reference is raised lazily, as on the one-tile path: a page whose column exceeds it by
+// more than 8 uses its own reference (the column maximum rounded up to an integer) and flags
+// the batch; after the barrier every warp raises the common reference to the batch's largest
+// and scales that batch's P and its own accumulators by exact powers of two.  Probabilities fed
+// to the MMAs stay <= 2^8.  Each warp sums the denominators of its own K pages; the sums meet
+// in the combine.
+template <int D, int NT, int K, int F>
+__device__ void run_unit_team(const DecodeParams& p, const SeqDesc& sd, const UnitDesc& u, int h,
+                              Smem sm) {
+  using C = Cfg<D, NT, K>;
+  using PG = Page<D, NT, K, F>;
+  constexpr int TW = C::TW, NST = PG::NST, STAGE = PG::STAGE;
+  constexpr int GW = (D / 32) / TW;  // channel groups of 32 per warp
+  static_assert(NST % TW == 0 && NST >= 2 * TW, "two batches in flight");
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = lane >> 2, c = lane & 3;
+  const uint8_t* slab = F == kTq3 ? p.tq3_slab : p.fp8_slab;
+  const int64_t slot_bytes = F == kTq3 ? p.tq3_slot_bytes : p.fp8_slot_bytes;
+
+  if (warp == TW - 1) {
+    if (lane == 0) {
+      for (int s = 0; s < NST; ++s) {
+        mbar_init(&sm.full[s], 1);
+        sm.cnt[s] = 0;
+        sm.fills[s] = 0;
+      }
+      sm.misc[1] = 0;
+      mbar_fence_init();
+    }
+    __syncwarp();
+    const int32_t* row = p.tables + static_cast<int64_t>(sd.row) * p.max_pages;
+    const int n = scan_range(p, row, u.first, u.last, F, lane, sm.list);
+    __syncwarp();
+    if (lane == 0) sm.misc[0] = n;
+    for (int i = 0; i < min(n, NST); ++i) fill_stage<PG, F>(sm, slab, slot_bytes, h, i, lane);
+  }
+  for (int nt = warp; nt < NT; nt += TW) {
+    const float ls = build_q<D, F == kFp8>(p, sd, h, nt, lane, sm.qf + nt * (D / 32) * 32,
+                                           reinterpret_cast<float*>(sm.corr + nt * (D / 32) * 4));
+    if (lane == 0) reinterpret_cast<float*>(sm.misc)[4 + nt] = ls;
+  }
+  __syncthreads();
+  const int count = sm.misc[0];
+
+  const float* lsc = reinterpret_cast<const float*>(sm.misc) + 4;  // logit scale per n-tile
+  const int min_lim = sd.ctx - p.q_len;
+  const int kbit = 24 * c - 7, vbit = 12 * r - 1;
+  const int kw = kbit >= 0 ? kbit >> 5 : -1, ks5 = kbit & 31;
+  const int vw = vbit >= 0 ? vbit >> 5 : -1, vs1 = vbit & 31;
+  const int g0 = warp * GW;
+  uint2* xp = reinterpret_cast<uint2*>(sm.xch);              // [2][TW][NT][32] P^T fragments
+  float* xr = reinterpret_cast<float*>(sm.xch + C::XCH_P);   // [2][TW][NT][8] page references
+  int32_t* xf = sm.cnt + NST;                                // [2][TW] page raised a reference
+
+  float acc[2 * GW][NT][4];
+#pragma unroll
+  for (int j = 0; j < 2 * GW; ++j)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) acc[j][nt][0] = acc[j][nt][1] = acc[j][nt][2] = acc[j][nt][3] = 0.f;
+  // common references (log2 units, integers once set) of columns 2c, 2c+1 and r of every
+  // n-tile; this lane's share of the denominators of its K pages (columns 2c, 2c+1)
+  float mc[NT][2], mr[NT], lk[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    mc[nt][0] = mc[nt][1] = mr[nt] = -INFINITY;
+    lk[nt][0] = lk[nt][1] = 0.f;
+  }
+
+  for (int b = 0; b < count; b += TW) {
+    const int par = (b / TW) & 1;
+    const int nb = min(TW, count - b);
+    // K: this warp's page of the batch
+    bool ok = true, raised = false;
+    float lp[NT][2];  // the page's denominator shares, relative to its references
+    float rf[NT][2];  // the page's references of columns 2c, 2c+1
+    const int ik = b + warp;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      lp[nt][0] = lp[nt][1] = 0.f;
+      rf[nt][0] = mc[nt][0];
+      rf[nt][1] = mc[nt][1];
+    }
+    if (ik < count) {
+      const int s = ik % NST;
+      ok = mbar_wait_warp(&sm.full[s], (ik / NST) & 1);
+      if (ok) {
+        const uint8_t* pg = sm.ring + s * STAGE;
+        float x[NT][4];
+        if constexpr (F == kFp8)
+          fp8_logits_nt<D, NT>(pg, sm.qf, lane, x);
+        else
+          tq3_logits_nt<D, NT>(pg, sm.qf, sm.corr, lane, kw, ks5, x);
+        const int tok0 = 16 * sm.list[ik].y;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const float ls = lsc[nt];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) x[nt][j] *= ls;
+          if (tok0 + 15 > min_lim) {
+            // causal limits of columns 2c, 2c+1 (padding columns see the whole context)
+            const int n0 = 8 * nt + 2 * c, n1 = n0 + 1;
+            mask_page(x[nt], tok0, r, n0 < p.NC ? min_lim + n0 / p.g : sd.ctx - 1,
+                      n1 < p.NC ? min_lim + n1 / p.g : sd.ctx - 1);
+          }
+          float m0 = fmaxf(x[nt][0], x[nt][2]), m1 = fmaxf(x[nt][1], x[nt][3]);
+          const bool need = m0 > mc[nt][0] + kLazyRescale || m1 > mc[nt][1] + kLazyRescale;
+          if (__any_sync(0xffffffffu, need)) {
+            // this page raises: its own references (column maximum rounded up) where needed
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+              m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
+              m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+            }
+            if (m0 > mc[nt][0] + kLazyRescale) rf[nt][0] = ceilf(m0);
+            if (m1 > mc[nt][1] + kLazyRescale) rf[nt][1] = ceilf(m1);
+            raised = true;
+          }
+          const float r0 = rf[nt][0] == -INFINITY ? 0.f : rf[nt][0];
+          const float r1 = rf[nt][1] == -INFINITY ? 0.f : rf[nt][1];
+          float pr[4];
+          pr[0] = fast_exp2(x[nt][0] - r0);
+          pr[1] = fast_exp2(x[nt][1] - r1);
+          pr[2] = fast_exp2(x[nt][2] - r0);
+          pr[3] = fast_exp2(x[nt][3] - r1);
+          lp[nt][0] = pr[0] + pr[2];
+          lp[nt][1] = pr[1] + pr[3];
+          xp[((par * TW + warp) * NT + nt) * 32 + lane] =
+              make_uint2(movmatrix_trans(pack_f16x2(pr[0], pr[1])),
+                         movmatrix_trans(pack_f16x2(pr[2], pr[3])));
+        }
+        if (raised) {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+            if (r == 0) {
+              xr[((par * TW + warp) * NT + nt) * 8 + 2 * c] = rf[nt][0];
+              xr[((par * TW + warp) * NT + nt) * 8 + 2 * c + 1] = rf[nt][1];
+            }
+        }
+      }
+    }
+    if (lane == 0) xf[par * TW + warp] = raised ? 1 : 0;
+    // the batch's probabilities are published; every warp of the team stops together on a
+    // failed wait
+    if (!barrier_and(1, 32 * TW, ok)) {
+      if (lane == 0) flag_status(p.status, kStatusTimeout);
+      break;
+    }
+    int any_raised = 0;
+    for (int q = 0; q < nb; ++q) any_raised |= xf[par * TW + q];
+    // P scale of each page of a raising batch (column r) and the page's own sums
+    float fq[TW][NT];
+    if (any_raised) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        float n0 = mc[nt][0], n1 = mc[nt][1], nr = mr[nt];
+        for (int q = 0; q < nb; ++q) {
+          if (!xf[par * TW + q]) continue;
+          const float* rq = xr + ((par * TW + q) * NT + nt) * 8;
+          n0 = fmaxf(n0, rq[2 * c]);
+          n1 = fmaxf(n1, rq[2 * c + 1]);
+          nr = fmaxf(nr, rq[r]);
+        }
+        const float a0 = pow2i(mc[nt][0] - n0), a1 = pow2i(mc[nt][1] - n1);  // 0 from -inf
+        lk[nt][0] *= a0;
+        lk[nt][1] *= a1;
+#pragma unroll
+        for (int j = 0; j < 2 * GW; ++j) {
+          acc[j][nt][0] *= a0;
+          acc[j][nt][2] *= a0;
+          acc[j][nt][1] *= a1;
+          acc[j][nt][3] *= a1;
+        }
+#pragma unroll
+        for (int q = 0; q < TW; ++q) {
+          const float rq = q < nb && xf[par * TW + q] ? xr[((par * TW + q) * NT + nt) * 8 + r]
+                                                       : mr[nt];
+          fq[q][nt] = rq == -INFINITY ? 0.f : pow2i(rq - nr);
+        }
+        // this warp's page: its sums move to the new references
+        lk[nt][0] = fmaf(lp[nt][0], rf[nt][0] == -INFINITY ? 0.f : pow2i(rf[nt][0] - n0), lk[nt][0]);
+        lk[nt][1] = fmaf(lp[nt][1], rf[nt][1] == -INFINITY ? 0.f : pow2i(rf[nt][1] - n1), lk[nt][1]);
+        mc[nt][0] = n0;
+        mc[nt][1] = n1;
+        mr[nt] = nr;
+      }
+    } else {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        lk[nt][0] += lp[nt][0];
+        lk[nt][1] += lp[nt][1];
+      }
+    }
+    // V: every page of the batch, this warp's channel groups
+    for (int q = 0; q < nb; ++q) {
+      const int iv = b + q, s = iv % NST;
+      // landed (its K warp waited for it before the barrier): returns at once
+      if (mbar_wait_warp(&sm.full[s], (iv / NST) & 1)) {
+        const uint8_t* pg = sm.ring + s * STAGE;
+        uint2 pb[NT];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          pb[nt] = xp[((par * TW + q) * NT + nt) * 32 + lane];
+          if (any_raised) {
+            float f = 0.f;
+#pragma unroll
+            for (int qq = 0; qq < TW; ++qq) f = qq == q ? fq[qq][nt] : f;
+            const uint32_t f2 = pack_f16x2(f, f);  // a power of two <= 1 (or 0)
+            pb[nt].x = hmul2_u32(pb[nt].x, f2);
+            pb[nt].y = hmul2_u32(pb[nt].y, f2);
+          }
+        }
+        if constexpr (F == kFp8) {
+          fp8_pv_nt<D, NT, GW>(acc, pg, lane, g0, pb);
+        } else {
+          const uint32_t vmax = tq3_v_scale_max<D>(pg, lane);
+          if (vmax >= kVScaleLo && vmax <= kVScaleHi)
+            tq3_pv_nt<D, NT, GW, false>(acc, pg, lane, vw, vs1, g0, pb);
+          else
+            tq3_pv_nt<D, NT, GW, true>(acc, pg, lane, vw, vs1, g0, pb);
+        }
+      } else if (lane == 0) {
+        flag_status(p.status, kStatusTimeout);
+      }
+      // release the stage: the last of the team's warps done with it refills it
+      if (iv + NST < count) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        bool last = false;
+        if (lane == 0) {
+          __threadfence_block();
+          last = atomicAdd(&sm.cnt[s], 1) == TW - 1;
+          if (last) sm.cnt[s] = 0;
+          __threadfence_block();
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) fill_stage<PG, F>(sm, slab, slot_bytes, h, iv + NST, lane);
+      }
+    }
+  }
+  // drain (bounded) after a failed wait: the last copy issued into every stage lands before the
+  // ring is reused
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      const int f = *reinterpret_cast<volatile int32_t*>(&sm.fills[s]);
+      if (f > 0) mbar_wait(&sm.full[s], (f - 1) & 1, 100000000ull);
+    }
+  }
+  __syncthreads();
+
+  // combine: per n-tile, (m, l) of its 8 columns and acc [8][D] (every warp its channels); the
+  // denominators are summed over the lanes of a column and then over the warps
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      lk[nt][0] += __shfl_xor_sync(0xffffffffu, lk[nt][0], o);
+      lk[nt][1] += __shfl_xor_sync(0xffffffffu, lk[nt][1], o);
+    }
+  float* cmb = reinterpret_cast<float*>(sm.ring);
+  constexpr int REGION = 8 * (D + 2);
+  float* lsum = cmb + NT * REGION;  // [TW][NT][8]
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    float* reg = cmb + nt * REGION;
+    if (r == 0) {
+      lsum[(warp * NT + nt) * 8 + 2 * c] = lk[nt][0];
+      lsum[(warp * NT + nt) * 8 + 2 * c + 1] = lk[nt][1];
+      if (warp == 0) {
+        reg[2 * (2 * c)] = mc[nt][0];
+        reg[2 * (2 * c + 1)] = mc[nt][1];
+      }
+    }
+    float* ra = reg + 16;
+#pragma unroll
+    for (int j = 0; j < 2 * GW; ++j) {
+      const int mt = 2 * g0 + j;
+      const int ch0 = 32 * (mt >> 1) + 4 * r + 2 * (mt & 1), ch1 = ch0 + 1;
+      ra[(2 * c) * D + ch0] = acc[j][nt][0];
+      ra[(2 * c + 1) * D + ch0] = acc[j][nt][1];
+      ra[(2 * c) * D + ch1] = acc[j][nt][2];
+      ra[(2 * c + 1) * D + ch1] = acc[j][nt][3];
+    }
+  }
+  __syncthreads();
+  const int part = sd.part0 + u.part;
+  for (int q = threadIdx.x; q < NT * 8 * (D / 4); q += C::THREADS) {
+    const int nt = q / (8 * (D / 4)), rem = q % (8 * (D / 4));
+    const int col = rem / (D / 4), ch = 4 * (rem % (D / 4));
+    const int n = 8 * nt + col;
+    if (n >= p.NC) continue;
+    const float* reg = cmb + nt * REGION;
+    const int64_t base = (static_cast<int64_t>(part) * p.Hkv + h) * p.NC + n;
+    if (ch == 0) {
+      float L = 0.f;
+      for (int w = 0; w < TW; ++w) L += lsum[(w * NT + nt) * 8 + col];
+      p.part_ml[2 * base] = reg[2 * col];
+      p.part_ml[2 * base + 1] = L;
+    }
+    *reinterpret_cast<float4*>(p.part_acc + base * D + ch) =
+        *reinterpret_cast<const float4*>(reg + 16 + col * D + ch);
+  }
+}
+
 // Merge of the partial states of one (sequence, KV head, query column): the globally
 // normalised combination M = max m, L = sum l 2^(m-M), O = sum acc 2^(m-M) / L.  One pass: a
 // thread owns 4 channels of a subset of the partials (every nsub-th one) and keeps a running
@@ -889,7 +1394,19 @@ __global__ void __launch_bounds__(Cfg<D, NT, K>::THREADS, Cfg<D, NT, K>::MINB)
   const int h = blockIdx.x % p.Hkv;
   const UnitDesc& u = p.unit[(K == kKindTq3 ? p.n_fp8 : 0) + blockIdx.x / p.Hkv];
   const SeqDesc& sd = p.seq[u.seq];
-  if constexpr (K == kKindFp8) {
+  if constexpr (Cfg<D, NT, K>::TEAM) {
+    if constexpr (K == kKindFp8) {
+      run_unit_team<D, NT, K, kFp8>(p, sd, u, h, sm);
+    } else if constexpr (K == kKindTq3) {
+      run_unit_team<D, NT, K, kTq3>(p, sd, u, h, sm);
+      pdl_wait();  // as below: the merge then sees both grids' partial states
+    } else {
+      if (u.fmt == kFp8)
+        run_unit_team<D, NT, K, kFp8>(p, sd, u, h, sm);
+      else
+        run_unit_team<D, NT, K, kTq3>(p, sd, u, h, sm);
+    }
+  } else if constexpr (K == kKindFp8) {
     run_unit<D, NT, K, kFp8>(p, sd, u, h, sm);
   } else if constexpr (K == kKindTq3) {
     run_unit<D, NT, K, kTq3>(p, sd, u, h, sm);

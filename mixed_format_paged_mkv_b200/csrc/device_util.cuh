@@ -89,6 +89,21 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity) {
   return __all_sync(0xffffffffu, ok);
 }
 
+// Barrier among `threads` threads (a multiple of 32) of the CTA on hardware barrier `id` (1-15;
+// 0 is __syncthreads) that also returns whether `pred` held on every participating thread.
+__device__ __forceinline__ bool barrier_and(int id, int threads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(threads)
+      : "memory");
+  return r != 0;
+}
+
 // Hide the values of bit-mask constants from the compiler so that it keeps them in registers
 // instead of re-materialising an immediate at every use (a LOP3 has one immediate slot, so
 // `(x & mask) | magic` with two literal constants costs an extra move per use).

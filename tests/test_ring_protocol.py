@@ -70,3 +70,91 @@ def test_kernel_rings_never_wait_ambiguously(nst, pw):
 def test_ring_shape_that_violates_the_rule_is_detected():
     # six stages shared by four warps: some stage is consumed by two different warps
     assert any(replay(45, 6, 4, seed) for seed in range(200))
+
+
+def replay_team(count, nst, tw, seed):
+    """Team layout (more than 8 query columns): pages go in batches of tw; warp w first waits
+    for page b + w of batch b (its K page), then all warps meet at the batch barrier, then every
+    warp waits for and consumes every page of the batch (V); a stage is refilled with page
+    i + nst once all tw warps released page i.  Returns True if some wait started for fill f of
+    a stage whose fill f-1 had not completed."""
+    rng = random.Random(seed)
+    completed = [0] * nst
+    releases = [0] * count
+    issued = 0
+    in_flight = []
+    batch = [0] * tw           # first page of each warp's current batch
+    step = ["k"] * tw          # "k": K page, "bar": at the barrier, int q: V page b + q
+    waiting = [None] * tw
+    ambiguous = False
+
+    def start_wait(w, i):
+        nonlocal ambiguous
+        if waiting[w] != i:
+            waiting[w] = i
+            if completed[i % nst] < i // nst:
+                ambiguous = True
+        return completed[i % nst] > i // nst
+
+    while any(b < count for b in batch):
+        moves = []
+        if issued < count and (issued < nst or releases[issued - nst] == tw):
+            moves.append("issue")
+        if in_flight:
+            moves.append("land")
+        arrived = [w for w in range(tw) if step[w] == "bar"]
+        if len(arrived) == tw:
+            moves.append("barrier")
+        ready = []                 # warps whose wait would end (or who have no K page)
+        for w in range(tw):
+            if batch[w] < count and step[w] != "bar":
+                moves.append(w)
+                i = batch[w] + (w if step[w] == "k" else step[w])
+                if (step[w] == "k" and i >= count) or completed[i % nst] > i // nst:
+                    ready.append(w)
+        if not (ready or "issue" in moves or "land" in moves or "barrier" in moves):
+            raise AssertionError("deadlock")
+        m = rng.choice(moves)
+        if m == "issue":
+            in_flight.append(issued)
+            issued += 1
+        elif m == "land":
+            i = in_flight.pop(rng.randrange(len(in_flight)))
+            completed[i % nst] += 1
+        elif m == "barrier":
+            step = [0] * tw
+        else:
+            w, b = m, batch[m]
+            if step[w] == "k":
+                i = b + w
+                if i >= count or start_wait(w, i):
+                    waiting[w] = None
+                    step[w] = "bar"
+            else:
+                i = b + step[w]
+                if start_wait(w, i):
+                    waiting[w] = None
+                    releases[i] += 1
+                    step[w] += 1
+                    if step[w] == min(tw, count - b):
+                        batch[w] += tw
+                        step[w] = "k"
+    return ambiguous
+
+
+@pytest.mark.parametrize("nst,tw", [(8, 4), (8, 2)])   # the kernel's team rings
+def test_team_ring_never_waits_ambiguously(nst, tw):
+    for seed in range(60):
+        for count in (1, 3, tw, nst - 1, nst, nst + 3, 3 * nst + 1, 45):
+            assert not replay_team(count, nst, tw, seed), (nst, tw, count, seed)
+
+
+def test_team_ring_needs_a_stage_per_page_of_a_batch():
+    # Every warp consumes every page, so a warp never waits on a fill whose predecessor it has
+    # not consumed itself: any ring of at least tw stages is unambiguous.  Fewer stages than a
+    # batch has pages deadlock (a K page waits for a stage whose page is consumed only after
+    # the barrier that K page gates), and the model says so.
+    assert not any(replay_team(45, 4, 4, seed) for seed in range(100))
+    with pytest.raises(AssertionError, match="deadlock"):
+        for seed in range(20):
+            replay_team(45, 2, 4, seed)
