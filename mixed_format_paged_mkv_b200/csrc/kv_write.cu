@@ -108,26 +108,107 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ App
 // 4 + #{k in 1..3 : x >= k*s}, for x < 0 it is 3 - #{k in 1..3 : |x| > k*s}; comparing the
 // fp32 bit patterns of |x| (less one for negative x, which turns > into >=) with those of k*s
 // (exact products) decides both as integer compares.
-__device__ __forceinline__ void tq3_record(const float (&x)[32], float amax, uint32_t& w0,
-                                           uint32_t& w1, uint32_t& w2, __half& sh) {
-  sh = __float2half_rn(fminf(__fdiv_rn(amax, 3.5f), 65504.f));
-  const float s = __half2float(sh);
-  const int t1 = __float_as_int(s), t2 = __float_as_int(2.f * s), t3 = __float_as_int(3.f * s);
-  uint32_t acc[3] = {0u, 0u, 0u};
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const uint32_t xb = __float_as_uint(x[j]);
-    const int neg = xb > 0x80000000u ? 1 : 0;
-    const int u = static_cast<int>(xb & 0x7fffffffu) - neg;
-    const int cnt = (u >= t1) + (u >= t2) + (u >= t3);
-    const uint32_t q = static_cast<uint32_t>(neg ? 3 - cnt : 4 + cnt);
-    const int bit = 3 * j;  // constant after unrolling
-    acc[bit >> 5] |= q << (bit & 31);
-    if ((bit & 31) > 29) acc[(bit >> 5) + 1] |= q >> (32 - (bit & 31));
-  }
-  w0 = acc[0];
-  w1 = acc[1];
-  w2 = acc[2];
+__device__ __forceinline__ uint32_t tq3_code(float x, int t1, int t2, int t3) {
+  const uint32_t xb = __float_as_uint(x);
+  const int neg = xb > 0x80000000u ? 1 : 0;
+  const int u = static_cast<int>(xb & 0x7fffffffu) - neg;
+  const int cnt = (u >= t1) + (u >= t2) + (u >= t3);
+  return static_cast<uint32_t>(neg ? 3 - cnt : 4 + cnt);
+}
+
+// Places code j (constant after unrolling) at bits 3j..3j+2 of the record words acc[0..2].
+__device__ __forceinline__ void put_code(uint32_t (&acc)[3], int j, uint32_t q) {
+  const int bit = 3 * j;
+  acc[bit >> 5] |= q << (bit & 31);
+  if ((bit & 31) > 29) acc[(bit >> 5) + 1] |= q >> (32 - (bit & 31));
+}
+
+// ------------------------------------------------------------------ codes in the source domain
+// The same threshold counts, taken four FP8 values (or two bf16 values) per 32-bit operation:
+// since x is a monotonic function of the stored value, "x >= theta" is "the stored magnitude is
+// at least the smallest magnitude whose x reaches theta", and those magnitude thresholds are
+// found once per record.  For a lane value (magnitude m in its low 7 or 15 bits, sign on top),
+// with P_k the threshold of x >= k*s (x >= 0) and N_k that of |x| > k*s (x < 0):
+//   count = #{k : m >= (negative ? N_k : P_k)}, q = negative ? 3 - count : 4 + count,
+// where "negative" excludes -0.  Setting bit 7 (15) of the magnitude and subtracting the lane's
+// threshold leaves bit 7 (15) set exactly when m >= threshold, with no borrow between lanes.
+// Since P_1 <= P_2 <= P_3 (and N likewise), count's bits are (ge2, ge1 ^ ge2 ^ ge3), and the
+// code's three bits are (not negative, ge2 ^ negative, ge1 ^ ge2 ^ ge3 ^ negative).
+
+// Replicates the top bit of every byte over the byte (prmt sign-replicate selectors).
+__device__ __forceinline__ uint32_t byte_sign_mask(uint32_t x) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, 0, 0xBA98;" : "=r"(d) : "r"(x));
+  return d;
+}
+// Replicates bit 15 (31) over the low (high) 16-bit half.
+__device__ __forceinline__ uint32_t half_sign_mask(uint32_t x) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, 0, 0xBB99;" : "=r"(d) : "r"(x));
+  return d;
+}
+
+// Codes of four E4M3 values (byte i = value i) as bits 3i..3i+2 of the result.  p_k: P_k in
+// every byte; d_k: P_k ^ N_k in every byte (all thresholds <= 127).
+__device__ __forceinline__ uint32_t tq3_codes_e4m3x4(uint32_t w, uint32_t p1, uint32_t p2,
+                                                     uint32_t p3, uint32_t d1, uint32_t d2,
+                                                     uint32_t d3) {
+  const uint32_t mag = w & 0x7F7F7F7Fu;
+  const uint32_t negb = ((mag + 0x7F7F7F7Fu) & w) & 0x80808080u;  // sign set and m != 0
+  const uint32_t negm = byte_sign_mask(negb);
+  const uint32_t t = w | 0x80808080u;
+  const uint32_t g1 = t - (p1 ^ (d1 & negm));
+  const uint32_t g2 = t - (p2 ^ (d2 & negm));
+  const uint32_t g3 = t - (p3 ^ (d3 & negm));
+  const uint32_t b0 = (g1 ^ g2 ^ g3 ^ negb) & 0x80808080u;
+  const uint32_t b1 = (g2 ^ negb) & 0x80808080u;
+  const uint32_t b2 = ~negb & 0x80808080u;
+  const uint32_t q = (b0 >> 7) | (b1 >> 6) | (b2 >> 5);  // code i in bits 8i..8i+2
+  const uint32_t pairs = q | (q >> 5);                    // codes 0,1 in bits 0-5; 2,3 in 16-21
+  return (pairs & 0x3Fu) | ((pairs >> 10) & 0xFC0u);
+}
+
+// Codes of two bf16 values (low half first) as bits 0..5; p_k, d_k replicated in both halves.
+__device__ __forceinline__ uint32_t tq3_codes_bf16x2(uint32_t w, uint32_t p1, uint32_t p2,
+                                                     uint32_t p3, uint32_t d1, uint32_t d2,
+                                                     uint32_t d3) {
+  const uint32_t mag = w & 0x7FFF7FFFu;
+  const uint32_t negb = ((mag + 0x7FFF7FFFu) & w) & 0x80008000u;
+  const uint32_t negm = half_sign_mask(negb);
+  const uint32_t t = w | 0x80008000u;
+  const uint32_t g1 = t - (p1 ^ (d1 & negm));
+  const uint32_t g2 = t - (p2 ^ (d2 & negm));
+  const uint32_t g3 = t - (p3 ^ (d3 & negm));
+  const uint32_t b0 = (g1 ^ g2 ^ g3 ^ negb) & 0x80008000u;
+  const uint32_t b1 = (g2 ^ negb) & 0x80008000u;
+  const uint32_t b2 = ~negb & 0x80008000u;
+  const uint32_t q = (b0 >> 15) | (b1 >> 14) | (b2 >> 13);  // code i in bits 16i..16i+2
+  return (q & 7u) | ((q >> 13) & 0x38u);
+}
+
+// 96-bit record from eight 12-bit chunks (chunk c = codes 4c..4c+3).
+__device__ __forceinline__ void record_from_chunks12(const uint32_t (&c)[8], uint32_t& w0,
+                                                     uint32_t& w1, uint32_t& w2) {
+  w0 = c[0] | (c[1] << 12) | (c[2] << 24);
+  w1 = (c[2] >> 8) | (c[3] << 4) | (c[4] << 16) | (c[5] << 28);
+  w2 = (c[5] >> 4) | (c[6] << 8) | (c[7] << 20);
+}
+
+// Smallest E4M3 magnitude code m (0..126) with fp32(dec(m) * scale) >= theta, or 127 when none
+// reaches it.  Exact for 2^-100 <= scale < 2^100 (every product of a nonzero code is then a
+// normal float, and consecutive codes differ by more than 1/16 in value, far above the fp32
+// rounding): with m* the largest code whose value is at most theta/scale, the answer is m* or
+// m* + 1, and the code nearest to (an approximation of) theta/scale is m* or m* + 1, so checking
+// it and the code below decides.
+__device__ __forceinline__ uint32_t e4m3_threshold(float theta, float scale, float rscale) {
+  const uint32_t m0 = float_to_e4m3(theta * rscale) & 0x7Fu;  // theta >= 0: RN, at most 126
+  const uint32_t lo = m0 > 0 ? m0 - 1 : 0;
+  const uint32_t h = e4m3x2_to_f16x2(lo | (m0 << 8));
+  const __half2 hh = *reinterpret_cast<const __half2*>(&h);
+  const float flo = __fmul_rn(__low2float(hh), scale), fm0 = __fmul_rn(__high2float(hh), scale);
+  if (m0 > 0 && flo >= theta) return lo;
+  if (fm0 >= theta) return m0;
+  return m0 + 1;
 }
 
 // Stores one record and its scale into a TQ3 page-head area ([G][16] records, then [G][16]
@@ -157,24 +238,55 @@ __global__ void __launch_bounds__(256) demote_kernel(const __grid_constant__ Dem
   const uint4* c4 = reinterpret_cast<const uint4*>(src + which * kPageTokens * D + t * D + 32 * grp);
   const uint4 ca = c4[0], cb = c4[1];
   const uint32_t cw[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
-  float x[32];
   uint32_t mx = 0;  // f16x2 of the largest |dec| (max.f16x2 skips NaN codes, like fmaxf)
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
     const uint32_t lo = e4m3x2_to_f16x2(cw[k]), hi = e4m3x2_to_f16x2(cw[k] >> 16);
     mx = hmax2_u32(mx, hmax2_u32(lo & 0x7fff7fffu, hi & 0x7fff7fffu));
-    const __half2 hl = *reinterpret_cast<const __half2*>(&lo);
-    const __half2 hh = *reinterpret_cast<const __half2*>(&hi);
-    x[4 * k + 0] = __fmul_rn(__low2float(hl), scale);
-    x[4 * k + 1] = __fmul_rn(__high2float(hl), scale);
-    x[4 * k + 2] = __fmul_rn(__low2float(hh), scale);
-    x[4 * k + 3] = __fmul_rn(__high2float(hh), scale);
   }
   const __half2 m2 = *reinterpret_cast<const __half2*>(&mx);
   const float amax = __fmul_rn(fmaxf(__low2float(m2), __high2float(m2)), scale);
   uint32_t w0, w1, w2;
   __half sh;
-  tq3_record(x, amax, w0, w1, w2, sh);
+  if (scale >= 0x1p-100f && scale < 0x1p100f) {
+    // code domain: the thresholds of x >= k*s and |x| > k*s as E4M3 magnitudes
+    sh = __float2half_rn(fminf(__fdiv_rn(amax, 3.5f), 65504.f));
+    const float s = __half2float(sh), rscale = 1.f / scale;
+    uint32_t pk[3], dk[3];
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      const float tk = static_cast<float>(k + 1) * s;  // exact
+      const uint32_t pt = e4m3_threshold(tk, scale, rscale);
+      const uint32_t nt = e4m3_threshold(__uint_as_float(__float_as_uint(tk) + 1u), scale, rscale);
+      pk[k] = pt * 0x01010101u;
+      dk[k] = (pt ^ nt) * 0x01010101u;
+    }
+    uint32_t ch[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      ch[k] = tq3_codes_e4m3x4(cw[k], pk[0], pk[1], pk[2], dk[0], dk[1], dk[2]);
+    record_from_chunks12(ch, w0, w1, w2);
+  } else {
+    // extreme page scales: the fp32 values themselves, x = fp32(dec * scale), with the
+    // record's thresholds t_k = bits(k*s)
+    sh = __float2half_rn(fminf(__fdiv_rn(amax, 3.5f), 65504.f));
+    const float s = __half2float(sh);
+    const int t1 = __float_as_int(s), t2 = __float_as_int(2.f * s), t3 = __float_as_int(3.f * s);
+    uint32_t acc[3] = {0u, 0u, 0u};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t lo = e4m3x2_to_f16x2(cw[k]), hi = e4m3x2_to_f16x2(cw[k] >> 16);
+      const __half2 hl = *reinterpret_cast<const __half2*>(&lo);
+      const __half2 hh = *reinterpret_cast<const __half2*>(&hi);
+      put_code(acc, 4 * k + 0, tq3_code(__fmul_rn(__low2float(hl), scale), t1, t2, t3));
+      put_code(acc, 4 * k + 1, tq3_code(__fmul_rn(__high2float(hl), scale), t1, t2, t3));
+      put_code(acc, 4 * k + 2, tq3_code(__fmul_rn(__low2float(hh), scale), t1, t2, t3));
+      put_code(acc, 4 * k + 3, tq3_code(__fmul_rn(__high2float(hh), scale), t1, t2, t3));
+    }
+    w0 = acc[0];
+    w1 = acc[1];
+    w2 = acc[2];
+  }
   store_record(dst + which * (G * kPageTokens * 14), G, grp, t, w0, w1, w2, sh);
   if (p.publish && h == 0 && threadIdx.x == 0)
     p.tables[d.table_index] = static_cast<int32_t>((1u << kFmtShift) | static_cast<uint32_t>(d.dst_slot));
@@ -196,30 +308,42 @@ __global__ void __launch_bounds__(256) pack_kernel(const __grid_constant__ PackP
                  static_cast<int64_t>(h) * (14 * D);
   const uint16_t* src = (which ? p.v : p.k) +
                         (static_cast<int64_t>(d.first_row + t) * p.Hkv + h) * D + 32 * grp;
-  float x[32];
-  float amax = 0.f;
+  uint32_t w[16];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    uint32_t w[4];
     if (p.vec16) {  // both input arrays 16-byte aligned (checked on the host)
       const uint4 v = reinterpret_cast<const uint4*>(src)[k];
-      w[0] = v.x, w[1] = v.y, w[2] = v.z, w[3] = v.w;
+      w[4 * k] = v.x, w[4 * k + 1] = v.y, w[4 * k + 2] = v.z, w[4 * k + 3] = v.w;
     } else {
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        w[e] = static_cast<uint32_t>(src[8 * k + 2 * e]) |
-               (static_cast<uint32_t>(src[8 * k + 2 * e + 1]) << 16);
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      x[8 * k + 2 * e] = __uint_as_float(w[e] << 16);
-      x[8 * k + 2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
-      amax = fmaxf(amax, fmaxf(fabsf(x[8 * k + 2 * e]), fabsf(x[8 * k + 2 * e + 1])));
+        w[4 * k + e] = static_cast<uint32_t>(src[8 * k + 2 * e]) |
+                       (static_cast<uint32_t>(src[8 * k + 2 * e + 1]) << 16);
     }
   }
+  float amax = 0.f;
+#pragma unroll
+  for (int e = 0; e < 16; ++e)
+    amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[e])), fabsf(bf16_hi(w[e]))));
+  // codes in the bf16 domain: x >= k*s is m >= ceil(t_k / 2^16) and |x| > k*s is
+  // m >= floor(t_k / 2^16) + 1, with m the bf16 magnitude bits and t_k the fp32 bits of k*s
   uint32_t w0, w1, w2;
-  __half sh;
-  tq3_record(x, amax, w0, w1, w2, sh);
+  const __half sh = __float2half_rn(fminf(__fdiv_rn(amax, 3.5f), 65504.f));
+  const float s = __half2float(sh);
+  uint32_t pk[3], dk[3];
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    const uint32_t tk = __float_as_uint(static_cast<float>(k + 1) * s);  // exact
+    const uint32_t pt = (tk + 0xFFFFu) >> 16, nt = (tk >> 16) + 1u;
+    pk[k] = pt * 0x00010001u;
+    dk[k] = (pt ^ nt) * 0x00010001u;
+  }
+  uint32_t ch[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    ch[k] = tq3_codes_bf16x2(w[2 * k], pk[0], pk[1], pk[2], dk[0], dk[1], dk[2]) |
+            (tq3_codes_bf16x2(w[2 * k + 1], pk[0], pk[1], pk[2], dk[0], dk[1], dk[2]) << 6);
+  record_from_chunks12(ch, w0, w1, w2);
   store_record(dst + which * (G * kPageTokens * 14), G, grp, t, w0, w1, w2, sh);
   if (h == 0 && threadIdx.x == 0)
     p.tables[d.table_index] = static_cast<int32_t>((1u << kFmtShift) | static_cast<uint32_t>(d.dst_slot));

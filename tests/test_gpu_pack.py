@@ -115,3 +115,31 @@ def test_copy_reset_and_slot_reuse():
     lp.append([1], [21], to_bf16_tensor(k2), to_bf16_tensor(v2))
     op.append([1], [21], F.bf16_bits_to_f64(k2), F.bf16_bits_to_f64(v2))
     compare(lp, op, [0, 1, 2])
+
+
+@pytest.mark.parametrize("D", [64, 256])
+def test_extreme_magnitudes_bit_exact(D):
+    """Pages whose values sit at bf16's extremes (subnormals near 1e-40, values near 1e38) and in
+    between: the TQ3 coder takes its exact fallback for page scales outside [2^-100, 2^100) and
+    the source-domain path elsewhere; both must give the oracle's bytes, for demotion and for
+    direct prefill packing."""
+    rng = np.random.default_rng(5)
+    Hkv, n = 2, 16 * 12
+    mags = np.array([1e-40, 3e-39, 1e-35, 1e-20, 1.0, 1e20, 1e30, 1e37, 4e37], np.float32)
+    k = np.empty((n, Hkv, D), np.uint16)
+    v = np.empty((n, Hkv, D), np.uint16)
+    for p in range(n // 16):
+        for h in range(Hkv):
+            sk, sv = mags[(p + h) % mags.size], mags[(3 * p + h) % mags.size]
+            k[16 * p:16 * p + 16, h] = _tokens(rng, 16, 1, D, sk)[:, 0]
+            v[16 * p:16 * p + 16, h] = _tokens(rng, 16, 1, D, sv)[:, 0]
+    k[5, 0, :7] = 0x8000                          # signed zeros among tiny values
+    v[40, 1, 3] = 0x0001                          # the smallest bf16 subnormal
+    lp = Pool(Hkv, D, 2, 16, 32, 32)
+    op = P.RefPool(Hkv, D, 2, 16, 32, 32)
+    lp.append([0], [n], to_bf16_tensor(k), to_bf16_tensor(v))
+    op.append([0], [n], F.bf16_bits_to_f64(k), F.bf16_bits_to_f64(v))
+    assert lp.demote([0], 16) == len(op.demote([0], 16))
+    lp.prefill([1], [n], to_bf16_tensor(k), to_bf16_tensor(v), window=16)
+    op.prefill([1], [n], F.bf16_bits_to_f64(k), F.bf16_bits_to_f64(v), window_tokens=16)
+    compare(lp, op, [0, 1])
