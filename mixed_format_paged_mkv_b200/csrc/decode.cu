@@ -1314,7 +1314,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
   const SeqDesc& sd = p.seq[pair / p.Hkv];
   const int h = pair % p.Hkv;
   const int S = sd.n_parts, D = p.D, tid = threadIdx.x;
-  const int groups = D / 4, nsub = kMergeThreads / groups;
+  const int groups = D / 4, nsub = static_cast<int>(blockDim.x) / groups;
   const int c4 = tid % groups, k = tid / groups;
   const int64_t base0 = (static_cast<int64_t>(sd.part0) * p.Hkv + h) * p.NC + n;
   const int64_t stride = static_cast<int64_t>(p.Hkv) * p.NC;
@@ -1531,7 +1531,14 @@ bool partial_supported(int D, int NC) {
 // The merge follows the last partial grid of the call as its programmatic dependent.
 cudaError_t launch_merge(const DecodeParams& p, cudaStream_t s) {
   if (p.n_seqs <= 0) return cudaSuccess;
-  return launch_ex(merge_kernel, dim3(p.n_seqs * p.Hkv * p.NC), kMergeThreads, 0,
+  // D/4 threads per subset of partials, as many subsets (a power of two, up to the block
+  // limit) as the call's largest partial count needs
+  int max_parts = 1;
+  for (int i = 0; i < p.n_seqs; ++i) max_parts = max(max_parts, p.seq[i].n_parts);
+  const int groups = p.D / 4;
+  int nsub = groups >= 32 ? 1 : 32 / groups;
+  while (nsub < max_parts && 2 * nsub * groups <= kMergeThreads) nsub *= 2;
+  return launch_ex(merge_kernel, dim3(p.n_seqs * p.Hkv * p.NC), nsub * groups, 0,
                    p.n_units > 0, s, p);
 }
 
