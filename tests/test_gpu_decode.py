@@ -140,19 +140,32 @@ def test_repeated_sequence_rows_and_order():
         assert_close(out[i], oracle_decode(op, w, s), what=f"row {i}")
 
 
+def _full_size_reference(args):
+    """Oracle output of one (sequence, KV head) of the full-size long-context layer (run in a
+    spawned worker: pages of a head depend only on that head's inputs)."""
+    s, h = args
+    w = WORKLOADS[4].scaled(layers=1)
+    op = oracle_pool(w, seqs=[s], heads=[h], shape=dict(w.pool_shape(), num_kv_heads=1))
+    return oracle_decode(op, w, s, heads=[h])
+
+
 @pytest.mark.slow
 def test_long_context_full_size_sampled():
     """The long-context workload at full size (4 x 131072 tokens, 24/4 heads, D 256), in the
-    launch configuration the benchmark times; the oracle checks one sequence's first KV head
-    group (pages of a head depend only on that head's inputs)."""
-    w = WORKLOADS[4].scaled(layers=1)
-    lp = lib_pool(w)
-    out = lp.decode(list(range(w.B)), q_tensor(w)).cpu().numpy()
-    lp.device_status()
+    launch configuration the benchmark times; the oracle checks one KV-head group of every
+    sequence, every KV head index once (24 of the 96 query-head outputs)."""
+    import multiprocessing as mp
+    pairs = [(0, 0), (1, 2), (2, 1), (3, 3)]
+    # the oracle workers start (spawned) before the first GPU call of this test
+    with mp.get_context("spawn").Pool(len(pairs)) as workers:
+        pending = workers.map_async(_full_size_reference, pairs)
+        w = WORKLOADS[4].scaled(layers=1)
+        lp = lib_pool(w)
+        out = lp.decode(list(range(w.B)), q_tensor(w)).cpu().numpy()
+        lp.device_status()
+        refs = pending.get(timeout=900)
     assert np.all(np.isfinite(out))
-    for s, h in ((1, 2),):
-        op = oracle_pool(w, seqs=[s], heads=[h], shape=dict(w.pool_shape(), num_kv_heads=1))
-        ref = oracle_decode(op, w, s, heads=[h])
+    for (s, h), ref in zip(pairs, refs):
         assert_close(out[s][:, h * w.g:(h + 1) * w.g], ref, what=f"full-size seq {s} head {h}")
 
 
