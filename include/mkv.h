@@ -235,9 +235,11 @@ MKV_API int mkv_decode_attention_noalloc(mkv_pool_t pool, const int32_t* seq_ids
  *     os resultados parciais são combinados"): the FP8 grid, then the TQ3 grid launched as its
  *     programmatic dependent, so both share one wave;
  *   MKV_DECODE_FUSED -- one grid whose CTAs branch on their unit's format;
- *   MKV_DECODE_AUTO (default) -- per call: FUSED when FP8 pages carry more than 15% of the
- *     call's planned time, else SPLIT (FP8 CTAs need more shared memory than TQ3 CTAs, so many
- *     of them no longer fit one wave of per-format grids).
+ *   MKV_DECODE_AUTO (default) -- per call: FUSED when the fused grid keeps as many CTAs per SM
+ *     as the TQ3 grid (head_dim 64 and 128), when FP8 pages carry more than 15% of the call's
+ *     planned time, or when the sequences holding FP8 pages times the KV heads exceed the SMs
+ *     the call is planned for; else SPLIT (for head_dim 256, FP8 CTAs need more shared memory
+ *     than TQ3 CTAs, so many of them no longer fit one wave of per-format grids).
  * Host only; applies to later decode calls on this pool.  Errors: INVALID_ARG. */
 #define MKV_DECODE_SPLIT 0
 #define MKV_DECODE_FUSED 1

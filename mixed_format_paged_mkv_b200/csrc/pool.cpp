@@ -140,29 +140,39 @@ bool valid_pool(mkv_pool_t p) { return p != nullptr; }
 constexpr int64_t kFp8PageCost = 11;
 constexpr int64_t kTq3PageCost = 10;
 // Automatic choice of partial kernels: one fused grid when FP8 pages carry more than this share
-// of the call's planned time.  Measured on the long-context workload: at 4% FP8 pages the
+// of the call's planned time, or when the FP8 grid alone would hold more than one CTA per SM
+// (many sequences, each with its own FP8 units: 64 sequences x 8 KV heads at D 128 decode in
+// 604 us fused against 631 us per format, with 0.9% of the pages FP8).  Measured on the long-context workload: at 4% FP8 pages the
 // per-format grids are faster (150.8 against 156.3 us), at 25% the fused grid (170.0 against
 // 198.8 us): FP8 CTAs need more shared memory than TQ3 CTAs, so beyond one FP8 CTA per SM the
 // per-format grids no longer fit one wave.
 constexpr double kFusedAboveFp8Share = 0.15;
 
-// Decode kernels of a call over these sequences (kDecodeSplit, kDecodeFused or kDecodeBf16).
-int decode_mode(const mkv_pool* p, const int32_t* seq_ids, int32_t n) {
+// SMs a decode call's cut is planned for: the device's, or fewer when the caller asked so.
+int plan_sms(const mkv_pool* p) {
+  return p->decode_sms > 0 && p->decode_sms < p->sm_count ? p->decode_sms : p->sm_count;
+}
+
+// Decode kernels of a call over these sequences with NC query columns per KV head
+// (kDecodeSplit, kDecodeFused or kDecodeBf16).
+int decode_mode(const mkv_pool* p, const int32_t* seq_ids, int32_t n, int32_t NC) {
   if (p->page_fmt == MKV_FMT_BF16) return kDecodeBf16;
   if (p->decode_kernels != MKV_DECODE_AUTO)
     return p->decode_kernels == MKV_DECODE_FUSED ? kDecodeFused : kDecodeSplit;
-  int64_t c8 = 0, c3 = 0;
+  int64_t c8 = 0, c3 = 0, groups8 = 0;
   for (int32_t i = 0; i < n; ++i) {
     const Seq& s = p->seqs[seq_ids[i]];
     c8 += static_cast<int64_t>(s.fp8_pages.size()) * kFp8PageCost;
     c3 += static_cast<int64_t>(s.n3) * kTq3PageCost;
+    groups8 += s.fp8_pages.empty() ? 0 : 1;
   }
+  // the fused grid keeps as many CTAs per SM as the TQ3 grid (D 64 and 128): one grid is enough
+  const int D = p->cfg.head_dim;
+  if (partial_ctas_per_sm(D, NC, kDecodeFused) >= partial_ctas_per_sm(D, NC, kDecodeSplit))
+    return kDecodeFused;
+  // every sequence with FP8 pages gives the FP8 grid at least one CTA per KV head
+  if (groups8 * p->cfg.num_kv_heads > plan_sms(p)) return kDecodeFused;
   return c8 > kFusedAboveFp8Share * static_cast<double>(c8 + c3) ? kDecodeFused : kDecodeSplit;
-}
-
-// SMs a decode call's cut is planned for: the device's, or fewer when the caller asked so.
-int plan_sms(const mkv_pool* p) {
-  return p->decode_sms > 0 && p->decode_sms < p->sm_count ? p->decode_sms : p->sm_count;
 }
 
 int64_t page_head_bytes(const mkv_pool_config& c) {
@@ -352,7 +362,7 @@ int plan_decode(mkv_pool_t p, const int32_t* seq_ids, int32_t n, int32_t q_len, 
   plan->pos.clear();
   plan->cost.clear();
   std::vector<int32_t> np(n);
-  plan->mode = decode_mode(p, seq_ids, n);
+  plan->mode = decode_mode(p, seq_ids, n, plan->NC);
   cut_units(p, seq_ids, n, plan->NC, plan->mode, np.data(),
             [&](const UnitDesc& u, int64_t cost, int32_t i) {
     plan->unit.push_back(u);
@@ -878,7 +888,7 @@ int mkv_decode_attention_noalloc(mkv_pool_t p, const int32_t* seq_ids, int32_t n
     t.cost[nu++] = cost;
     return true;
   };
-  const int mode = decode_mode(p, seq_ids, n_seqs);
+  const int mode = decode_mode(p, seq_ids, n_seqs, NC);
   const int64_t cut = cut_units(p, seq_ids, n_seqs, NC, mode, np, keep);
   if (cut < 0)
     return fail(MKV_ERR_UNSUPPORTED, "the no-allocation decode takes at most %d work units per call", kDecodeMaxUnits);
