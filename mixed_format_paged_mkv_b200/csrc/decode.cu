@@ -77,7 +77,7 @@ struct Cfg {
   // Stage s only ever holds pages i with i % NST == s, and they belong to warp group i % PW:
   // with NST a multiple of PW each stage has a fixed owner, which refills it when done.
   static constexpr int FP8_NST = 8;
-  static constexpr int TQ3_NST = 8;
+  static constexpr int TQ3_NST = TEAM ? 2 * TW : 8;
   static constexpr int BF16_NST = 8;
   static_assert(FP8_NST % PW == 0 && TQ3_NST % PW == 0 && BF16_NST % PW == 0, "stage ownership");
   static constexpr int RING_FP8 = (K == kKindFp8 || K == kKindFused) ? FP8_NST * FP8_STAGE : 0;
@@ -1044,7 +1044,7 @@ __device__ void run_unit_team(const DecodeParams& p, const SeqDesc& sd, const Un
   const int g0 = warp * GW;
   uint2* xp = reinterpret_cast<uint2*>(sm.xch);              // [2][TW][NT][32] P^T fragments
   float* xr = reinterpret_cast<float*>(sm.xch + C::XCH_P);   // [2][TW][NT][8] page references
-  int32_t* xf = sm.cnt + NST;                                // [2][TW] page raised a reference
+  int32_t* xf = sm.cnt;  // [2][TW] per page: bit 0 raised a reference, bit 1 V scales out of range
 
   float acc[2 * GW][NT][4];
 #pragma unroll
@@ -1064,7 +1064,7 @@ __device__ void run_unit_team(const DecodeParams& p, const SeqDesc& sd, const Un
     const int par = (b / TW) & 1;
     const int nb = min(TW, count - b);
     // K: this warp's page of the batch
-    bool ok = true, raised = false;
+    bool ok = true, raised = false, wide = false;
     float lp[NT][2];  // the page's denominator shares, relative to its references
     float rf[NT][2];  // the page's references of columns 2c, 2c+1
     const int ik = b + warp;
@@ -1085,12 +1085,18 @@ __device__ void run_unit_team(const DecodeParams& p, const SeqDesc& sd, const Un
         else
           tq3_logits_nt<D, NT>(pg, sm.qf, sm.corr, lane, kw, ks5, x);
         const int tok0 = 16 * sm.list[ik].y;
+        const bool edge = tok0 + 15 > min_lim;
+        if constexpr (F == kTq3) {
+          // the V range check, once per page for the whole team
+          const uint32_t vmax = tq3_v_scale_max<D>(pg, lane);
+          wide = !(vmax >= kVScaleLo && vmax <= kVScaleHi);
+        }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           const float ls = lsc[nt];
 #pragma unroll
           for (int j = 0; j < 4; ++j) x[nt][j] *= ls;
-          if (tok0 + 15 > min_lim) {
+          if (edge) {
             // causal limits of columns 2c, 2c+1 (padding columns see the whole context)
             const int n0 = 8 * nt + 2 * c, n1 = n0 + 1;
             mask_page(x[nt], tok0, r, n0 < p.NC ? min_lim + n0 / p.g : sd.ctx - 1,
@@ -1132,15 +1138,24 @@ __device__ void run_unit_team(const DecodeParams& p, const SeqDesc& sd, const Un
         }
       }
     }
-    if (lane == 0) xf[par * TW + warp] = raised ? 1 : 0;
+    if (lane == 0) xf[par * TW + warp] = (raised ? 1 : 0) | (wide ? 2 : 0);
     // the batch's probabilities are published; every warp of the team stops together on a
     // failed wait
     if (!barrier_and(1, 32 * TW, ok)) {
       if (lane == 0) flag_status(p.status, kStatusTimeout);
       break;
     }
+    // the previous batch's stages: every warp fenced its reads of them before this barrier, so
+    // warp w refills the stage of page b - TW + w with the page NST ahead
+    if (b >= TW && b - TW + warp + NST < count)
+      fill_stage<PG, F>(sm, slab, slot_bytes, h, b - TW + warp + NST, lane);
+    int flags[TW];
     int any_raised = 0;
-    for (int q = 0; q < nb; ++q) any_raised |= xf[par * TW + q];
+#pragma unroll
+    for (int q = 0; q < TW; ++q) {
+      flags[q] = q < nb ? xf[par * TW + q] : 0;
+      any_raised |= flags[q] & 1;
+    }
     // P scale of each page of a raising batch (column r) and the page's own sums
     float fq[TW][NT];
     if (any_raised) {
@@ -1148,7 +1163,7 @@ __device__ void run_unit_team(const DecodeParams& p, const SeqDesc& sd, const Un
       for (int nt = 0; nt < NT; ++nt) {
         float n0 = mc[nt][0], n1 = mc[nt][1], nr = mr[nt];
         for (int q = 0; q < nb; ++q) {
-          if (!xf[par * TW + q]) continue;
+          if (!(xf[par * TW + q] & 1)) continue;
           const float* rq = xr + ((par * TW + q) * NT + nt) * 8;
           n0 = fmaxf(n0, rq[2 * c]);
           n1 = fmaxf(n1, rq[2 * c + 1]);
@@ -1166,8 +1181,7 @@ __device__ void run_unit_team(const DecodeParams& p, const SeqDesc& sd, const Un
         }
 #pragma unroll
         for (int q = 0; q < TW; ++q) {
-          const float rq = q < nb && xf[par * TW + q] ? xr[((par * TW + q) * NT + nt) * 8 + r]
-                                                       : mr[nt];
+          const float rq = (flags[q] & 1) ? xr[((par * TW + q) * NT + nt) * 8 + r] : mr[nt];
           fq[q][nt] = rq == -INFINITY ? 0.f : pow2i(rq - nr);
         }
         // this warp's page: its sums move to the new references
@@ -1192,9 +1206,10 @@ __device__ void run_unit_team(const DecodeParams& p, const SeqDesc& sd, const Un
         const uint8_t* pg = sm.ring + s * STAGE;
         uint2 pb[NT];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          pb[nt] = xp[((par * TW + q) * NT + nt) * 32 + lane];
-          if (any_raised) {
+        for (int nt = 0; nt < NT; ++nt) pb[nt] = xp[((par * TW + q) * NT + nt) * 32 + lane];
+        if (any_raised) {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
             float f = 0.f;
 #pragma unroll
             for (int qq = 0; qq < TW; ++qq) f = qq == q ? fq[qq][nt] : f;
@@ -1206,8 +1221,10 @@ __device__ void run_unit_team(const DecodeParams& p, const SeqDesc& sd, const Un
         if constexpr (F == kFp8) {
           fp8_pv_nt<D, NT, GW>(acc, pg, lane, g0, pb);
         } else {
-          const uint32_t vmax = tq3_v_scale_max<D>(pg, lane);
-          if (vmax >= kVScaleLo && vmax <= kVScaleHi)
+          int fq_flags = 0;
+#pragma unroll
+          for (int qq = 0; qq < TW; ++qq) fq_flags = qq == q ? flags[qq] : fq_flags;
+          if (!(fq_flags & 2))
             tq3_pv_nt<D, NT, GW, false>(acc, pg, lane, vw, vs1, g0, pb);
           else
             tq3_pv_nt<D, NT, GW, true>(acc, pg, lane, vw, vs1, g0, pb);
@@ -1215,21 +1232,10 @@ __device__ void run_unit_team(const DecodeParams& p, const SeqDesc& sd, const Un
       } else if (lane == 0) {
         flag_status(p.status, kStatusTimeout);
       }
-      // release the stage: the last of the team's warps done with it refills it
-      if (iv + NST < count) {
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncwarp();
-        bool last = false;
-        if (lane == 0) {
-          __threadfence_block();
-          last = atomicAdd(&sm.cnt[s], 1) == TW - 1;
-          if (last) sm.cnt[s] = 0;
-          __threadfence_block();
-        }
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (last) fill_stage<PG, F>(sm, slab, slot_bytes, h, iv + NST, lane);
-      }
     }
+    // this warp's reads of the batch's stages come before the async-proxy refills that follow
+    // the next barrier
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   // drain (bounded) after a failed wait: the last copy issued into every stage lands before the
   // ring is reused

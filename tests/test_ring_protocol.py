@@ -75,9 +75,10 @@ def test_ring_shape_that_violates_the_rule_is_detected():
 def replay_team(count, nst, tw, seed):
     """Team layout (more than 8 query columns): pages go in batches of tw; warp w first waits
     for page b + w of batch b (its K page), then all warps meet at the batch barrier, then every
-    warp waits for and consumes every page of the batch (V); a stage is refilled with page
-    i + nst once all tw warps released page i.  Returns True if some wait started for fill f of
-    a stage whose fill f-1 had not completed."""
+    warp waits for and consumes every page of the batch (V).  A batch's stages are released at
+    the next batch's barrier (every warp has consumed them by then) and refilled with the pages
+    nst ahead.  Returns True if some wait started for fill f of a stage whose fill f-1 had not
+    completed."""
     rng = random.Random(seed)
     completed = [0] * nst
     releases = [0] * count
@@ -122,6 +123,9 @@ def replay_team(count, nst, tw, seed):
             i = in_flight.pop(rng.randrange(len(in_flight)))
             completed[i % nst] += 1
         elif m == "barrier":
+            b = batch[0]
+            for i in range(max(0, b - tw), min(b, count)):   # the previous batch is released
+                releases[i] = tw
             step = [0] * tw
         else:
             w, b = m, batch[m]
@@ -134,7 +138,6 @@ def replay_team(count, nst, tw, seed):
                 i = b + step[w]
                 if start_wait(w, i):
                     waiting[w] = None
-                    releases[i] += 1
                     step[w] += 1
                     if step[w] == min(tw, count - b):
                         batch[w] += tw
@@ -142,7 +145,7 @@ def replay_team(count, nst, tw, seed):
     return ambiguous
 
 
-@pytest.mark.parametrize("nst,tw", [(8, 4), (8, 2)])   # the kernel's team rings
+@pytest.mark.parametrize("nst,tw", [(8, 4), (4, 2), (8, 2)])   # the kernel's team rings
 def test_team_ring_never_waits_ambiguously(nst, tw):
     for seed in range(60):
         for count in (1, 3, tw, nst - 1, nst, nst + 3, 3 * nst + 1, 45):
@@ -151,10 +154,10 @@ def test_team_ring_never_waits_ambiguously(nst, tw):
 
 def test_team_ring_needs_a_stage_per_page_of_a_batch():
     # Every warp consumes every page, so a warp never waits on a fill whose predecessor it has
-    # not consumed itself: any ring of at least tw stages is unambiguous.  Fewer stages than a
-    # batch has pages deadlock (a K page waits for a stage whose page is consumed only after
-    # the barrier that K page gates), and the model says so.
-    assert not any(replay_team(45, 4, 4, seed) for seed in range(100))
+    # not consumed itself.  Stages are released a batch late, so the ring needs two batches:
+    # with one, a K page waits for a stage released only at the barrier that K page gates, and
+    # the model reports the deadlock.
+    assert not any(replay_team(45, 8, 4, seed) for seed in range(100))
     with pytest.raises(AssertionError, match="deadlock"):
         for seed in range(20):
-            replay_team(45, 2, 4, seed)
+            replay_team(45, 4, 4, seed)
