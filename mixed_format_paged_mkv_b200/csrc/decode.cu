@@ -1542,13 +1542,15 @@ bool partial_supported(int D, int NC) {
 // The merge follows the last partial grid of the call as its programmatic dependent.
 cudaError_t launch_merge(const DecodeParams& p, cudaStream_t s) {
   if (p.n_seqs <= 0) return cudaSuccess;
-  // D/4 threads per subset of partials, as many subsets (a power of two, up to the block
-  // limit) as the call's largest partial count needs
+  // D/4 threads per subset of partials; a thread keeps kMergeBatch partials in flight, so the
+  // call's largest partial count needs ceil(max / kMergeBatch) subsets (a power of two, up to
+  // the block limit; at least one warp)
   int max_parts = 1;
   for (int i = 0; i < p.n_seqs; ++i) max_parts = max(max_parts, p.seq[i].n_parts);
   const int groups = p.D / 4;
+  const int want = (max_parts + kMergeBatch - 1) / kMergeBatch;
   int nsub = groups >= 32 ? 1 : 32 / groups;
-  while (nsub < max_parts && 2 * nsub * groups <= kMergeThreads) nsub *= 2;
+  while (nsub < want && 2 * nsub * groups <= kMergeThreads) nsub *= 2;
   return launch_ex(merge_kernel, dim3(p.n_seqs * p.Hkv * p.NC), nsub * groups, 0,
                    p.n_units > 0, s, p);
 }
