@@ -194,12 +194,6 @@ __device__ __forceinline__ void softmax_k(KState& st, float (&x)[4], float (&pr)
   st.l[1] += pr[1] + pr[3];
 }
 
-// 2^d for an integer-valued d <= 127, built from its exponent bits (exact); 0 for d < -126,
-// -inf included.
-__device__ __forceinline__ float pow2i(float d) {
-  return d < -126.f ? 0.f : __int_as_float((static_cast<int>(d) + 127) << 23);
-}
-
 __device__ __forceinline__ void mask_page(float (&x)[4], int tok0, int r, int lim0, int lim1) {
   if (tok0 + r > lim0) x[0] = -INFINITY;
   if (tok0 + r > lim1) x[1] = -INFINITY;
@@ -993,10 +987,10 @@ __device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDes
 // every warp), and publishes their P^T fragments; after one team barrier every warp multiplies
 // the whole batch by the V of its own channel groups.  Every page's codes are decoded once.
 // The reference is raised lazily, as on the one-tile path: a page whose column exceeds it by
-// more than 8 uses its own reference (the column maximum rounded up to an integer) and flags
-// the batch; after the barrier every warp raises the common reference to the batch's largest
-// and scales that batch's P and its own accumulators by exact powers of two.  Probabilities fed
-// to the MMAs stay <= 2^8.  Each warp sums the denominators of its own K pages; the sums meet
+// more than 8 uses its own reference (the column maximum, so the dominant token's probability
+// is exactly 1) and flags the batch; after the barrier every warp raises the common reference
+// to the batch's largest and rescales that batch's P and its own accumulators.  Probabilities
+// fed to the MMAs stay <= 2^8.  Each warp sums the denominators of its own K pages; the sums meet
 // in the combine.
 template <int D, int NT, int K, int F>
 __device__ void run_unit_team(const DecodeParams& p, const SeqDesc& sd, const UnitDesc& u, int h,
@@ -1105,14 +1099,14 @@ __device__ void run_unit_team(const DecodeParams& p, const SeqDesc& sd, const Un
           float m0 = fmaxf(x[nt][0], x[nt][2]), m1 = fmaxf(x[nt][1], x[nt][3]);
           const bool need = m0 > mc[nt][0] + kLazyRescale || m1 > mc[nt][1] + kLazyRescale;
           if (__any_sync(0xffffffffu, need)) {
-            // this page raises: its own references (column maximum rounded up) where needed
+            // this page raises: its own references (the column maxima) where needed
 #pragma unroll
             for (int o = 4; o < 32; o <<= 1) {
               m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
               m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
             }
-            if (m0 > mc[nt][0] + kLazyRescale) rf[nt][0] = ceilf(m0);
-            if (m1 > mc[nt][1] + kLazyRescale) rf[nt][1] = ceilf(m1);
+            if (m0 > mc[nt][0] + kLazyRescale) rf[nt][0] = m0;
+            if (m1 > mc[nt][1] + kLazyRescale) rf[nt][1] = m1;
             raised = true;
           }
           const float r0 = rf[nt][0] == -INFINITY ? 0.f : rf[nt][0];
@@ -1169,7 +1163,7 @@ __device__ void run_unit_team(const DecodeParams& p, const SeqDesc& sd, const Un
           n1 = fmaxf(n1, rq[2 * c + 1]);
           nr = fmaxf(nr, rq[r]);
         }
-        const float a0 = pow2i(mc[nt][0] - n0), a1 = pow2i(mc[nt][1] - n1);  // 0 from -inf
+        const float a0 = fast_exp2(mc[nt][0] - n0), a1 = fast_exp2(mc[nt][1] - n1);  // 0 from -inf
         lk[nt][0] *= a0;
         lk[nt][1] *= a1;
 #pragma unroll
@@ -1180,8 +1174,8 @@ __device__ void run_unit_team(const DecodeParams& p, const SeqDesc& sd, const Un
           acc[j][nt][3] *= a1;
         }
         // this warp's page: its sums move to the new references
-        lk[nt][0] = fmaf(lp[nt][0], rf[nt][0] == -INFINITY ? 0.f : pow2i(rf[nt][0] - n0), lk[nt][0]);
-        lk[nt][1] = fmaf(lp[nt][1], rf[nt][1] == -INFINITY ? 0.f : pow2i(rf[nt][1] - n1), lk[nt][1]);
+        lk[nt][0] = fmaf(lp[nt][0], rf[nt][0] == -INFINITY ? 0.f : fast_exp2(rf[nt][0] - n0), lk[nt][0]);
+        lk[nt][1] = fmaf(lp[nt][1], rf[nt][1] == -INFINITY ? 0.f : fast_exp2(rf[nt][1] - n1), lk[nt][1]);
         mc[nt][0] = n0;
         mc[nt][1] = n1;
         mr[nt] = nr;
@@ -1209,8 +1203,8 @@ __device__ void run_unit_team(const DecodeParams& p, const SeqDesc& sd, const Un
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
             const float rq = (fq & 1) ? xr[((par * TW + q) * NT + nt) * 8 + r] : mr_old[nt];
-            const float f = rq == -INFINITY ? 0.f : pow2i(rq - mr[nt]);
-            const uint32_t f2 = pack_f16x2(f, f);  // a power of two <= 1 (or 0)
+            const float f = rq == -INFINITY ? 0.f : fast_exp2(rq - mr[nt]);
+            const uint32_t f2 = pack_f16x2(f, f);  // <= 1 (0 for a column the page does not see)
             pb[nt].x = hmul2_u32(pb[nt].x, f2);
             pb[nt].y = hmul2_u32(pb[nt].y, f2);
           }

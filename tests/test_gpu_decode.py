@@ -82,6 +82,19 @@ def test_gqa_widths_and_multi_token(Hq, Hkv, q_len):
     run_and_check(w)
 
 
+@pytest.mark.parametrize("D,Hq,Hkv,q_len", [(64, 16, 2, 3), (64, 8, 1, 4), (128, 24, 4, 4),
+                                            (256, 24, 2, 1)])
+def test_team_layout_shapes(D, Hq, Hkv, q_len):
+    """More than 8 query columns per KV head (the team layout: one page decoded once for all
+    n-tiles) at every head size, and 12 query heads per KV head at q_len 1 (two n-tiles)."""
+    w = Workload("team", 20 + D + q_len, B=2, Hq=Hq, Hkv=Hkv, D=D, q_len=q_len, window=48,
+                 ctx=(1100, 123), outliers=True)
+    for fused in (False, True):
+        lp = lib_pool(w)
+        lp.set_decode_kernels(fused)
+        run_and_check(w, lp=lp)
+
+
 @pytest.mark.parametrize("ctx", [(1,), (15,), (16,), (17,), (33,), (4, 300)])
 def test_short_and_ragged_contexts(ctx):
     w = Workload("short", 12, B=len(ctx), Hq=8, Hkv=2, D=128, q_len=1, window=16, ctx=ctx)

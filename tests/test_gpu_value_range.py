@@ -60,8 +60,21 @@ def test_uniform_scales(k_scale, v_scale, D):
                      what=f"K x{k_scale:g} V x{v_scale:g} D {D} seq {s}")
 
 
+@pytest.mark.parametrize("k_scale,v_scale", [(1.0, 1e-4), (4.0, 1e3), (4.0, 3e4), (1e3, 1e3)])
+@pytest.mark.parametrize("D", [64, 256])
+def test_uniform_scales_many_query_columns(k_scale, v_scale, D):
+    """q_len 4 with 6 query heads per KV head: 24 query columns, the team layout (each page
+    decoded once for three n-tiles; two warps for D 64, four for D 256)."""
+    w = _base(D=D, Hq=12, Hkv=2, q_len=4, k_scale=k_scale, v_scale=v_scale, cfg=45 + D,
+              ctx=(900, 260))
+    out, refs, _ = _decode(w)
+    for s in range(w.B):
+        assert_close(out[s] / v_scale, refs[s] / v_scale,
+                     what=f"q_len 4 K x{k_scale:g} V x{v_scale:g} D {D} seq {s}")
+
+
 @pytest.mark.parametrize("D,q_len,k_scale", [(256, 1, 1.0), (128, 1, 4.0), (256, 3, 1.0),
-                                             (64, 2, 1.0)])
+                                             (64, 2, 1.0), (64, 4, 4.0)])
 def test_mixed_group_and_token_scales(D, q_len, k_scale):
     """Every (token, KV head, 32-channel group) of K and V has its own multiplier from 1e-4 to
     3e4, so one page mixes scales across groups and tokens."""
