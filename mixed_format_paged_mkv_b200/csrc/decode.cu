@@ -1188,10 +1188,11 @@ __device__ void run_unit_team(const DecodeParams& p, const SeqDesc& sd, const Un
       }
     }
     // V: every page of the batch, this warp's channel groups
+    // No wait here: the page's K warp observed its copy complete (mbarrier acquire) before the
+    // team barrier, whose memory ordering carries that to every warp of the team.
     auto v_page = [&](int q) {
-      const int iv = b + q, s = iv % NST;
-      // landed (its K warp waited for it before the barrier): returns at once
-      if (mbar_wait_warp(&sm.full[s], (iv / NST) & 1)) {
+      const int s = (b + q) % NST;
+      {
         const uint8_t* pg = sm.ring + s * STAGE;
         uint2 pb[NT];
 #pragma unroll
@@ -1217,8 +1218,6 @@ __device__ void run_unit_team(const DecodeParams& p, const SeqDesc& sd, const Un
           else
             tq3_pv_nt<D, NT, GW, true>(acc, pg, lane, vw, vs1, g0, pb);
         }
-      } else if (lane == 0) {
-        flag_status(p.status, kStatusTimeout);
       }
     };
     if constexpr (K == kKindFused) {
