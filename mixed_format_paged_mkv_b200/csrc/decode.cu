@@ -7,14 +7,15 @@
 // copy of the cache is made (section "... sem a chamada sombra densa").
 //
 // The host cuts every sequence into work units -- (format, logical page range) -- and orders
-// them largest first.  Three launches per call (per launch group): the TQ3 partial kernel over
-// the TQ3 units, the FP8 partial kernel over the FP8 units and the merge kernel.  The FP8 and
-// merge kernels are programmatic dependents of the kernel before them: the FP8 CTAs take SM
-// room as soon as TQ3 CTAs retire (one wave of both formats), the merge CTAs are resident
-// before the partial kernels end and wait for their results with griddepcontrol.wait.  (A fused
-// variant runs both formats in one grid, branching per CTA; it is kept for the comparison.)
+// them largest first.  Three launches per call (per launch group): the FP8 partial kernel over
+// the FP8 units, the TQ3 partial kernel over the TQ3 units and the merge kernel.  The TQ3 and
+// merge kernels are programmatic dependents of the kernel before them: the TQ3 CTAs fill the
+// SM room the FP8 CTAs leave (one wave of both formats), and the merge CTAs wait for the
+// partial states with griddepcontrol.wait.  A fused variant runs both formats in one grid,
+// branching per CTA; the host picks it per call where it keeps the same occupancy or where the
+// FP8 units would overflow the wave.
 //
-// A partial CTA takes one (unit, KV head):
+// A partial CTA with at most 8 query columns per KV head takes one (unit, KV head):
 //   1. one warp scans the block-table entries of the range, keeps the pages of the unit's format
 //      and starts the first bulk async copies of those pages into a shared-memory ring;
 //   2. the warps take pages round-robin; each ring stage always belongs to the same warp(s),
@@ -23,6 +24,8 @@
 //   3. per page the logits, the online softmax (running max m and denominator l per query
 //      column) and P.V;
 //   4. the CTA combines its warps and writes its partial state (m, l, acc) per query column.
+// With more query columns a CTA is a team of warps that decodes each page once for all
+// n-tiles (run_unit_team).
 // The merge kernel combines, per (sequence, KV head, query column), all partial states of both
 // formats: M = max m, L = sum l 2^(m-M), O = sum acc 2^(m-M) / L.
 //
