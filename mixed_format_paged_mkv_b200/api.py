@@ -246,14 +246,14 @@ class Pool:
         return b.value
 
     def decode_plan(self, seq_ids, q_len, num_q_heads):
-        """The work units a decode call would cut (mkv_decode_plan): int32 [units, 5] rows of
-        (call position, format, first logical page, end logical page, pages of that format), and
-        the CTA budget of one wave."""
+        """The work units a decode call would cut (mkv_decode_plan): int32 [units, 6] rows of
+        (call position, format, first logical page, end logical page, pages of that format, CTA),
+        CTA by CTA, and the CTA budget of one wave."""
         s, sp = _i32_array(seq_ids)
         n, wave = ctypes.c_int32(), ctypes.c_int32()
         _check(lib().mkv_decode_plan(self.handle, sp, s.size, q_len, num_q_heads, None, 0,
                                      ctypes.byref(n), ctypes.byref(wave)), "mkv_decode_plan")
-        u = np.zeros((max(n.value, 1), 5), dtype=np.int32)
+        u = np.zeros((max(n.value, 1), 6), dtype=np.int32)
         _check(lib().mkv_decode_plan(self.handle, sp, s.size, q_len, num_q_heads,
                                      u.ctypes.data_as(_I32P), n.value, ctypes.byref(n), None),
                "mkv_decode_plan")

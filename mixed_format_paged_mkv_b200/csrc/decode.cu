@@ -116,6 +116,10 @@ struct Cfg {
                                                              : (D == 128 ? 5 : 6);
 };
 
+// Stage barriers in the header (full[]): every unit initialises all of them, whatever its
+// format's ring length, so that a CTA's next unit can invalidate and initialise them again.
+constexpr int kRingBarriers = 16;
+
 struct Smem {
   uint64_t* full;   // [stage]: the stage's page landed (arrive + bulk-copy bytes)
   int32_t* cnt;     // [stage]: warps done with the stage's page (several n-tiles per page);
@@ -748,6 +752,20 @@ struct Page {
   static constexpr int HEAD = F == kFp8 ? 32 * D + 16 : (F == kTq3 ? 14 * D : 64 * D);
 };
 
+// One thread: (re)initialise the stage barriers and counters for a unit.  For a CTA's second
+// and later units the barriers are invalidated first: the previous unit waited for every copy
+// it issued and the CTA synchronised since, so none of them is in use.
+__device__ __forceinline__ void init_ring(const Smem& sm, bool again) {
+  for (int s = 0; s < kRingBarriers; ++s) {
+    if (again) mbar_inval(&sm.full[s]);
+    mbar_init(&sm.full[s], 1);
+    sm.cnt[s] = 0;
+    sm.fills[s] = 0;
+  }
+  sm.misc[1] = 0;
+  mbar_fence_init();
+}
+
 // Warp-collective: start the bulk copy of page i of the unit (list entry i) into its ring
 // stage.  FP8 and TQ3 pages are one contiguous copy issued by lane 0; a BF16 page is 32 row
 // copies, one per lane, into padded stage rows.
@@ -773,7 +791,7 @@ __device__ __forceinline__ void fill_stage(const Smem& sm, const uint8_t* slab, 
 
 template <int D, int NT, int K, int F>
 __device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDesc& u, int h,
-                         Smem sm) {
+                         Smem sm, bool again) {
   using C = Cfg<D, NT, K>;
   using PG = Page<D, NT, K, F>;
   constexpr int STAGE = PG::STAGE;
@@ -787,15 +805,7 @@ __device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDes
   const int64_t slot_bytes = F == kTq3 ? p.tq3_slot_bytes : p.fp8_slot_bytes;
   if (warp == SCANNER) {
     // the first fills are in flight while the other warps build their Q fragments
-    if (lane == 0) {
-      for (int s = 0; s < NST; ++s) {
-        mbar_init(&sm.full[s], 1);
-        sm.cnt[s] = 0;
-        sm.fills[s] = 0;
-      }
-      sm.misc[1] = 0;
-      mbar_fence_init();
-    }
+    if (lane == 0) init_ring(sm, again);
     __syncwarp();
     const int32_t* row = p.tables + static_cast<int64_t>(sd.row) * p.max_pages;
     const int n = scan_range(p, row, u.first, u.last, F, lane, sm.list);
@@ -997,7 +1007,7 @@ __device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDes
 // in the combine.
 template <int D, int NT, int K, int F>
 __device__ void run_unit_team(const DecodeParams& p, const SeqDesc& sd, const UnitDesc& u, int h,
-                              Smem sm) {
+                              Smem sm, bool again) {
   using C = Cfg<D, NT, K>;
   using PG = Page<D, NT, K, F>;
   constexpr int TW = C::TW, NST = PG::NST, STAGE = PG::STAGE;
@@ -1009,15 +1019,7 @@ __device__ void run_unit_team(const DecodeParams& p, const SeqDesc& sd, const Un
   const int64_t slot_bytes = F == kTq3 ? p.tq3_slot_bytes : p.fp8_slot_bytes;
 
   if (warp == TW - 1) {
-    if (lane == 0) {
-      for (int s = 0; s < NST; ++s) {
-        mbar_init(&sm.full[s], 1);
-        sm.cnt[s] = 0;
-        sm.fills[s] = 0;
-      }
-      sm.misc[1] = 0;
-      mbar_fence_init();
-    }
+    if (lane == 0) init_ring(sm, again);
     __syncwarp();
     const int32_t* row = p.tables + static_cast<int64_t>(sd.row) * p.max_pages;
     const int n = scan_range(p, row, u.first, u.last, F, lane, sm.list);
@@ -1139,7 +1141,10 @@ __device__ void run_unit_team(const DecodeParams& p, const SeqDesc& sd, const Un
     // the batch's probabilities are published; every warp of the team stops together on a
     // failed wait
     if (!barrier_and(1, 32 * TW, ok)) {
-      if (lane == 0) flag_status(p.status, kStatusTimeout);
+      if (lane == 0) {
+        flag_status(p.status, kStatusTimeout);
+        atomicExch(&sm.misc[1], 1);
+      }
       break;
     }
     // the previous batch's stages: every warp fenced its reads of them before this barrier, so
@@ -1388,8 +1393,38 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
   }
 }
 
-// Partial-attention kernel of one kind.  Grid = units x KV heads; the FP8 grid covers units
-// [0, n_fp8), the TQ3 grid [n_fp8, n_units), the fused and BF16 grids all of them.
+// Partial-attention kernel of one kind.  Grid = CTAs x KV heads: CTA c of KV head h takes
+// units [cta_unit0[c], cta_unit0[c+1]) one after another.  The FP8 grid covers CTAs
+// [0, n_fp8), the TQ3 grid [n_fp8, n_ctas), the fused and BF16 grids all of them.
+template <int D, int NT, int K>
+__device__ __forceinline__ void run_one(const DecodeParams& p, const UnitDesc& u, int h,
+                                        const Smem& sm, bool again) {
+  const SeqDesc& sd = p.seq[u.seq];
+  if constexpr (Cfg<D, NT, K>::TEAM) {
+    if constexpr (K == kKindFp8) {
+      run_unit_team<D, NT, K, kFp8>(p, sd, u, h, sm, again);
+    } else if constexpr (K == kKindTq3) {
+      run_unit_team<D, NT, K, kTq3>(p, sd, u, h, sm, again);
+    } else {
+      if (u.fmt == kFp8)
+        run_unit_team<D, NT, K, kFp8>(p, sd, u, h, sm, again);
+      else
+        run_unit_team<D, NT, K, kTq3>(p, sd, u, h, sm, again);
+    }
+  } else if constexpr (K == kKindFp8) {
+    run_unit<D, NT, K, kFp8>(p, sd, u, h, sm, again);
+  } else if constexpr (K == kKindTq3) {
+    run_unit<D, NT, K, kTq3>(p, sd, u, h, sm, again);
+  } else if constexpr (K == kKindBf16) {
+    run_unit<D, NT, K, kBf16>(p, sd, u, h, sm, again);
+  } else {
+    if (u.fmt == kFp8)
+      run_unit<D, NT, K, kFp8>(p, sd, u, h, sm, again);
+    else
+      run_unit<D, NT, K, kTq3>(p, sd, u, h, sm, again);
+  }
+}
+
 template <int D, int NT, int K>
 __global__ void __launch_bounds__(Cfg<D, NT, K>::THREADS, Cfg<D, NT, K>::MINB)
     partial_kernel(const __grid_constant__ DecodeParams p) {
@@ -1399,35 +1434,18 @@ __global__ void __launch_bounds__(Cfg<D, NT, K>::THREADS, Cfg<D, NT, K>::MINB)
   pdl_launch_dependents();
   const Smem sm = carve<D, NT, K>(smem_raw);
   const int h = blockIdx.x % p.Hkv;
-  const UnitDesc& u = p.unit[(K == kKindTq3 ? p.n_fp8 : 0) + blockIdx.x / p.Hkv];
-  const SeqDesc& sd = p.seq[u.seq];
-  if constexpr (Cfg<D, NT, K>::TEAM) {
-    if constexpr (K == kKindFp8) {
-      run_unit_team<D, NT, K, kFp8>(p, sd, u, h, sm);
-    } else if constexpr (K == kKindTq3) {
-      run_unit_team<D, NT, K, kTq3>(p, sd, u, h, sm);
-      pdl_wait();  // as below: the merge then sees both grids' partial states
-    } else {
-      if (u.fmt == kFp8)
-        run_unit_team<D, NT, K, kFp8>(p, sd, u, h, sm);
-      else
-        run_unit_team<D, NT, K, kTq3>(p, sd, u, h, sm);
-    }
-  } else if constexpr (K == kKindFp8) {
-    run_unit<D, NT, K, kFp8>(p, sd, u, h, sm);
-  } else if constexpr (K == kKindTq3) {
-    run_unit<D, NT, K, kTq3>(p, sd, u, h, sm);
-    // the TQ3 grid, a programmatic dependent of the FP8 grid, ends only after it: the merge, a
-    // dependent of this grid, then sees both grids' partial states
-    pdl_wait();
-  } else if constexpr (K == kKindBf16) {
-    run_unit<D, NT, K, kBf16>(p, sd, u, h, sm);
-  } else {
-    if (u.fmt == kFp8)
-      run_unit<D, NT, K, kFp8>(p, sd, u, h, sm);
-    else
-      run_unit<D, NT, K, kTq3>(p, sd, u, h, sm);
+  const int cta = (K == kKindTq3 ? p.n_fp8 : 0) + blockIdx.x / p.Hkv;
+  const int k0 = p.cta_unit0[cta], k1 = p.cta_unit0[cta + 1];
+  for (int k = k0; k < k1; ++k) {
+    run_one<D, NT, K>(p, p.unit[k], h, sm, k > k0);
+    // every warp is done with the unit's combine (which reuses the ring) before the next unit
+    // refills the ring
+    __syncthreads();
+    if (sm.misc[1]) break;  // a bounded wait ran out (status flagged): skip the rest
   }
+  // the TQ3 grid, a programmatic dependent of the FP8 grid, ends only after it: the merge, a
+  // dependent of this grid, then sees both grids' partial states
+  if constexpr (K == kKindTq3) pdl_wait();
 }
 
 // Per-instantiation launch set-up, done once: the dynamic shared-memory opt-in and the number of
@@ -1471,11 +1489,11 @@ cudaError_t launch_ex(void (*kernel)(Args...), dim3 grid, int threads, int smem,
 }
 
 template <int D, int NT, int K>
-cudaError_t launch_t(const DecodeParams& p, int n_units, bool dependent, cudaStream_t s) {
+cudaError_t launch_t(const DecodeParams& p, int n_ctas, bool dependent, cudaStream_t s) {
   using C = Cfg<D, NT, K>;
   const KernelInfo<D, NT, K>& info = KernelInfo<D, NT, K>::get();
   if (info.err != cudaSuccess) return info.err;
-  return launch_ex(partial_kernel<D, NT, K>, dim3(n_units * p.Hkv), C::THREADS, C::SMEM,
+  return launch_ex(partial_kernel<D, NT, K>, dim3(n_ctas * p.Hkv), C::THREADS, C::SMEM,
                    dependent, s, p);
 }
 
@@ -1490,23 +1508,23 @@ int ctas_per_sm_d(int nt) {
 }
 
 template <int D, int K>
-cudaError_t launch_d(const DecodeParams& p, int n_units, bool dependent, cudaStream_t s) {
+cudaError_t launch_d(const DecodeParams& p, int n_ctas, bool dependent, cudaStream_t s) {
   switch ((p.NC + 7) / 8) {
-    case 1: return launch_t<D, 1, K>(p, n_units, dependent, s);
-    case 2: return launch_t<D, 2, K>(p, n_units, dependent, s);
-    case 3: return launch_t<D, 3, K>(p, n_units, dependent, s);
-    case 4: return launch_t<D, 4, K>(p, n_units, dependent, s);
+    case 1: return launch_t<D, 1, K>(p, n_ctas, dependent, s);
+    case 2: return launch_t<D, 2, K>(p, n_ctas, dependent, s);
+    case 3: return launch_t<D, 3, K>(p, n_ctas, dependent, s);
+    case 4: return launch_t<D, 4, K>(p, n_ctas, dependent, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
 template <int K>
-cudaError_t launch_kind(const DecodeParams& p, int n_units, bool dependent, cudaStream_t s) {
-  if (n_units <= 0) return cudaSuccess;
+cudaError_t launch_kind(const DecodeParams& p, int n_ctas, bool dependent, cudaStream_t s) {
+  if (n_ctas <= 0) return cudaSuccess;
   switch (p.D) {
-    case 64: return launch_d<64, K>(p, n_units, dependent, s);
-    case 128: return launch_d<128, K>(p, n_units, dependent, s);
-    case 256: return launch_d<256, K>(p, n_units, dependent, s);
+    case 64: return launch_d<64, K>(p, n_ctas, dependent, s);
+    case 128: return launch_d<128, K>(p, n_ctas, dependent, s);
+    case 256: return launch_d<256, K>(p, n_ctas, dependent, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -1548,18 +1566,23 @@ cudaError_t launch_merge(const DecodeParams& p, cudaStream_t s) {
   int nsub = groups >= 32 ? 1 : 32 / groups;
   while (nsub < want && 2 * nsub * groups <= kMergeThreads) nsub *= 2;
   return launch_ex(merge_kernel, dim3(p.n_seqs * p.Hkv * p.NC), nsub * groups, 0,
-                   p.n_units > 0, s, p);
+                   p.n_ctas > 0, s, p);
 }
 
-// Split: the FP8 grid (units [0, n_fp8)), then the TQ3 grid as its programmatic dependent, so
+// Split: the FP8 grid (CTAs [0, n_fp8)), then the TQ3 grid as its programmatic dependent, so
 // the TQ3 CTAs fill the SM room the FP8 CTAs leave in the same wave.  Fused: one grid over all
-// units.  The first partial grid waits for everything before it.
+// CTAs.  The first partial grid waits for everything before it.
 cudaError_t launch_partial(const DecodeParams& p, cudaStream_t s) {
-  if (p.n_units <= 0) return cudaSuccess;
-  if (p.page_fmt == kBf16) return launch_kind<kKindBf16>(p, p.n_units, false, s);
-  if (p.fused) return launch_kind<kKindFused>(p, p.n_units, false, s);
+  if (p.n_ctas <= 0) return cudaSuccess;
+  if (p.n_ctas > kDecodeMaxUnits || p.n_fp8 < 0 || p.n_fp8 > p.n_ctas ||
+      p.cta_unit0[0] != 0 || p.cta_unit0[p.n_ctas] != p.n_units || p.n_units > kDecodeMaxUnits)
+    return cudaErrorInvalidValue;
+  for (int c = 0; c < p.n_ctas; ++c)
+    if (p.cta_unit0[c + 1] <= p.cta_unit0[c]) return cudaErrorInvalidValue;
+  if (p.page_fmt == kBf16) return launch_kind<kKindBf16>(p, p.n_ctas, false, s);
+  if (p.fused) return launch_kind<kKindFused>(p, p.n_ctas, false, s);
   cudaError_t e = launch_kind<kKindFp8>(p, p.n_fp8, false, s);
-  if (e == cudaSuccess) e = launch_kind<kKindTq3>(p, p.n_units - p.n_fp8, p.n_fp8 > 0, s);
+  if (e == cudaSuccess) e = launch_kind<kKindTq3>(p, p.n_ctas - p.n_fp8, p.n_fp8 > 0, s);
   return e;
 }
 

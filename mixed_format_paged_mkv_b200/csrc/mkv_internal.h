@@ -122,11 +122,12 @@ struct MaterialiseParams {
 };
 
 // ------------------------------------------------------------------ decode
-// Decode = partial kernel + merge kernel.  Work unit = (sequence, format, logical page range);
-// a partial CTA takes one (unit, KV head): it scans the block-table entries of its range,
-// streams the pages of its format through a shared-memory ring and writes one partial state
-// per query column.  The merge kernel combines every partial state of a (sequence, KV head,
-// column).
+// Decode = partial kernel + merge kernel.  Work unit = (sequence, format, logical page range).
+// A partial CTA takes a run of consecutive units for one KV head: for each it scans the
+// block-table entries of the range, streams the pages of its format through a shared-memory
+// ring and writes one partial state per query column.  The units of a CTA are cut from a line
+// of all sequences' pages of its grid, so a CTA may finish one sequence and start the next.
+// The merge kernel combines every partial state of a (sequence, KV head, column).
 struct SeqDesc {
   int32_t row;      // table row (sequence id)
   int32_t ctx;      // context length L (includes the q_len new tokens)
@@ -138,13 +139,14 @@ struct SeqDesc {
 struct UnitDesc {
   int32_t first;  // logical pages [first, last)
   int32_t last;
-  int16_t seq;    // index into DecodeParams::seq
-  int16_t fmt;    // 0 FP8, 1 TQ3
-  int32_t part;   // index of this unit's partial state within its sequence
+  uint8_t seq;    // index into DecodeParams::seq
+  uint8_t fmt;    // 0 FP8, 1 TQ3, 2 BF16
+  uint16_t part;  // index of this unit's partial state within its sequence
 };
 constexpr int kDecodeMaxSeqs = 256;
 constexpr int kDecodeMaxUnits = 1536;
 constexpr int kMaxPagesPerUnit = 512;  // pages of the unit's format inside its range
+static_assert(kDecodeMaxSeqs <= 256 && kDecodeMaxUnits <= 65535, "UnitDesc field widths");
 struct DecodeParams {
   const uint8_t* fp8_slab;
   const uint8_t* tq3_slab;
@@ -159,12 +161,14 @@ struct DecodeParams {
   int32_t max_pages, fp8_slots, tq3_slots;
   float logit_scale;  // sm_scale * log2(e)
   int32_t n_seqs;     // sequences in this launch
-  int32_t n_units;    // units in this launch: FP8 units [0, n_fp8), then TQ3 units
-  int32_t n_fp8;      // (the fused kernel takes every unit in one grid of n_units * Hkv CTAs)
+  int32_t n_units;    // units in this launch, CTA by CTA
+  int32_t n_ctas;     // CTAs per KV head: FP8 CTAs [0, n_fp8), then TQ3 CTAs (per-format
+  int32_t n_fp8;      // grids); the fused and BF16 grids take all n_ctas x Hkv CTAs
   int32_t fused;      // 1: one grid branching per unit; 0: an FP8 grid, then a TQ3 grid
   int32_t page_fmt;   // format of written pages: 0 FP8 (mixed pools), 2 BF16 (control pools)
   SeqDesc seq[kDecodeMaxSeqs];
   UnitDesc unit[kDecodeMaxUnits];
+  uint16_t cta_unit0[kDecodeMaxUnits + 1];  // CTA c takes units [cta_unit0[c], cta_unit0[c+1])
 };
 
 // Every parameter block fits the 32,764-byte kernel-parameter limit.

@@ -140,12 +140,11 @@ bool valid_pool(mkv_pool_t p) { return p != nullptr; }
 constexpr int64_t kFp8PageCost = 11;
 constexpr int64_t kTq3PageCost = 10;
 // Automatic choice of partial kernels: one fused grid when FP8 pages carry more than this share
-// of the call's planned time, or when the FP8 grid alone would hold more than one CTA per SM
-// (many sequences, each with its own FP8 units: 64 sequences x 8 KV heads at D 128 decode in
-// 604 us fused against 631 us per format, with 0.9% of the pages FP8).  Measured on the long-context workload: at 4% FP8 pages the
+// of the call's planned time.  Measured on the long-context workload: at 4% FP8 pages the
 // per-format grids are faster (150.8 against 156.3 us), at 25% the fused grid (170.0 against
 // 198.8 us): FP8 CTAs need more shared memory than TQ3 CTAs, so beyond one FP8 CTA per SM the
-// per-format grids no longer fit one wave.
+// per-format grids no longer fit one wave.  (The FP8 grid gets CTAs in proportion to its cost,
+// so below this share it holds fewer CTAs than there are SMs.)
 constexpr double kFusedAboveFp8Share = 0.15;
 
 // SMs a decode call's cut is planned for: the device's, or fewer when the caller asked so.
@@ -159,19 +158,16 @@ int decode_mode(const mkv_pool* p, const int32_t* seq_ids, int32_t n, int32_t NC
   if (p->page_fmt == MKV_FMT_BF16) return kDecodeBf16;
   if (p->decode_kernels != MKV_DECODE_AUTO)
     return p->decode_kernels == MKV_DECODE_FUSED ? kDecodeFused : kDecodeSplit;
-  int64_t c8 = 0, c3 = 0, groups8 = 0;
+  int64_t c8 = 0, c3 = 0;
   for (int32_t i = 0; i < n; ++i) {
     const Seq& s = p->seqs[seq_ids[i]];
     c8 += static_cast<int64_t>(s.fp8_pages.size()) * kFp8PageCost;
     c3 += static_cast<int64_t>(s.n3) * kTq3PageCost;
-    groups8 += s.fp8_pages.empty() ? 0 : 1;
   }
   // the fused grid keeps as many CTAs per SM as the TQ3 grid (D 64 and 128): one grid is enough
   const int D = p->cfg.head_dim;
   if (partial_ctas_per_sm(D, NC, kDecodeFused) >= partial_ctas_per_sm(D, NC, kDecodeSplit))
     return kDecodeFused;
-  // every sequence with FP8 pages gives the FP8 grid at least one CTA per KV head
-  if (groups8 * p->cfg.num_kv_heads > plan_sms(p)) return kDecodeFused;
   return c8 > kFusedAboveFp8Share * static_cast<double>(c8 + c3) ? kDecodeFused : kDecodeSplit;
 }
 
@@ -226,117 +222,174 @@ cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 // Device status buffer: the status word (padded to 256 bytes).
 size_t status_bytes(const mkv_pool_config&) { return 256; }
 
+struct LaunchDesc {
+  int32_t s0 = 0, s1 = 0;   // call positions [s0, s1)
+  int32_t u0 = 0, u1 = 0;   // units [u0, u1) of DecodePlan::unit, CTA by CTA
+  int32_t n_ctas = 0;       // CTAs per KV head
+  int32_t n_fp8 = 0;        // of which FP8 CTAs (per-format grids), the first ones
+};
+
 struct DecodePlan {
   int32_t NC = 0, g = 0;
-  int mode = kDecodeSplit;     // partial kernels of the call
-  std::vector<SeqDesc> seq;    // per call position
-  std::vector<UnitDesc> unit;  // per sequence, in order
-  std::vector<int32_t> pos;    // call position of each unit's sequence
-  std::vector<int64_t> cost;   // relative time of each unit (per KV head)
+  int mode = kDecodeSplit;         // partial kernels of the call
+  std::vector<SeqDesc> seq;        // per call position
+  std::vector<UnitDesc> unit;      // launch by launch, CTA by CTA
+  std::vector<int32_t> pos;        // call position of each unit's sequence
+  std::vector<int32_t> cta;        // CTA of each unit within its launch
+  std::vector<int64_t> cost;       // relative time of each unit (per KV head)
+  std::vector<LaunchDesc> launch;
   int64_t parts = 0;
   size_t off_ml = 0, off_acc = 0, bytes = 0;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Work-unit cut shared by both decode entry points (no allocation).  A unit is one format's
-// pages inside a logical page range of one sequence; the partial kernel runs one CTA per (unit,
-// KV head).  Units are cut for a single wave: at most SMs x resident CTAs per SM CTAs, each
-// (sequence, format) group split into equal parts, and the unit cost chosen as the smallest that
-// fits that budget, so the longest CTA, which ends the wave, is as short as the groups allow.
-// A single balanced wave measured faster than several smaller ones: each CTA sets up and
-// combines its warps once and no partial last wave is left.  Units hold at most
-// kMaxPagesPerUnit and at least a few pages.  `emit(unit, cost, pos)` is called in sequence
-// order, pos the sequence's call position (UnitDesc::seq is left 0: it is the position within
-// one launch, set when the units are grouped); UnitDesc::part numbers the units of a sequence.  Returns the unit count, or -1 as soon as
-// `emit` returns false.
+// Work-unit cut shared by both decode entry points (no allocation).  A launch runs one grid per
+// page format (or one fused grid) of CTAs x KV heads, sized for a single wave: at most
+// SMs x resident CTAs per SM.  A grid's pages -- every sequence's pages of its format, in call
+// order -- form one line, cut into CTAs of equal cost; a CTA takes the pieces of the sequences
+// its share of the line touches, one unit each (a unit is one format's pages inside a logical
+// page range of one sequence, and yields one partial state).  So the longest CTA, which ends
+// the wave, is within a few pages of the average however unequal the sequences are.  A single
+// balanced wave measured faster than several smaller ones: each CTA sets up and combines its
+// warps once per unit and no partial last wave is left.  Cut points that would leave a unit of
+// fewer than a few pages move to the sequence's edge; a unit holds at most kMaxPagesPerUnit
+// pages.  Pages are weighted by measured time per CTA (FP8 11, TQ3 10), not by bytes.
 constexpr int kMinTq3PagesPerUnit = 8;
 constexpr int kMinFp8PagesPerUnit = 4;
 
+// Pages of format slot f (0: FP8 or BF16, 1: TQ3) of a sequence.
+inline int64_t group_pages(const Seq& s, int f) {
+  return f == 0 ? static_cast<int64_t>(s.fp8_pages.size()) : static_cast<int64_t>(s.n3);
+}
+
+// Cut one line -- the pages of the format slots in `fmts` (bit f) of call positions [s0, s1),
+// in order -- into at most k CTAs of equal cost, numbered from *n_ctas on.  emit(unit, cost,
+// pos, cta) is called CTA by CTA; n_parts[pos] counts each sequence's units (their part
+// indices).  Returns false as soon as emit does.
 template <class Emit>
-int64_t cut_units(const mkv_pool* p, const int32_t* seq_ids, int32_t n, int32_t NC, int mode,
-                  int32_t* n_parts, Emit&& emit) {
-  const int64_t b8 = kFp8PageCost, b3 = kTq3PageCost;
-  const int Hkv = p->cfg.num_kv_heads;
-  int64_t total = 0;
-  for (int32_t i = 0; i < n; ++i) {
+bool cut_line(const mkv_pool* p, const int32_t* seq_ids, int32_t s0, int32_t s1, unsigned fmts,
+              int64_t k, int32_t* n_parts, int32_t* n_ctas, Emit&& emit) {
+  const int64_t b[2] = {kFp8PageCost, kTq3PageCost};
+  const int64_t m[2] = {kMinFp8PagesPerUnit, kMinTq3PagesPerUnit};
+  int64_t T = 0, pages = 0;
+  for (int32_t i = s0; i < s1; ++i)
+    for (int f = 0; f < 2; ++f)
+      if (fmts >> f & 1) {
+        const int64_t n = group_pages(p->seqs[seq_ids[i]], f);
+        T += n * b[f];
+        pages += n;
+      }
+  if (T == 0 || k <= 0) return true;
+  // pieces of at least a few pages each
+  k = std::max<int64_t>(1, std::min<int64_t>(k, pages / ((fmts & 2) ? m[1] : m[0])));
+  int64_t j = 0;        // current piece
+  int64_t owner = -1;   // the piece that last took a CTA number
+  int64_t G0 = 0;       // line position (cost) of the current group's first page
+  for (int32_t i = s0; i < s1; ++i) {
     const Seq& s = p->seqs[seq_ids[i]];
-    total += static_cast<int64_t>(s.fp8_pages.size()) * b8 + static_cast<int64_t>(s.n3) * b3;
+    const std::vector<int32_t>& f8 = s.fp8_pages;
+    const int64_t n8 = static_cast<int64_t>(f8.size());
+    const int32_t table = static_cast<int32_t>(s.table.size());
+    for (int f = 0; f < 2; ++f) {
+      if (!(fmts >> f & 1)) continue;
+      const int64_t n = group_pages(s, f);
+      if (n == 0) continue;
+      const int64_t G1 = G0 + n * b[f];
+      int64_t c8 = 0;  // FP8 pages before the current TQ3 page (logical = TQ3 number + c8)
+      auto logical = [&](int64_t t) {  // logical page of TQ3 page number t (t < n)
+        while (c8 < n8 && f8[c8] <= t + c8) ++c8;
+        return static_cast<int32_t>(t + c8);
+      };
+      auto put = [&](int64_t a, int64_t e) -> bool {  // pages [a, e) of this group, piece j
+        if (owner != j) {
+          owner = j;
+          ++*n_ctas;
+        }
+        const int64_t parts = (e - a + kMaxPagesPerUnit - 1) / kMaxPagesPerUnit;
+        for (int64_t q = 0; q < parts; ++q) {
+          const int64_t u0 = a + q * (e - a) / parts, u1 = a + (q + 1) * (e - a) / parts;
+          UnitDesc u{};
+          if (f == 0) {
+            u.first = f8[u0];
+            u.last = f8[u1 - 1] + 1;
+            u.fmt = static_cast<uint8_t>(p->page_fmt);
+          } else {
+            // TQ3 ranges tile the table: the first starts at page 0, the last ends at its end,
+            // each other one at the logical page of its first TQ3 page
+            u.first = u0 == 0 ? 0 : logical(u0);
+            u.last = u1 == n ? table : logical(u1);
+            u.fmt = 1;
+          }
+          u.part = static_cast<uint16_t>(std::min<int32_t>(n_parts[i], 65535));
+          ++n_parts[i];
+          if (!emit(u, (u1 - u0) * b[f], i, *n_ctas - 1)) return false;
+        }
+        return true;
+      };
+      int64_t a = 0;
+      while (a < n) {
+        const int64_t x = j + 1 < k ? T * (j + 1) / k : T;  // where piece j ends on the line
+        if (x >= G1) {  // piece j takes the rest of the group
+          if (!put(a, n)) return false;
+          a = n;
+          break;
+        }
+        // piece j ends inside the group: nearest page boundary, moved so that no unit of this
+        // group is shorter than m pages where the group allows
+        int64_t e = x <= G0 ? 0 : (x - G0 + b[f] / 2) / b[f];
+        e = std::max(a, std::min(e, n));
+        if (e > a && e - a < m[f]) e = a == 0 ? 0 : std::min(n, a + m[f]);
+        if (e < n && n - e < m[f]) e = n;
+        if (e > a && !put(a, e)) return false;
+        a = e;
+        ++j;
+      }
+      G0 = G1;
+    }
   }
+  return true;
+}
+
+// Units of one launch (call positions [s0, s1)): the wave's CTAs shared by the grids in
+// proportion to their cost.  Returns false when emit does.
+template <class Emit>
+bool cut_launch(const mkv_pool* p, const int32_t* seq_ids, int32_t s0, int32_t s1, int32_t NC,
+                int mode, int32_t* n_parts, LaunchDesc* ld, Emit&& emit) {
+  const int Hkv = p->cfg.num_kv_heads;
   const int64_t slots =
       static_cast<int64_t>(plan_sms(p)) * partial_ctas_per_sm(p->cfg.head_dim, NC, mode);
-  const int64_t U = std::max<int64_t>(1, slots / Hkv);
-  // units of a group at unit cost c: as many as its cost needs, clamped to the page limits
-  auto units_at = [](double c, int64_t cost, int64_t pages, int min_pages) -> int64_t {
-    const int64_t lo = (pages + kMaxPagesPerUnit - 1) / kMaxPagesPerUnit;
-    const int64_t hi = std::max<int64_t>(lo, std::max<int64_t>(1, pages / min_pages));
-    const int64_t u = static_cast<int64_t>(std::ceil(static_cast<double>(cost) / c - 1e-9));
-    return std::max(lo, std::min(std::max<int64_t>(u, 1), hi));
-  };
-  auto count_at = [&](double c) -> int64_t {
-    int64_t sum = 0;
-    for (int32_t i = 0; i < n; ++i) {
-      const Seq& s = p->seqs[seq_ids[i]];
-      const int64_t n8 = static_cast<int64_t>(s.fp8_pages.size()), n3 = s.n3;
-      if (n8 > 0) sum += units_at(c, n8 * b8, n8, kMinFp8PagesPerUnit);
-      if (n3 > 0) sum += units_at(c, n3 * b3, n3, kMinTq3PagesPerUnit);
-    }
-    return sum;
-  };
-  // smallest unit cost whose cut needs at most U units (the largest unit bounds the wave)
-  double lo_c = std::max(1.0, static_cast<double>(total) / U), hi_c = lo_c;
-  while (count_at(hi_c) > U && hi_c < 4.0 * total) hi_c *= 2.0;
-  for (int it = 0; it < 40 && hi_c - lo_c > 0.5; ++it) {
-    const double mid = 0.5 * (lo_c + hi_c);
-    (count_at(mid) <= U ? hi_c : lo_c) = mid;
-  }
-  const double unit_cost = hi_c;
-  int64_t nu = 0;
-  for (int32_t i = 0; i < n; ++i) {
+  int64_t U = std::max<int64_t>(1, slots / Hkv);
+  int64_t c8 = 0, c3 = 0, bound = 0;
+  for (int32_t i = s0; i < s1; ++i) {
     const Seq& s = p->seqs[seq_ids[i]];
-    int32_t np = 0;
-    const auto& f8 = s.fp8_pages;
-    const int64_t n8 = static_cast<int64_t>(f8.size());
-    if (n8 > 0) {
-      const int64_t u = units_at(unit_cost, n8 * b8, n8, kMinFp8PagesPerUnit);
-      for (int64_t k = 0; k < u; ++k) {
-        const int64_t j0 = k * n8 / u, j1 = (k + 1) * n8 / u;
-        if (j1 <= j0) continue;
-        if (!emit(UnitDesc{f8[j0], f8[j1 - 1] + 1, 0, static_cast<int16_t>(p->page_fmt), np++},
-                  (j1 - j0) * b8, i))
-          return -1;
-        ++nu;
-      }
+    for (int f = 0; f < 2; ++f) {
+      const int64_t n = group_pages(s, f);
+      (f == 0 ? c8 : c3) += n * (f == 0 ? kFp8PageCost : kTq3PageCost);
+      // units beyond one per CTA: one more per group a cut crosses, and the 512-page splits
+      if (n > 0) bound += 1 + n / kMaxPagesPerUnit;
     }
-    const int64_t n3 = s.n3;
-    if (n3 > 0) {
-      const int64_t u = units_at(unit_cost, n3 * b3, n3, kMinTq3PagesPerUnit);
-      // unit k takes TQ3 pages number [k n3 / u, (k+1) n3 / u) in logical order; its range
-      // starts at the logical page of its first TQ3 page (the first unit at page 0) and ends
-      // where the next one starts (the last at the end of the table).  Every page of the table
-      // is FP8 or TQ3, so TQ3 page number j sits at logical page j + c, c the number of FP8
-      // pages before it: one merge over the ascending FP8 list finds all boundaries, without
-      // walking the table.
-      const int32_t pages = static_cast<int32_t>(s.table.size());
-      int64_t c = 0;
-      int32_t start = 0;
-      for (int64_t k = 0; k < u; ++k) {
-        const int64_t j0 = k * n3 / u, j1 = (k + 1) * n3 / u;
-        int32_t end = pages;
-        if (k + 1 < u) {
-          while (c < n8 && f8[c] <= j1 + c) ++c;
-          end = static_cast<int32_t>(j1 + c);
-        }
-        if (j1 > j0) {
-          if (!emit(UnitDesc{start, end, 0, 1, np++}, (j1 - j0) * b3, i)) return -1;
-          ++nu;
-        }
-        start = end;
-      }
-    }
-    n_parts[i] = np;
   }
-  return nu;
+  // the launch's units fit the parameter block: units <= CTAs + bound
+  U = std::max<int64_t>(1, std::min<int64_t>(U, kDecodeMaxUnits - 2 - bound));
+  ld->s0 = s0;
+  ld->s1 = s1;
+  ld->n_ctas = 0;
+  ld->n_fp8 = 0;
+  if (mode == kDecodeSplit) {
+    int64_t k8 = 0, k3 = 0;
+    if (c8 > 0 && c3 > 0) {
+      k8 = std::llround(static_cast<double>(U) * c8 / static_cast<double>(c8 + c3));
+      k8 = std::max<int64_t>(1, std::min<int64_t>(k8, U - 1));
+      k3 = std::max<int64_t>(1, U - k8);
+    } else {
+      (c8 > 0 ? k8 : k3) = U;
+    }
+    if (!cut_line(p, seq_ids, s0, s1, 1u, k8, n_parts, &ld->n_ctas, emit)) return false;
+    ld->n_fp8 = ld->n_ctas;
+    return cut_line(p, seq_ids, s0, s1, 2u, k3, n_parts, &ld->n_ctas, emit);
+  }
+  return cut_line(p, seq_ids, s0, s1, 3u, U, n_parts, &ld->n_ctas, emit);
 }
 
 int plan_decode(mkv_pool_t p, const int32_t* seq_ids, int32_t n, int32_t q_len, int32_t Hq,
@@ -356,24 +409,37 @@ int plan_decode(mkv_pool_t p, const int32_t* seq_ids, int32_t n, int32_t q_len, 
     const Seq& s = p->seqs[seq_ids[i]];
     if (s.ctx < q_len || s.ctx == 0)
       return fail(MKV_ERR_EMPTY_CONTEXT, "sequence %d has %d tokens < q_len %d", seq_ids[i], s.ctx, q_len);
+    if (group_pages(s, 0) > static_cast<int64_t>(kMaxPagesPerUnit) * kDecodeMaxUnits ||
+        group_pages(s, 1) > static_cast<int64_t>(kMaxPagesPerUnit) * kDecodeMaxUnits)
+      return fail(MKV_ERR_UNSUPPORTED, "sequence %d has more than %d pages of one format",
+                  seq_ids[i], kMaxPagesPerUnit * kDecodeMaxUnits);
   }
   plan->seq.resize(n);
   plan->unit.clear();
   plan->pos.clear();
+  plan->cta.clear();
   plan->cost.clear();
-  std::vector<int32_t> np(n);
+  plan->launch.clear();
+  std::vector<int32_t> np(n, 0);
   plan->mode = decode_mode(p, seq_ids, n, plan->NC);
-  cut_units(p, seq_ids, n, plan->NC, plan->mode, np.data(),
-            [&](const UnitDesc& u, int64_t cost, int32_t i) {
-    plan->unit.push_back(u);
-    plan->pos.push_back(i);
-    plan->cost.push_back(cost);
-    return true;
-  });
-  for (int32_t i = 0; i < n; ++i)
-    if (np[i] > kDecodeMaxUnits)
-      return fail(MKV_ERR_UNSUPPORTED, "sequence %d needs %d work units; one launch holds %d",
-                  seq_ids[i], np[i], kDecodeMaxUnits);
+  // launches over groups of at most kDecodeMaxSeqs whole sequences, one wave each
+  for (int32_t s0 = 0; s0 < n; s0 += kDecodeMaxSeqs) {
+    LaunchDesc ld;
+    ld.u0 = static_cast<int32_t>(plan->unit.size());
+    cut_launch(p, seq_ids, s0, std::min(n, s0 + kDecodeMaxSeqs), plan->NC, plan->mode,
+               np.data(), &ld, [&](const UnitDesc& u, int64_t cost, int32_t i, int32_t cta) {
+      plan->unit.push_back(u);
+      plan->pos.push_back(i);
+      plan->cta.push_back(cta);
+      plan->cost.push_back(cost);
+      return true;
+    });
+    ld.u1 = static_cast<int32_t>(plan->unit.size());
+    if (ld.u1 - ld.u0 > kDecodeMaxUnits)
+      return fail(MKV_ERR_UNSUPPORTED, "a launch needs %d work units; one holds %d",
+                  ld.u1 - ld.u0, kDecodeMaxUnits);
+    plan->launch.push_back(ld);
+  }
   int64_t parts = 0;
   for (int32_t i = 0; i < n; ++i) {
     SeqDesc& d = plan->seq[i];
@@ -394,6 +460,24 @@ int plan_decode(mkv_pool_t p, const int32_t* seq_ids, int32_t n, int32_t q_len, 
   return MKV_OK;
 }
 
+// Fill a launch's CTA table from the CTA number of each of its units (units come CTA by CTA).
+// Returns false when the units are not in CTA order or a CTA has none.
+bool fill_cta_table(DecodeParams* prm, const int32_t* cta, int32_t nu, int32_t n_ctas) {
+  if (n_ctas < 0 || n_ctas > kDecodeMaxUnits || nu > kDecodeMaxUnits) return false;
+  int32_t c = -1;
+  for (int32_t k = 0; k < nu; ++k) {
+    if (cta[k] == c) continue;
+    if (cta[k] != c + 1) return false;
+    c = cta[k];
+    prm->cta_unit0[c] = static_cast<uint16_t>(k);
+  }
+  if (c + 1 != n_ctas) return false;
+  prm->cta_unit0[n_ctas] = static_cast<uint16_t>(nu);
+  prm->n_units = nu;
+  prm->n_ctas = n_ctas;
+  return true;
+}
+
 // Every device operation of a state-changing call (kernel launch or memset) goes through here:
 // the test hook can make it fail, host-only pools skip it, and launches are counted.  The calls
 // stage their host-state changes and commit them only after all their device operations were
@@ -409,20 +493,6 @@ int device_op(mkv_pool_t p, const char* what, F&& f) {
   ++p->launches;
   const cudaError_t e = f();
   return e == cudaSuccess ? MKV_OK : cuda_fail(e, what);
-}
-
-// Launch order of a group's units: largest cost first; with per-format grids the FP8 units
-// (first grid) before the TQ3 units (second grid).  Returns the FP8 unit count.
-template <class Fmt, class Cost>
-int32_t order_units(int32_t* order, int32_t n, bool fused, Fmt&& fmt, Cost&& cost) {
-  for (int32_t k = 0; k < n; ++k) order[k] = k;
-  std::sort(order, order + n, [&](int32_t x, int32_t y) {
-    if (!fused && fmt(x) != fmt(y)) return fmt(x) < fmt(y);  // FP8 (0) first
-    return cost(x) != cost(y) ? cost(x) > cost(y) : x < y;
-  });
-  int32_t n8 = 0;
-  for (int32_t k = 0; k < n; ++k) n8 += fmt(k) == 0 ? 1 : 0;
-  return fused ? 0 : n8;
 }
 
 cudaEvent_t get_event(mkv_pool_t p) {
@@ -733,15 +803,19 @@ int mkv_decode_plan(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, int32_
     *ctas_per_wave = plan_sms(p) * partial_ctas_per_sm(p->cfg.head_dim, plan.NC, plan.mode);
   if (!units_out) return ok();  // count query
   if (nu > cap) return fail(MKV_ERR_INVALID_ARG, "%lld units do not fit in %d", (long long)nu, cap);
-  const int64_t b[2] = {kFp8PageCost, kTq3PageCost};
-  for (int64_t k = 0; k < nu; ++k) {
-    const UnitDesc& u = plan.unit[k];
-    int32_t* o = units_out + 5 * k;
-    o[0] = plan.pos[k];
-    o[1] = u.fmt;
-    o[2] = u.first;
-    o[3] = u.last;
-    o[4] = static_cast<int32_t>(plan.cost[k] / b[u.fmt]);
+  int32_t cta0 = 0;
+  for (const LaunchDesc& ld : plan.launch) {
+    for (int32_t k = ld.u0; k < ld.u1; ++k) {
+      const UnitDesc& u = plan.unit[k];
+      int32_t* o = units_out + 6 * k;
+      o[0] = plan.pos[k];
+      o[1] = u.fmt;
+      o[2] = u.first;
+      o[3] = u.last;
+      o[4] = static_cast<int32_t>(plan.cost[k] / (u.fmt == 1 ? kTq3PageCost : kFp8PageCost));
+      o[5] = cta0 + plan.cta[k];
+    }
+    cta0 += ld.n_ctas;
   }
   return ok();
 }
@@ -789,46 +863,28 @@ int mkv_decode_attention(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, i
     for (auto& e : rec.ev)
       if (!(e = get_event(p))) timed = false;
   cudaError_t err = timed ? cudaEventRecord(rec.ev[0], st) : cudaSuccess;
-  // launches over groups of whole sequences, each within the parameter-block limits
-  size_t u0 = 0;
-  int32_t s0 = 0;
-  std::vector<int32_t> order;
-  while (s0 < n_seqs && err == cudaSuccess) {
-    int32_t s1 = s0;
-    size_t u1 = u0;
-    while (s1 < n_seqs && s1 - s0 < kDecodeMaxSeqs) {
-      size_t ue = u1;
-      while (ue < plan.unit.size() && plan.pos[ue] == s1) ++ue;
-      if (ue - u0 > static_cast<size_t>(kDecodeMaxUnits) && s1 > s0) break;
-      if (ue - u0 > static_cast<size_t>(kDecodeMaxUnits)) {
-        err = cudaErrorInvalidValue;
-        break;
-      }
-      u1 = ue;
-      ++s1;
+  // one launch (partial grids + merge) per group of whole sequences
+  for (size_t li = 0; li < plan.launch.size() && err == cudaSuccess; ++li) {
+    const LaunchDesc& ld = plan.launch[li];
+    for (int32_t i = ld.s0; i < ld.s1; ++i) prm->seq[i - ld.s0] = plan.seq[i];
+    const int32_t nu = ld.u1 - ld.u0;
+    for (int32_t k = 0; k < nu; ++k) {
+      prm->unit[k] = plan.unit[ld.u0 + k];
+      prm->unit[k].seq = static_cast<uint8_t>(plan.pos[ld.u0 + k] - ld.s0);
     }
-    if (err != cudaSuccess) break;
-    for (int32_t i = s0; i < s1; ++i) prm->seq[i - s0] = plan.seq[i];
-    order.resize(u1 - u0);
-    prm->n_fp8 = order_units(
-        order.data(), static_cast<int32_t>(order.size()), plan.mode != kDecodeSplit,
-        [&](int32_t k) { return static_cast<int>(plan.unit[u0 + k].fmt); },
-        [&](int32_t k) { return plan.cost[u0 + k]; });
-    for (size_t k = 0; k < order.size(); ++k) {
-      prm->unit[k] = plan.unit[u0 + order[k]];
-      prm->unit[k].seq = static_cast<int16_t>(plan.pos[u0 + order[k]] - s0);
+    if (!fill_cta_table(prm, plan.cta.data() + ld.u0, nu, ld.n_ctas)) {
+      err = cudaErrorInvalidValue;
+      break;
     }
-    prm->n_seqs = s1 - s0;
-    prm->n_units = static_cast<int32_t>(order.size());
+    prm->n_fp8 = plan.mode == kDecodeSplit ? ld.n_fp8 : 0;
+    prm->n_seqs = ld.s1 - ld.s0;
     prm->fused = plan.mode == kDecodeFused ? 1 : 0;
     prm->page_fmt = p->page_fmt;
-    const bool last = s1 >= n_seqs;
+    const bool last = li + 1 == plan.launch.size();
     err = launch_partial(*prm, st);
     ++p->launches;
     if (timed && last && err == cudaSuccess) err = cudaEventRecord(rec.ev[1], st);
     if (err == cudaSuccess) err = launch_merge(*prm, st), ++p->launches;
-    s0 = s1;
-    u0 = u1;
   }
   if (timed && err == cudaSuccess) err = cudaEventRecord(rec.ev[2], st);
   delete prm;
@@ -843,15 +899,6 @@ int mkv_decode_attention(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs, i
 // Decode with the library's static partial-state scratch instead of a caller workspace.  Same
 // units, order and kernels as mkv_decode_attention (so the same results), planned into a
 // parameter block on the stack: no device allocation and, on success, no host allocation.
-namespace {
-struct NoAllocPlan {
-  DecodeParams prm;
-  int64_t cost[kDecodeMaxUnits];
-  UnitDesc unit[kDecodeMaxUnits];
-  int32_t order[kDecodeMaxUnits];
-};
-}  // namespace
-
 int mkv_decode_attention_noalloc(mkv_pool_t p, const int32_t* seq_ids, int32_t n_seqs,
                                  int32_t q_len, const void* q_bf16, int32_t Hq, float sm_scale,
                                  float* out, void* stream) {
@@ -877,21 +924,25 @@ int mkv_decode_attention_noalloc(mkv_pool_t p, const int32_t* seq_ids, int32_t n
   }
   if (n_seqs == 0) return ok();
   if (!q_bf16 || !out) return fail(MKV_ERR_INVALID_ARG, "q/out is NULL");
-  NoAllocPlan t;  // about 75 KB of stack
-  DecodeParams& prm = t.prm;
-  int32_t np[kDecodeMaxSeqs];
-  int32_t nu = 0;
-  auto keep = [&](const UnitDesc& u, int64_t cost, int32_t i) {
-    if (nu >= kDecodeMaxUnits) return false;
-    t.unit[nu] = u;
-    t.unit[nu].seq = static_cast<int16_t>(i);  // n_seqs <= kDecodeMaxSeqs: one launch
-    t.cost[nu++] = cost;
+  DecodeParams prm;  // about 30 KB of stack
+  int32_t np[kDecodeMaxSeqs] = {};
+  int32_t nu = 0, last_cta = -1;
+  auto keep = [&](const UnitDesc& u, int64_t, int32_t i, int32_t cta) {
+    if (nu >= kDecodeMaxUnits || cta < last_cta || cta > last_cta + 1) return false;
+    if (cta != last_cta) prm.cta_unit0[cta] = static_cast<uint16_t>(nu);
+    last_cta = cta;
+    prm.unit[nu] = u;
+    prm.unit[nu].seq = static_cast<uint8_t>(i);  // n_seqs <= kDecodeMaxSeqs: one launch
+    ++nu;
     return true;
   };
   const int mode = decode_mode(p, seq_ids, n_seqs, NC);
-  const int64_t cut = cut_units(p, seq_ids, n_seqs, NC, mode, np, keep);
-  if (cut < 0)
+  LaunchDesc ld;
+  if (!cut_launch(p, seq_ids, 0, n_seqs, NC, mode, np, &ld, keep) || last_cta + 1 != ld.n_ctas)
     return fail(MKV_ERR_UNSUPPORTED, "the no-allocation decode takes at most %d work units per call", kDecodeMaxUnits);
+  prm.cta_unit0[ld.n_ctas] = static_cast<uint16_t>(nu);
+  prm.n_ctas = ld.n_ctas;
+  prm.n_fp8 = mode == kDecodeSplit ? ld.n_fp8 : 0;
   int32_t parts = 0;
   for (int32_t i = 0; i < n_seqs; ++i) {
     SeqDesc& d = prm.seq[i];
@@ -913,12 +964,8 @@ int mkv_decode_attention_noalloc(mkv_pool_t p, const int32_t* seq_ids, int32_t n
   if (bytes > cap)
     return fail(MKV_ERR_WORKSPACE_TOO_SMALL,
                 "call needs %zu bytes of partial-state scratch; the static scratch holds %zu", bytes, cap);
-  prm.n_fp8 = order_units(t.order, nu, mode != kDecodeSplit,
-                          [&](int32_t k) { return static_cast<int>(t.unit[k].fmt); },
-                          [&](int32_t k) { return t.cost[k]; });
   prm.fused = mode == kDecodeFused ? 1 : 0;
   prm.page_fmt = p->page_fmt;
-  for (int32_t k = 0; k < nu; ++k) prm.unit[k] = t.unit[t.order[k]];
   uint8_t* ws = static_cast<uint8_t*>(scratch);
   prm.fp8_slab = p->fp8_slab;
   prm.tq3_slab = p->tq3_slab;

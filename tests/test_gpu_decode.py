@@ -70,6 +70,24 @@ def test_decode_planned_for_fewer_sms():
     run_and_check(w, lp=lp)
 
 
+@pytest.mark.parametrize("fused", [False, True])
+@pytest.mark.parametrize("D,Hq,Hkv,q_len", [(128, 8, 2, 1), (256, 12, 2, 1), (64, 16, 2, 2),
+                                            (256, 24, 4, 4)])
+def test_ctas_spanning_many_sequences(D, Hq, Hkv, q_len, fused):
+    """Planned for 2 SMs, a CTA takes the pieces of many sequences (and, fused, of both
+    formats) one after another, re-initialising its ring between them; every piece's partial
+    state reaches the merge.  One-tile and team layouts."""
+    w = Workload("span", 23, B=9, Hq=Hq, Hkv=Hkv, D=D, q_len=q_len, window=64,
+                 ctx_range=(40, 1500), protect_frac=0.1, outliers=True)
+    lp = lib_pool(w)
+    lp.set_decode_kernels(fused)
+    lp.set_decode_sms(2)
+    units, _ = lp.decode_plan(list(range(w.B)), q_len, Hq)
+    per_cta = np.bincount(units[:, 5])
+    assert per_cta.max() >= 3, per_cta
+    run_and_check(w, lp=lp)
+
+
 def test_long_qlen4_scaled():
     run_and_check(long_qlen4().scaled(B=2, ctx=(3001, 1200), layers=1))
 

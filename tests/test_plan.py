@@ -1,10 +1,12 @@
 """The decode work-unit cut (mkv_decode_plan) on host-only pools.
 
-The cut is host logic: every sequence's pages of each format are split into units of whole pages,
-one CTA per (unit, KV head).  These tests check what any correct cut must satisfy -- each page of a
-format in exactly one unit of that format, TQ3 units splitting the TQ3 pages into equal shares in
-logical order, the page limits per unit, the one-wave budget -- and, on small cases, that the
-longest unit is within one page of the best cut a brute-force search finds under the same rules.
+The cut is host logic.  A grid's pages -- every sequence's pages of its format (or of both, for
+the fused grid), in call order -- form a line that is cut into CTAs of equal cost; a CTA takes one
+unit (pages of one format inside a logical page range of one sequence) per sequence its share
+touches.  These tests check what any correct cut must satisfy -- each page of a format in exactly
+one unit of that format, TQ3 ranges tiling each table in logical order, the page limits per unit,
+the one-wave budget, units listed CTA by CTA -- and that the costliest CTA is within a few pages of
+the average.
 """
 import numpy as np
 import pytest
@@ -39,8 +41,10 @@ def formats(pool, s):
 
 def check_cut(pool, seqs, units, wave, Hkv):
     units = np.asarray(units)
-    assert np.all(np.diff(units[:, 0]) >= 0), "units not in sequence order"
-    min_units = 0
+    assert units.ndim == 2 and units.shape[1] == 6
+    cta = units[:, 5]
+    # CTA by CTA, numbered 0, 1, 2, ... with at least one unit each
+    assert cta[0] == 0 and np.all(np.diff(cta) >= 0) and np.all(np.diff(cta) <= 1)
     for pos, s in enumerate(seqs):
         fm = formats(pool, s)
         mine = units[units[:, 0] == pos]
@@ -50,61 +54,33 @@ def check_cut(pool, seqs, units, wave, Hkv):
             if idx.size == 0:
                 assert us.size == 0
                 continue
-            min_units += -(-idx.size // MAX_PAGES)
+            us = us[np.argsort(us[:, 2], kind="stable")]
             covered = []
-            for _, _, first, end, cnt in us:
+            for _, _, first, end, cnt, _ in us:
                 inside = idx[(idx >= first) & (idx < end)]
                 assert inside.size == cnt > 0
                 assert cnt <= MAX_PAGES and cnt >= min(MIN_PAGES[f], idx.size)
                 covered.extend(inside.tolist())
             assert covered == idx.tolist(), f"seq {s} fmt {f}: pages not covered exactly once"
             if f == TQ3:
-                # ranges tile the table; unit k holds TQ3 pages number [k n / u, (k+1) n / u)
-                u, n = len(us), idx.size
+                # ranges tile the table; each after the first starts on a TQ3 page
                 assert us[0, 2] == 0 and us[-1, 3] == fm.size
                 assert np.array_equal(us[1:, 2], us[:-1, 3])
-                for k in range(u):
-                    assert us[k, 4] == (k + 1) * n // u - k * n // u
-                    if k:
-                        assert us[k, 2] == idx[k * n // u]
+                assert np.all(fm[us[1:, 2]] == TQ3)
             else:
                 # ranges start and end on FP8 pages
                 assert np.all(fm[us[:, 2]] == FP8) and np.all(fm[us[:, 3] - 1] == FP8)
-                sizes = us[:, 4]
-                assert sizes.max() - sizes.min() <= 1
+    n_ctas = int(cta[-1]) + 1
     budget = max(1, wave // Hkv)
-    if min_units <= budget:
-        assert len(units) <= budget, (len(units), budget)
+    if len(seqs) <= 256:
+        assert n_ctas <= budget, (n_ctas, budget)
     return units
 
 
-def group_pages(pool, seqs):
-    out = []
-    for s in seqs:
-        fm = formats(pool, s)
-        for f in (FP8, TQ3):
-            n = int((fm == f).sum())
-            if n:
-                out.append((f, n))
-    return out
-
-
-def best_longest_unit(groups, budget):
-    """Brute force: the smallest possible cost of the longest unit when group (f, n) is cut into
-    u equal shares, ceil(n / MAX_PAGES) <= u <= max(1, n // MIN_PAGES[f]), sum of u <= budget."""
-    def need(f, n, c):
-        lo, hi = -(-n // MAX_PAGES), max(-(-n // MAX_PAGES), 1, n // MIN_PAGES[f])
-        for u in range(lo, hi + 1):
-            if -(-n // u) * PAGE_COST[f] <= c:
-                return u
-        return None
-    cands = sorted({-(-n // u) * PAGE_COST[f] for f, n in groups
-                    for u in range(1, max(1, n // MIN_PAGES[f]) + 1)})
-    for c in cands:
-        us = [need(f, n, c) for f, n in groups]
-        if all(u is not None for u in us) and sum(us) <= budget:
-            return c
-    return None
+def cta_costs(units):
+    units = np.asarray(units)
+    cost = units[:, 4] * np.where(units[:, 1] == TQ3, PAGE_COST[TQ3], PAGE_COST[FP8])
+    return np.bincount(units[:, 5], weights=cost)
 
 
 @pytest.mark.parametrize("lens,Hkv,window", [
@@ -120,19 +96,35 @@ def test_cut_covers_every_page_once_within_one_wave(lens, Hkv, window):
         check_cut(pool, seqs, units, wave, Hkv)
 
 
-@pytest.mark.parametrize("seed", range(6))
-def test_longest_unit_is_within_one_page_of_the_best_cut(seed):
+@pytest.mark.parametrize("seed", range(8))
+def test_ctas_are_balanced(seed):
+    """The costliest CTA is within a few pages of the line's average: a cut point moves at most
+    a few pages to keep units from being shorter than the minimum, and a CTA has two."""
     rng = np.random.default_rng(100 + seed)
-    Hkv = int(rng.choice([2, 4, 8]))
-    lens = rng.integers(16, 20000, size=int(rng.integers(1, 7))).tolist()
+    Hkv = int(rng.choice([1, 2, 4, 8]))
+    lens = rng.integers(16, 40000, size=int(rng.integers(1, 40))).tolist()
     pool, seqs = mixed_pool(lens, Hkv=Hkv, window=int(rng.choice([0, 64, 512])),
                             protect_frac=float(rng.choice([0.0, 0.05, 0.3])), seed=seed)
     units, wave = pool.decode_plan(seqs, 1, Hkv)
-    check_cut(pool, seqs, units, wave, Hkv)
-    longest = max(int(c) * PAGE_COST[int(f)] for _, f, _, _, c in units)
-    best = best_longest_unit(group_pages(pool, seqs), max(1, wave // Hkv))
-    if best is not None:
-        assert best <= longest <= best + max(PAGE_COST.values()), (longest, best)
+    units = check_cut(pool, seqs, units, wave, Hkv)
+    costs = cta_costs(units)
+    total_pages = int(units[:, 4].sum())
+    k = max(1, min(max(1, wave // Hkv), total_pages // MIN_PAGES[TQ3]))
+    slack = 2 * MIN_PAGES[TQ3] * PAGE_COST[FP8] + PAGE_COST[FP8]
+    assert costs.max() <= costs.sum() / k + slack, (costs.max(), costs.sum() / k)
+
+
+def test_a_ragged_batch_fills_the_wave_evenly():
+    """32 sequences of 2K-32K tokens: cutting each sequence into whole shares would leave the
+    longest CTA far above the average; the line cut keeps every CTA within a few pages of it."""
+    rng = np.random.default_rng(7)
+    lens = rng.integers(2048, 32769, size=32).tolist()
+    pool, seqs = mixed_pool(lens, Hkv=4, window=512, protect_frac=0.02, seed=7)
+    units, wave = pool.decode_plan(seqs, 1, 24)
+    units = check_cut(pool, seqs, units, wave, 4)
+    costs = cta_costs(units)
+    assert len(costs) == wave // 4
+    assert costs.max() <= 1.05 * costs.mean() + 2 * MIN_PAGES[TQ3] * PAGE_COST[FP8]
 
 
 def test_one_long_tq3_run_splits_evenly():
@@ -141,8 +133,9 @@ def test_one_long_tq3_run_splits_evenly():
     units = check_cut(pool, seqs, units, wave, 4)
     tq3 = units[units[:, 1] == TQ3]
     budget = wave // 4
-    assert len(units) <= budget
-    assert tq3[:, 4].max() - tq3[:, 4].min() <= 1 and tq3[:, 4].sum() == 8191
+    assert units[-1, 5] + 1 <= budget
+    # the first CTA also holds the FP8 page 0; every other takes an equal TQ3 share
+    assert tq3[1:, 4].max() - tq3[1:, 4].min() <= 1 and tq3[:, 4].sum() == 8191
 
 
 def test_call_positions_beyond_int16():
@@ -151,9 +144,11 @@ def test_call_positions_beyond_int16():
     seqs = list(range(n))[::-1]
     pool.append(seqs, [16] * n)
     units, _ = pool.decode_plan(seqs, 1, 1)
-    assert units.shape == (n, 5)
+    assert units.shape == (n, 6)
     assert np.array_equal(units[:, 0], np.arange(n))
-    assert np.all(units[:, 1:] == [FP8, 0, 1, 1])
+    assert np.all(units[:, 1:5] == [FP8, 0, 1, 1])
+    # launches of at most 256 sequences, CTA numbers running on across them
+    assert units[0, 5] == 0 and np.all(np.diff(units[:, 5]) >= 0)
 
 
 def test_plan_count_query_and_small_buffer():
@@ -163,7 +158,7 @@ def test_plan_count_query_and_small_buffer():
     units, _ = pool.decode_plan(seqs, 1, 2)
     assert len(units) > 1
     s = np.array(seqs, dtype=np.int32)
-    buf = np.zeros((len(units) - 1, 5), dtype=np.int32)
+    buf = np.zeros((len(units) - 1, 6), dtype=np.int32)
     n = ctypes.c_int32()
     rc = lib().mkv_decode_plan(pool.handle, s.ctypes.data_as(_I32P), s.size, 1, 2,
                                buf.ctypes.data_as(_I32P), len(units) - 1, ctypes.byref(n), None)
