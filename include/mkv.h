@@ -168,15 +168,18 @@ MKV_API int mkv_decode_workspace_bytes(mkv_pool_t pool, const int32_t* seq_ids,
                                        size_t* bytes);
 
 /* The work units mkv_decode_attention would cut for this call (host computation; also on
- * host-only pools), for inspection and tests.  A unit is the pages of one format (0 FP8, 1 TQ3)
- * inside a logical page range of one sequence; the partial kernel runs one CTA per (unit, KV
- * head).  units_out (host int32 [cap][5]) receives, per unit in sequence order: {call position
- * of the sequence, format, first logical page, end logical page (exclusive), pages of that
- * format in the range}; with units_out NULL the call only counts.  *n_units receives the unit
- * count, also when it exceeds cap (then INVALID_ARG and nothing is written); *ctas_per_wave
- * (may be NULL) the CTA
- * budget of one wave the cut aims at (SMs x resident partial CTAs per SM; 148 x 1 where no
- * device is visible).  Errors: as mkv_decode_workspace_bytes, INVALID_ARG. */
+ * host-only pools), for inspection and tests.  A unit is the pages of one format (0 FP8, 1 TQ3,
+ * 2 BF16) inside a logical page range of one sequence, and yields one partial state per query
+ * column and KV head.  Per launch (at most 256 sequences), a grid's pages -- all sequences'
+ * pages of its format, or of both for the fused grid, in call order -- are cut into CTAs of
+ * equal cost; a CTA (of each KV head) takes the units of its share one after another, so it
+ * may span sequences.  units_out (host int32 [cap][6]) receives, CTA by CTA: {call position of
+ * the sequence, format, first logical page, end logical page (exclusive), pages of that format
+ * in the range, CTA number (counted on across launches)}; with units_out NULL the call only
+ * counts.  *n_units receives the unit count, also when it exceeds cap (then INVALID_ARG and
+ * nothing is written); *ctas_per_wave (may be NULL) the CTA budget of one wave the cut aims at
+ * (SMs x resident partial CTAs per SM; 148 x 1 where no device is visible).  Errors: as
+ * mkv_decode_workspace_bytes, INVALID_ARG. */
 MKV_API int mkv_decode_plan(mkv_pool_t pool, const int32_t* seq_ids, int32_t n_seqs,
                             int32_t q_len, int32_t num_q_heads, int32_t* units_out, int32_t cap,
                             int32_t* n_units, int32_t* ctas_per_wave);
@@ -185,9 +188,9 @@ MKV_API int mkv_decode_plan(mkv_pool_t pool, const int32_t* seq_ids, int32_t n_s
  * parciais são combinados"): for sequence seq_ids[i] of length L, query j < q_len (the new
  * tokens are the last q_len positions), query head hq (KV head hq / (num_q_heads/Hkv)):
  *     out[i][j][hq][:] = sum_t softmax_t(sm_scale * q . K_t) V_t   over t <= L - q_len + j
- * with K, V the dequantised cache.  Two kernel launches (more only for very large calls):
- * every sequence is cut into units of one page format and a logical page range; each format
- * has its own partial-attention code producing (running max, denominator, unnormalised
+ * with K, V the dequantised cache.  Per group of up to 256 sequences, the partial grids and a
+ * merge: every sequence is cut into units of one page format and a logical page range; each
+ * format has its own partial-attention code producing (running max, denominator, unnormalised
  * accumulator) per query column of a unit; the merge kernel combines all partial states of a
  * (sequence, KV head, column) with global normalisation.  No dense copy of the cache is made;
  * the workspace holds only partial states.
@@ -196,7 +199,8 @@ MKV_API int mkv_decode_plan(mkv_pool_t pool, const int32_t* seq_ids, int32_t n_s
  *   workspace device scratch of ws_bytes >= mkv_decode_workspace_bytes(...), 256-B aligned
  * Constraints: num_q_heads % Hkv == 0, q_len * (num_q_heads / Hkv) <= 32 (else UNSUPPORTED),
  * n_seqs <= max_seqs (rows may repeat), at most 1536 x 512 pages of one format per sequence
- * (else UNSUPPORTED: one launch group holds 1536 work units of at most 512 pages).
+ * and 1536 work units per group of 256 sequences (else UNSUPPORTED: a unit holds at most 512
+ * pages).
  * Errors: BAD_SEQ, EMPTY_CONTEXT, INVALID_ARG, UNSUPPORTED, WORKSPACE_TOO_SMALL, CUDA. */
 MKV_API int mkv_decode_attention(mkv_pool_t pool, const int32_t* seq_ids, int32_t n_seqs,
                                  int32_t q_len, const void* q_bf16, int32_t num_q_heads,
@@ -218,8 +222,8 @@ MKV_API int mkv_decode_attention(mkv_pool_t pool, const int32_t* seq_ids, int32_
  *     with that device current) and keeps it for the life of the process; make that first call
  *     before any stream capture.  After cudaDeviceReset on that device the kept address is
  *     stale: do not call this entry point on that device again in the same process.
- *   - The call plans its launch in a block of about 75 KB on the calling thread's stack: call
- *     it from threads with at least 128 KB of stack to spare.
+ *   - The call plans its launch in a block of about 30 KB on the calling thread's stack: call
+ *     it from threads with at least 64 KB of stack to spare.
  *   - All calls share the array and it keeps the last call's contents; nothing in it needs to
  *     start at zero.  Calls that overlap on the GPU (other streams, other pools on the same
  *     device) race on it: order them.
@@ -236,10 +240,9 @@ MKV_API int mkv_decode_attention_noalloc(mkv_pool_t pool, const int32_t* seq_ids
  *     programmatic dependent, so both share one wave;
  *   MKV_DECODE_FUSED -- one grid whose CTAs branch on their unit's format;
  *   MKV_DECODE_AUTO (default) -- per call: FUSED when the fused grid keeps as many CTAs per SM
- *     as the TQ3 grid (head_dim 64 and 128), when FP8 pages carry more than 15% of the call's
- *     planned time, or when the sequences holding FP8 pages times the KV heads exceed the SMs
- *     the call is planned for; else SPLIT (for head_dim 256, FP8 CTAs need more shared memory
- *     than TQ3 CTAs, so many of them no longer fit one wave of per-format grids).
+ *     as the TQ3 grid (head_dim 64 and 128) or when FP8 pages carry more than 15% of the call's
+ *     planned time; else SPLIT (for head_dim 256, FP8 CTAs need more shared memory than TQ3
+ *     CTAs, so many of them no longer fit one wave of per-format grids).
  * Host only; applies to later decode calls on this pool.  Errors: INVALID_ARG. */
 #define MKV_DECODE_SPLIT 0
 #define MKV_DECODE_FUSED 1

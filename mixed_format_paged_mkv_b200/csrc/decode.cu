@@ -114,6 +114,10 @@ struct Cfg {
   static constexpr int MINB = TEAM ? (D == 64 ? 8 : (D == 256 ? 3 : 4))
                              : K == kKindBf16 ? 1 : D == 256 ? (K == kKindFused ? 3 : 4)
                                                              : (D == 128 ? 5 : 6);
+  // table entries per lane in flight while scanning a unit's range: deep where the launch
+  // bounds leave more than 128 registers, or 128 to a one-tile kernel (the others spill)
+  static constexpr int REG_BUDGET = 65536 / (THREADS * MINB);
+  static constexpr int SCAN = REG_BUDGET > 128 || (REG_BUDGET == 128 && NT == 1) ? 32 : 8;
 };
 
 // Stage barriers in the header (full[]): every unit initialises all of them, whatever its
@@ -705,22 +709,25 @@ __device__ __forceinline__ float build_q_bf16(const DecodeParams& p, const SeqDe
   return p.logit_scale;
 }
 
-// Scanner warp: collect the unit's pages of format fmt from table entries [first, last).
+// Scanner warp: collect the unit's pages of format fmt from table entries [first, last).  A
+// round reads 32 x DEPTH entries (DEPTH loads per lane in flight), so a sparse range of a few
+// thousand pages costs a few memory latencies.  Kernels with registers to spare take 32.
+template <int DEPTH>
 __device__ __forceinline__ int scan_range(const DecodeParams& p, const int32_t* row, int first,
                                           int last, int fmt, int lane, int2* list) {
   const int nslots = fmt == 1 ? p.tq3_slots : p.fp8_slots;
   const unsigned lt = (1u << lane) - 1u;
   int count = 0;
   bool bad = false;
-  for (int base = first; base < last; base += 256) {
-    int32_t e[8];
+  for (int base = first; base < last; base += 32 * DEPTH) {
+    int32_t e[DEPTH];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < DEPTH; ++j) {
       const int idx = base + 32 * j + lane;
       e[j] = idx < last ? row[idx] : -1;
     }
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < DEPTH; ++j) {
       const int idx = base + 32 * j + lane;
       const uint32_t f = static_cast<uint32_t>(e[j]) >> kFmtShift;
       const int slot = static_cast<int>(static_cast<uint32_t>(e[j]) & kSlotMask);
@@ -808,7 +815,7 @@ __device__ void run_unit(const DecodeParams& p, const SeqDesc& sd, const UnitDes
     if (lane == 0) init_ring(sm, again);
     __syncwarp();
     const int32_t* row = p.tables + static_cast<int64_t>(sd.row) * p.max_pages;
-    const int n = scan_range(p, row, u.first, u.last, F, lane, sm.list);
+    const int n = scan_range<C::SCAN>(p, row, u.first, u.last, F, lane, sm.list);
     __syncwarp();
     if (lane == 0) sm.misc[0] = n;
     for (int i = 0; i < min(n, NST); ++i) fill_stage<PG, F>(sm, slab, slot_bytes, h, i, lane);
@@ -1022,7 +1029,7 @@ __device__ void run_unit_team(const DecodeParams& p, const SeqDesc& sd, const Un
     if (lane == 0) init_ring(sm, again);
     __syncwarp();
     const int32_t* row = p.tables + static_cast<int64_t>(sd.row) * p.max_pages;
-    const int n = scan_range(p, row, u.first, u.last, F, lane, sm.list);
+    const int n = scan_range<C::SCAN>(p, row, u.first, u.last, F, lane, sm.list);
     __syncwarp();
     if (lane == 0) sm.misc[0] = n;
     for (int i = 0; i < min(n, NST); ++i) fill_stage<PG, F>(sm, slab, slot_bytes, h, i, lane);

@@ -247,20 +247,37 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 // Work-unit cut shared by both decode entry points (no allocation).  A launch runs one grid per
 // page format (or one fused grid) of CTAs x KV heads, sized for a single wave: at most
 // SMs x resident CTAs per SM.  A grid's pages -- every sequence's pages of its format, in call
-// order -- form one line, cut into CTAs of equal cost; a CTA takes the pieces of the sequences
-// its share of the line touches, one unit each (a unit is one format's pages inside a logical
-// page range of one sequence, and yields one partial state).  So the longest CTA, which ends
-// the wave, is within a few pages of the average however unequal the sequences are.  A single
-// balanced wave measured faster than several smaller ones: each CTA sets up and combines its
-// warps once per unit and no partial last wave is left.  Cut points that would leave a unit of
-// fewer than a few pages move to the sequence's edge; a unit holds at most kMaxPagesPerUnit
-// pages.  Pages are weighted by measured time per CTA (FP8 11, TQ3 10), not by bytes.
+// order -- form one line, cut into CTAs of equal cost; a CTA takes a unit for each sequence its
+// share of the line touches (a unit is one format's pages inside a logical page range of one
+// sequence, and yields one partial state).  So the longest CTA, which ends the wave, is within a
+// few pages of the average however unequal the sequences are.  A single balanced wave measured
+// faster than several smaller ones: each CTA sets up and combines its warps once per unit and no
+// partial last wave is left.
+//   - Pages are weighted by measured time per CTA (FP8 11, TQ3 10), not by bytes, and every
+//     run of pages that starts a unit adds kUnitCost (the unit's scan, Q set-up, ring refill
+//     and combine), so a CTA that starts several units takes fewer pages.
+//   - A sequence's FP8 pages are split into runs at gaps of more than kFp8RunGap pages (the
+//     sink pages and the recent window are far apart): a unit's kernel scans its whole logical
+//     range for pages of its format, and one run keeps that range short.
+//   - Cut points that would leave a unit of fewer than a few pages move to the run's edge; a
+//     unit holds at most kMaxPagesPerUnit pages.
 constexpr int kMinTq3PagesPerUnit = 8;
 constexpr int kMinFp8PagesPerUnit = 4;
+constexpr int64_t kUnitCost = 60;
+constexpr int32_t kFp8RunGap = 2048;
 
 // Pages of format slot f (0: FP8 or BF16, 1: TQ3) of a sequence.
 inline int64_t group_pages(const Seq& s, int f) {
   return f == 0 ? static_cast<int64_t>(s.fp8_pages.size()) : static_cast<int64_t>(s.n3);
+}
+
+// End of the run of format slot f that starts at page number a (of n) of the sequence.
+inline int64_t run_end(const Seq& s, int f, int64_t a, int64_t n) {
+  if (f == 1) return n;
+  const std::vector<int32_t>& f8 = s.fp8_pages;
+  int64_t e = a + 1;
+  while (e < n && f8[e] - f8[e - 1] <= kFp8RunGap) ++e;
+  return e;
 }
 
 // Cut one line -- the pages of the format slots in `fmts` (bit f) of call positions [s0, s1),
@@ -276,7 +293,9 @@ bool cut_line(const mkv_pool* p, const int32_t* seq_ids, int32_t s0, int32_t s1,
   for (int32_t i = s0; i < s1; ++i)
     for (int f = 0; f < 2; ++f)
       if (fmts >> f & 1) {
-        const int64_t n = group_pages(p->seqs[seq_ids[i]], f);
+        const Seq& s = p->seqs[seq_ids[i]];
+        const int64_t n = group_pages(s, f);
+        for (int64_t a = 0; a < n; a = run_end(s, f, a, n)) T += kUnitCost;
         T += n * b[f];
         pages += n;
       }
@@ -285,7 +304,7 @@ bool cut_line(const mkv_pool* p, const int32_t* seq_ids, int32_t s0, int32_t s1,
   k = std::max<int64_t>(1, std::min<int64_t>(k, pages / ((fmts & 2) ? m[1] : m[0])));
   int64_t j = 0;        // current piece
   int64_t owner = -1;   // the piece that last took a CTA number
-  int64_t G0 = 0;       // line position (cost) of the current group's first page
+  int64_t R0 = 0;       // line position of the current run (its unit cost, then its pages)
   for (int32_t i = s0; i < s1; ++i) {
     const Seq& s = p->seqs[seq_ids[i]];
     const std::vector<int32_t>& f8 = s.fp8_pages;
@@ -294,8 +313,6 @@ bool cut_line(const mkv_pool* p, const int32_t* seq_ids, int32_t s0, int32_t s1,
     for (int f = 0; f < 2; ++f) {
       if (!(fmts >> f & 1)) continue;
       const int64_t n = group_pages(s, f);
-      if (n == 0) continue;
-      const int64_t G1 = G0 + n * b[f];
       int64_t c8 = 0;  // FP8 pages before the current TQ3 page (logical = TQ3 number + c8)
       auto logical = [&](int64_t t) {  // logical page of TQ3 page number t (t < n)
         while (c8 < n8 && f8[c8] <= t + c8) ++c8;
@@ -327,32 +344,49 @@ bool cut_line(const mkv_pool* p, const int32_t* seq_ids, int32_t s0, int32_t s1,
         }
         return true;
       };
-      int64_t a = 0;
-      while (a < n) {
-        const int64_t x = j + 1 < k ? T * (j + 1) / k : T;  // where piece j ends on the line
-        if (x >= G1) {  // piece j takes the rest of the group
-          if (!put(a, n)) return false;
-          a = n;
-          break;
+      for (int64_t ra = 0; ra < n;) {
+        const int64_t rb = run_end(s, f, ra, n);
+        const int64_t P0 = R0 + kUnitCost, R1 = P0 + (rb - ra) * b[f];
+        int64_t a = ra;
+        while (a < rb) {
+          const int64_t x = j + 1 < k ? T * (j + 1) / k : T;  // where piece j ends on the line
+          if (x >= R1) {  // piece j takes the rest of the run
+            if (!put(a, rb)) return false;
+            a = rb;
+            break;
+          }
+          // piece j ends inside the run: nearest page boundary, moved so that no unit of the
+          // run is shorter than m pages where the run allows
+          int64_t e = x <= P0 ? ra : ra + (x - P0 + b[f] / 2) / b[f];
+          e = std::max(a, std::min(e, rb));
+          if (e > a && e - a < m[f]) e = a == ra ? ra : std::min(rb, a + m[f]);
+          if (e < rb && rb - e < m[f]) e = rb;
+          if (e > a && !put(a, e)) return false;
+          a = e;
+          ++j;
         }
-        // piece j ends inside the group: nearest page boundary, moved so that no unit of this
-        // group is shorter than m pages where the group allows
-        int64_t e = x <= G0 ? 0 : (x - G0 + b[f] / 2) / b[f];
-        e = std::max(a, std::min(e, n));
-        if (e > a && e - a < m[f]) e = a == 0 ? 0 : std::min(n, a + m[f]);
-        if (e < n && n - e < m[f]) e = n;
-        if (e > a && !put(a, e)) return false;
-        a = e;
-        ++j;
+        R0 = R1;
+        ra = rb;
       }
-      G0 = G1;
     }
   }
   return true;
 }
 
-// Units of one launch (call positions [s0, s1)): the wave's CTAs shared by the grids in
-// proportion to their cost.  Returns false when emit does.
+// Units of one launch (call positions [s0, s1)), one of two cuts:
+//   - per group (the default): every (sequence, format) group is split into equal parts, one
+//     CTA each, the unit cost chosen by bisection as the smallest whose cut fits the wave
+//     (or, when the groups alone outnumber the wave, one unit per group and 512 pages, the
+//     hardware scheduler then balancing the waves); units go largest first, FP8 units first
+//     for the per-format grids.  Every CTA starts one unit.
+//   - the line cut (cut_line) when the per-group cut fits one wave but its longest unit is
+//     more than 1 / kLineCutBelow times the wave's average: many unequal sequences (32 of 2K to
+//     32K tokens left it 38% above).  A few CTAs then start two or more units, which costs more
+//     than their unit cost accounts for where the per-group cut is already balanced (the
+//     long-context workload: 157 against 151 us).
+// Returns false when emit does.
+constexpr double kLineCutBelow = 0.85;
+
 template <class Emit>
 bool cut_launch(const mkv_pool* p, const int32_t* seq_ids, int32_t s0, int32_t s1, int32_t NC,
                 int mode, int32_t* n_parts, LaunchDesc* ld, Emit&& emit) {
@@ -360,27 +394,139 @@ bool cut_launch(const mkv_pool* p, const int32_t* seq_ids, int32_t s0, int32_t s
   const int64_t slots =
       static_cast<int64_t>(plan_sms(p)) * partial_ctas_per_sm(p->cfg.head_dim, NC, mode);
   int64_t U = std::max<int64_t>(1, slots / Hkv);
-  int64_t c8 = 0, c3 = 0, bound = 0;
-  for (int32_t i = s0; i < s1; ++i) {
-    const Seq& s = p->seqs[seq_ids[i]];
-    for (int f = 0; f < 2; ++f) {
-      const int64_t n = group_pages(s, f);
-      (f == 0 ? c8 : c3) += n * (f == 0 ? kFp8PageCost : kTq3PageCost);
-      // units beyond one per CTA: one more per group a cut crosses, and the 512-page splits
-      if (n > 0) bound += 1 + n / kMaxPagesPerUnit;
-    }
-  }
-  // the launch's units fit the parameter block: units <= CTAs + bound
-  U = std::max<int64_t>(1, std::min<int64_t>(U, kDecodeMaxUnits - 2 - bound));
   ld->s0 = s0;
   ld->s1 = s1;
   ld->n_ctas = 0;
   ld->n_fp8 = 0;
+
+  // ---- per-group cut
+  const int64_t b[2] = {kFp8PageCost, kTq3PageCost};
+  const int mins[2] = {kMinFp8PagesPerUnit, kMinTq3PagesPerUnit};
+  int64_t total = 0;
+  for (int32_t i = s0; i < s1; ++i)
+    for (int f = 0; f < 2; ++f) total += group_pages(p->seqs[seq_ids[i]], f) * b[f];
+  // units of a group at unit cost c: as many as its cost needs, clamped to the page limits
+  auto units_at = [](double c, int64_t cost, int64_t pages, int min_pages) -> int64_t {
+    const int64_t lo = (pages + kMaxPagesPerUnit - 1) / kMaxPagesPerUnit;
+    const int64_t hi = std::max<int64_t>(lo, std::max<int64_t>(1, pages / min_pages));
+    const int64_t u = static_cast<int64_t>(std::ceil(static_cast<double>(cost) / c - 1e-9));
+    return std::max(lo, std::min(std::max<int64_t>(u, 1), hi));
+  };
+  auto count_at = [&](double c) -> int64_t {
+    int64_t sum = 0;
+    for (int32_t i = s0; i < s1; ++i)
+      for (int f = 0; f < 2; ++f) {
+        const int64_t n = group_pages(p->seqs[seq_ids[i]], f);
+        if (n > 0) sum += units_at(c, n * b[f], n, mins[f]);
+      }
+    return sum;
+  };
+  // smallest unit cost whose cut needs at most U units (the largest unit bounds the wave)
+  double lo_c = std::max(1.0, static_cast<double>(total) / U), hi_c = lo_c;
+  while (count_at(hi_c) > U && hi_c < 4.0 * total) hi_c *= 2.0;
+  for (int it = 0; it < 40 && hi_c - lo_c > 0.5; ++it) {
+    const double mid = 0.5 * (lo_c + hi_c);
+    (count_at(mid) <= U ? hi_c : lo_c) = mid;
+  }
+  const double unit_cost = hi_c;
+  const bool fits = count_at(unit_cost) <= U;
+  // groups in launch order: per-format grids take the FP8 groups first; largest units first
+  int32_t order[2 * kDecodeMaxSeqs];
+  int64_t ucost[2 * kDecodeMaxSeqs];
+  int32_t ng = 0;
+  int64_t longest = 0;
+  for (int32_t i = s0; i < s1; ++i)
+    for (int f = 0; f < 2; ++f) {
+      const int64_t n = group_pages(p->seqs[seq_ids[i]], f);
+      if (n == 0) continue;
+      const int64_t u = units_at(unit_cost, n * b[f], n, mins[f]);
+      ucost[ng] = (n + u - 1) / u * b[f];
+      longest = std::max(longest, ucost[ng]);
+      order[ng++] = 2 * (i - s0) + f;
+    }
+  const bool line = fits && static_cast<double>(total) / static_cast<double>(U) <
+                                kLineCutBelow * static_cast<double>(longest);
+  if (!line) {
+    int32_t idx[2 * kDecodeMaxSeqs];
+    for (int32_t g = 0; g < ng; ++g) idx[g] = g;
+    std::sort(idx, idx + ng, [&](int32_t x, int32_t y) {
+      const int fx = order[x] & 1, fy = order[y] & 1;
+      if (mode == kDecodeSplit && fx != fy) return fx < fy;  // FP8 (0) first
+      return ucost[x] != ucost[y] ? ucost[x] > ucost[y] : x < y;
+    });
+    for (int32_t g = 0; g < ng; ++g) {
+      const int32_t i = s0 + order[idx[g]] / 2;
+      const int f = order[idx[g]] & 1;
+      if (mode == kDecodeSplit && f == 1 && ld->n_fp8 == 0) ld->n_fp8 = ld->n_ctas;
+      const Seq& s = p->seqs[seq_ids[i]];
+      const std::vector<int32_t>& f8 = s.fp8_pages;
+      const int64_t n8 = static_cast<int64_t>(f8.size());
+      const int64_t n = group_pages(s, f);
+      const int64_t u = units_at(unit_cost, n * b[f], n, mins[f]);
+      // unit k takes pages number [k n / u, (k+1) n / u) of the group.  TQ3 ranges tile the
+      // table: each starts at the logical page of its first TQ3 page (the first at page 0) and
+      // ends where the next one starts (the last at the end of the table); every page is FP8
+      // or TQ3, so TQ3 page number j sits at logical page j + c, c the FP8 pages before it
+      const int32_t table = static_cast<int32_t>(s.table.size());
+      int64_t c = 0;
+      int32_t start = 0;
+      for (int64_t k = 0; k < u; ++k) {
+        const int64_t j0 = k * n / u, j1 = (k + 1) * n / u;
+        UnitDesc d{};
+        if (f == 0) {
+          if (j1 <= j0) continue;
+          d.first = f8[j0];
+          d.last = f8[j1 - 1] + 1;
+          d.fmt = static_cast<uint8_t>(p->page_fmt);
+        } else {
+          int32_t end = table;
+          if (k + 1 < u) {
+            while (c < n8 && f8[c] <= j1 + c) ++c;
+            end = static_cast<int32_t>(j1 + c);
+          }
+          d.first = start;
+          d.last = end;
+          d.fmt = 1;
+          start = end;
+          if (j1 <= j0) continue;
+        }
+        d.part = static_cast<uint16_t>(std::min<int32_t>(n_parts[i], 65535));
+        ++n_parts[i];
+        if (!emit(d, (j1 - j0) * b[f], i, ld->n_ctas)) return false;
+        ++ld->n_ctas;
+      }
+    }
+    if (mode == kDecodeSplit && ld->n_fp8 == 0) {  // no TQ3 group: every CTA is an FP8 one
+      bool any3 = false;
+      for (int32_t g = 0; g < ng; ++g) any3 |= (order[g] & 1) == 1;
+      if (!any3) ld->n_fp8 = ld->n_ctas;
+    }
+    return true;
+  }
+
+  // ---- line cut
+  int64_t c8 = 0, c3 = 0, bound = 0, runs8 = 0;
+  for (int32_t i = s0; i < s1; ++i) {
+    const Seq& s = p->seqs[seq_ids[i]];
+    for (int f = 0; f < 2; ++f) {
+      const int64_t n = group_pages(s, f);
+      int64_t runs = 0;
+      for (int64_t a = 0; a < n; a = run_end(s, f, a, n)) ++runs;
+      (f == 0 ? c8 : c3) += n * b[f] + runs * kUnitCost;
+      if (f == 0) runs8 += runs;
+      // units beyond one per CTA: one more per run a cut crosses, and the 512-page splits
+      bound += runs + n / kMaxPagesPerUnit;
+    }
+  }
+  // the launch's units fit the parameter block: units <= CTAs + bound
+  U = std::max<int64_t>(1, std::min<int64_t>(U, kDecodeMaxUnits - 2 - bound));
   if (mode == kDecodeSplit) {
     int64_t k8 = 0, k3 = 0;
     if (c8 > 0 && c3 > 0) {
       k8 = std::llround(static_cast<double>(U) * c8 / static_cast<double>(c8 + c3));
-      k8 = std::max<int64_t>(1, std::min<int64_t>(k8, U - 1));
+      // an FP8 CTA starts at most a few units (each a ring refill from memory)
+      k8 = std::max<int64_t>((runs8 + 3) / 4, k8);
+      k8 = std::max<int64_t>(1, std::min<int64_t>(k8, U - 1));  // both grids get a CTA
       k3 = std::max<int64_t>(1, U - k8);
     } else {
       (c8 > 0 ? k8 : k3) = U;

@@ -16,6 +16,9 @@ from mixed_format_paged_mkv_b200 import Pool
 FP8, TQ3 = 0, 1
 MAX_PAGES, MIN_PAGES = 512, {FP8: 4, TQ3: 8}
 PAGE_COST = {FP8: 11, TQ3: 10}   # relative time of one page per CTA, as the planner weighs them
+UNIT_COST = 60                   # and of starting a unit
+LINE_CUT_BELOW = 0.85            # the line cut replaces a per-group cut this far from balance
+FP8_RUN_GAP = 2048               # FP8 pages farther apart than this start a new run
 
 
 def mixed_pool(lens, Hkv=4, sink=1, window=64, protect_frac=0.03, seed=0):
@@ -55,11 +58,16 @@ def check_cut(pool, seqs, units, wave, Hkv):
                 assert us.size == 0
                 continue
             us = us[np.argsort(us[:, 2], kind="stable")]
+            # runs: FP8 pages split where the gap exceeds FP8_RUN_GAP pages; TQ3 pages form one
+            run = np.zeros(idx.size, dtype=np.int64)
+            if f == FP8:
+                run[1:] = np.cumsum(np.diff(idx) > FP8_RUN_GAP)
             covered = []
             for _, _, first, end, cnt, _ in us:
                 inside = idx[(idx >= first) & (idx < end)]
                 assert inside.size == cnt > 0
-                assert cnt <= MAX_PAGES and cnt >= min(MIN_PAGES[f], idx.size)
+                r = run[np.searchsorted(idx, inside[0])]
+                assert cnt <= MAX_PAGES and cnt >= min(MIN_PAGES[f], int((run == r).sum()))
                 covered.extend(inside.tolist())
             assert covered == idx.tolist(), f"seq {s} fmt {f}: pages not covered exactly once"
             if f == TQ3:
@@ -72,12 +80,20 @@ def check_cut(pool, seqs, units, wave, Hkv):
                 assert np.all(fm[us[:, 2]] == FP8) and np.all(fm[us[:, 3] - 1] == FP8)
     n_ctas = int(cta[-1]) + 1
     budget = max(1, wave // Hkv)
-    if len(seqs) <= 256:
+    min_units = 0   # at least one unit per group and per 512 pages
+    for s in seqs:
+        fm = formats(pool, s)
+        for f in (FP8, TQ3):
+            min_units += -(-int((fm == f).sum()) // MAX_PAGES)
+    if len(seqs) <= 256 and min_units <= budget:
         assert n_ctas <= budget, (n_ctas, budget)
     return units
 
 
 def cta_costs(units):
+    """Cost of each CTA as the planner weighs it: its pages, and a unit cost for every unit
+    that starts a run (the planner charges a run's start once, to the CTA that starts it; a
+    unit that continues a run another CTA started costs that CTA nothing extra here)."""
     units = np.asarray(units)
     cost = units[:, 4] * np.where(units[:, 1] == TQ3, PAGE_COST[TQ3], PAGE_COST[FP8])
     return np.bincount(units[:, 5], weights=cost)
@@ -108,23 +124,41 @@ def test_ctas_are_balanced(seed):
     units, wave = pool.decode_plan(seqs, 1, Hkv)
     units = check_cut(pool, seqs, units, wave, Hkv)
     costs = cta_costs(units)
+    U = max(1, wave // Hkv)
+    if units[-1, 5] + 1 > U:
+        return  # more groups than the wave holds: one unit per group, the scheduler balances
     total_pages = int(units[:, 4].sum())
-    k = max(1, min(max(1, wave // Hkv), total_pages // MIN_PAGES[TQ3]))
+    k = max(1, min(U, total_pages // MIN_PAGES[TQ3]))
+    runs = n_runs(pool, seqs)
     slack = 2 * MIN_PAGES[TQ3] * PAGE_COST[FP8] + PAGE_COST[FP8]
-    assert costs.max() <= costs.sum() / k + slack, (costs.max(), costs.sum() / k)
+    # the per-group cut where its longest unit is within 1 / 0.85 of the average, else the
+    # line cut, within a few pages of it
+    bound = max(costs.sum() / U / LINE_CUT_BELOW + PAGE_COST[FP8],
+                (costs.sum() + runs * UNIT_COST) / k + slack)
+    assert costs.max() <= bound, (costs.max(), costs.sum() / U)
+
+
+def n_runs(pool, seqs):
+    total = 0
+    for s in seqs:
+        fm = formats(pool, s)
+        idx = np.nonzero(fm == FP8)[0]
+        total += (idx.size > 0) + int((np.diff(idx) > FP8_RUN_GAP).sum()) + int((fm == TQ3).any())
+    return total
 
 
 def test_a_ragged_batch_fills_the_wave_evenly():
-    """32 sequences of 2K-32K tokens: cutting each sequence into whole shares would leave the
-    longest CTA far above the average; the line cut keeps every CTA within a few pages of it."""
+    """32 sequences of 2K-32K tokens in a wave of 148 CTAs: cutting each sequence into whole
+    shares would leave the longest CTA far above the average, so the planner takes the line cut,
+    whose CTAs (some starting several units) stay within a few pages of it."""
     rng = np.random.default_rng(7)
     lens = rng.integers(2048, 32769, size=32).tolist()
-    pool, seqs = mixed_pool(lens, Hkv=4, window=512, protect_frac=0.02, seed=7)
-    units, wave = pool.decode_plan(seqs, 1, 24)
-    units = check_cut(pool, seqs, units, wave, 4)
+    pool, seqs = mixed_pool(lens, Hkv=1, window=512, protect_frac=0.02, seed=7)
+    units, wave = pool.decode_plan(seqs, 1, 6)
+    units = check_cut(pool, seqs, units, wave, 1)
     costs = cta_costs(units)
-    assert len(costs) == wave // 4
-    assert costs.max() <= 1.05 * costs.mean() + 2 * MIN_PAGES[TQ3] * PAGE_COST[FP8]
+    assert len(costs) == wave and np.bincount(units[:, 5]).max() >= 2
+    assert costs.max() <= 1.05 * costs.mean() + 2 * MIN_PAGES[TQ3] * PAGE_COST[FP8] + UNIT_COST
 
 
 def test_one_long_tq3_run_splits_evenly():
@@ -201,3 +235,16 @@ def test_decode_sms_caps_the_wave():
     from mixed_format_paged_mkv_b200.api import MkvError
     with pytest.raises(MkvError):
         pool.set_decode_sms(-1)
+
+
+@pytest.mark.parametrize("fused", [False, True])
+@pytest.mark.parametrize("sms", [1, 2, 3])
+def test_tiny_wave_still_covers_both_formats(fused, sms):
+    """A wave of one or two CTAs per KV head: each grid still gets a CTA, so both formats'
+    pages are covered."""
+    pool, seqs = mixed_pool((3000, 700, 45, 1600), Hkv=4, window=64, protect_frac=0.1)
+    pool.set_decode_kernels(fused)
+    pool.set_decode_sms(sms)
+    units, wave = pool.decode_plan(seqs, 1, 4)
+    check_cut(pool, seqs, units, max(wave, 2 * 4), 4)
+    assert set(units[:, 1].tolist()) == {FP8, TQ3}
