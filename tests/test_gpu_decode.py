@@ -94,16 +94,22 @@ def test_ctas_spanning_many_sequences(D, Hq, Hkv, q_len, fused):
 
 @pytest.mark.parametrize("fused", [False, True])
 def test_fp8_runs_far_apart(fused):
-    """The sink page and the recent window lie more than 2048 pages apart: each is its own FP8
-    unit (a short scan range), and the result still matches the oracle."""
-    w = Workload("runs", 29, B=2, Hq=8, Hkv=2, D=128, q_len=1, window=64, ctx=(40000, 36011),
-                 outliers=True)
+    """Under the line cut, the sink page and the recent window, more than 2048 pages apart, are
+    separate FP8 runs, each its own unit (a short scan range); the result still matches the
+    oracle.  Unequal lengths and a small SM budget make the planner take the line cut."""
+    w = Workload("runs", 29, B=3, Hq=8, Hkv=2, D=128, q_len=1, window=64,
+                 ctx=(40000, 36011, 300), outliers=True)
     lp = lib_pool(w)
     lp.set_decode_kernels(fused)
-    units, _ = lp.decode_plan([0, 1], 1, 8)
-    for pos in (0, 1):
-        fp8 = units[(units[:, 0] == pos) & (units[:, 1] == 0)]
-        assert len(fp8) >= 2 and fp8[:, 2].min() == 0 and fp8[:, 3].max() - fp8[:, 2].max() < 16
+    for sms in range(1, 148):
+        lp.set_decode_sms(sms)
+        units, _ = lp.decode_plan([0, 1, 2], 1, 8)
+        fp8 = units[(units[:, 0] == 0) & (units[:, 1] == 0)]
+        if len(fp8) >= 2:
+            break
+    else:
+        pytest.fail("no plan split the FP8 pages into runs")
+    assert fp8[:, 2].min() == 0 and fp8[:, 3].max() - fp8[:, 2].max() < 16
     run_and_check(w, lp=lp)
 
 
