@@ -39,7 +39,8 @@ PROFILES = os.path.join(ROOT, "profiles")
 
 def kernel_hash() -> str:
     h = hashlib.sha256()
-    for f in ("decode.cu", "device_util.cuh", "mkv_internal.h"):
+    for f in ("decode.cu", "decode_partial.cuh", "decode_d64.cu", "decode_d128.cu",
+              "decode_d256.cu", "device_util.cuh", "mkv_internal.h"):
         with open(os.path.join(ROOT, "mixed_format_paged_mkv_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
