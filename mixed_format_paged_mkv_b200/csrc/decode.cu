@@ -6,16 +6,18 @@
 // normalisation combines them -- no page is converted to a common format first and no dense
 // copy of the cache is made (section "... sem a chamada sombra densa").
 //
-// The host cuts every sequence into work units -- (format, logical page range) -- and orders
-// them largest first.  Three launches per call (per launch group): the FP8 partial kernel over
-// the FP8 units, the TQ3 partial kernel over the TQ3 units and the merge kernel.  The TQ3 and
-// merge kernels are programmatic dependents of the kernel before them: the TQ3 CTAs fill the
-// SM room the FP8 CTAs leave (one wave of both formats), and the merge CTAs wait for the
-// partial states with griddepcontrol.wait.  A fused variant runs both formats in one grid,
-// branching per CTA; the host picks it per call where it keeps the same occupancy or where the
-// FP8 units would overflow the wave.
+// The host cuts every sequence into work units -- (format, logical page range) -- and gives
+// each CTA one unit or, when that balances the wave badly, a run of units of several sequences.
+// Three launches per call (per launch group): the FP8 partial kernel over the FP8 CTAs, the
+// TQ3 partial kernel over the TQ3 CTAs and the merge kernel.  The TQ3 and merge kernels are
+// programmatic dependents of the kernel before them: the TQ3 CTAs fill the SM room the FP8
+// CTAs leave (one wave of both formats), and the merge CTAs wait for the partial states with
+// griddepcontrol.wait.  A fused variant runs both formats in one grid, branching per unit; the
+// host picks it per call where it keeps the same occupancy or where FP8 pages carry much of the
+// work.  The partial kernels are templates (decode_partial.cuh) compiled per head dimension
+// (decode_d64.cu, decode_d128.cu, decode_d256.cu); this file holds the merge and the launches.
 //
-// A partial CTA with at most 8 query columns per KV head takes one (unit, KV head):
+// A partial CTA with at most 8 query columns per KV head takes each of its units in turn:
 //   1. one warp scans the block-table entries of the range, keeps the pages of the unit's format
 //      and starts the first bulk async copies of those pages into a shared-memory ring;
 //   2. the warps take pages round-robin; each ring stage always belongs to the same warp(s),
