@@ -222,8 +222,8 @@ MKV_API int mkv_decode_attention(mkv_pool_t pool, const int32_t* seq_ids, int32_
  *     with that device current) and keeps it for the life of the process; make that first call
  *     before any stream capture.  After cudaDeviceReset on that device the kept address is
  *     stale: do not call this entry point on that device again in the same process.
- *   - The call plans its launch in a block of about 30 KB on the calling thread's stack: call
- *     it from threads with at least 64 KB of stack to spare.
+ *   - The call plans its launch in about 40 KB on the calling thread's stack: call it from
+ *     threads with at least 64 KB of stack to spare.
  *   - All calls share the array and it keeps the last call's contents; nothing in it needs to
  *     start at zero.  Calls that overlap on the GPU (other streams, other pools on the same
  *     device) race on it: order them.

@@ -51,3 +51,25 @@ def test_control_materialise_is_exact():
         assert np.array_equal(k.cpu().numpy().astype(np.float64), K)
         assert np.array_equal(v.cpu().numpy().astype(np.float64), V)
     lp.device_status()
+
+
+@pytest.mark.parametrize("D,Hq,Hkv,q_len", [(128, 8, 2, 1), (256, 24, 4, 2)])
+def test_control_decode_with_ctas_spanning_sequences(D, Hq, Hkv, q_len):
+    """The BF16 control kernel under the line cut: unequal sequences and a small SM budget give
+    CTAs that take the pieces of several sequences one after another."""
+    w = Workload("ctlspan", 63, B=5, Hq=Hq, Hkv=Hkv, D=D, q_len=q_len, window=32,
+                 ctx=(1500, 1300, 120, 60, 33))
+    lp, op = pools(w)
+    for sms in range(1, 64):
+        lp.set_decode_sms(sms)
+        units, _ = lp.decode_plan(list(range(w.B)), q_len, Hq)
+        if np.bincount(units[:, 5]).max() >= 2:
+            break
+    else:
+        pytest.fail("no plan with a CTA that starts several units")
+    q = to_bf16_tensor(np.stack([w.q(s) for s in range(w.B)]))
+    out = lp.decode(list(range(w.B)), q).cpu().numpy()
+    torch.cuda.synchronize()
+    lp.device_status()
+    for s in range(w.B):
+        assert_close(out[s], oracle_decode(op, w, s), what=f"{w.name} seq {s}")
