@@ -568,11 +568,22 @@ int plan_decode(mkv_pool_t p, const int32_t* seq_ids, int32_t n, int32_t q_len, 
   plan->launch.clear();
   std::vector<int32_t> np(n, 0);
   plan->mode = decode_mode(p, seq_ids, n, plan->NC);
-  // launches over groups of at most kDecodeMaxSeqs whole sequences, one wave each
-  for (int32_t s0 = 0; s0 < n; s0 += kDecodeMaxSeqs) {
+  // launches over groups of whole sequences, each cut for one wave: at most kDecodeMaxSeqs
+  // sequences, and no more 512-page units than a launch holds (the per-group cut needs one per
+  // group and 512 pages when the groups outnumber the wave; the line cut sizes itself)
+  for (int32_t s0 = 0, s1 = 0; s0 < n; s0 = s1) {
+    int64_t need = 0;
+    for (s1 = s0; s1 < n && s1 - s0 < kDecodeMaxSeqs; ++s1) {
+      const Seq& s = p->seqs[seq_ids[s1]];
+      int64_t add = 0;
+      for (int f = 0; f < 2; ++f)
+        add += (group_pages(s, f) + kMaxPagesPerUnit - 1) / kMaxPagesPerUnit;
+      if (s1 > s0 && need + add > kDecodeMaxUnits) break;
+      need += add;
+    }
     LaunchDesc ld;
     ld.u0 = static_cast<int32_t>(plan->unit.size());
-    cut_launch(p, seq_ids, s0, std::min(n, s0 + kDecodeMaxSeqs), plan->NC, plan->mode,
+    cut_launch(p, seq_ids, s0, s1, plan->NC, plan->mode,
                np.data(), &ld, [&](const UnitDesc& u, int64_t cost, int32_t i, int32_t cta) {
       plan->unit.push_back(u);
       plan->pos.push_back(i);

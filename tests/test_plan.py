@@ -248,3 +248,18 @@ def test_tiny_wave_still_covers_both_formats(fused, sms):
     units, wave = pool.decode_plan(seqs, 1, 4)
     check_cut(pool, seqs, units, max(wave, 2 * 4), 4)
     assert set(units[:, 1].tolist()) == {FP8, TQ3}
+
+
+def test_launches_split_where_units_would_overflow():
+    """200 sequences of 4000 pages need at least 8 units of at most 512 pages each: the call is
+    planned as launches of at most 1536 units (192 sequences, then the other 8, which fit one
+    wave and get finer units); CTA numbers run on across launches."""
+    n, pages = 200, 4000
+    pool = Pool(1, 64, n, pages, n * pages, 1, host_only=True)
+    seqs = list(range(n))
+    pool.append(seqs, [16 * pages] * n)
+    units, wave = pool.decode_plan(seqs, 1, 1)
+    assert units[:, 4].max() <= MAX_PAGES
+    first = units[units[:, 0] < 192]
+    assert len(first) == 192 * 8 and first[-1, 5] + 1 == 192 * 8
+    check_cut(pool, seqs, units, wave, 1)
