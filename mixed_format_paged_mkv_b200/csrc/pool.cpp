@@ -246,13 +246,12 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Work-unit cut shared by both decode entry points (no allocation).  A launch runs one grid per
 // page format (or one fused grid) of CTAs x KV heads, sized for a single wave: at most
-// SMs x resident CTAs per SM.  A grid's pages -- every sequence's pages of its format, in call
-// order -- form one line, cut into CTAs of equal cost; a CTA takes a unit for each sequence its
-// share of the line touches (a unit is one format's pages inside a logical page range of one
-// sequence, and yields one partial state).  So the longest CTA, which ends the wave, is within a
-// few pages of the average however unequal the sequences are.  A single balanced wave measured
-// faster than several smaller ones: each CTA sets up and combines its warps once per unit and no
-// partial last wave is left.
+// SMs x resident CTAs per SM.  A unit is one format's pages inside a logical page range of one
+// sequence and yields one partial state.  cut_launch picks one of two cuts: per group (below) or
+// the line cut, where a grid's pages -- every sequence's pages of its format, in call order --
+// form one line, cut into CTAs of equal cost; a CTA takes a unit for each sequence its share of
+// the line touches, so the longest CTA, which ends the wave, is within a few pages of the
+// average however unequal the sequences are.  For the line cut:
 //   - Pages are weighted by measured time per CTA (FP8 11, TQ3 10), not by bytes, and every
 //     run of pages that starts a unit adds kUnitCost (the unit's scan, Q set-up, ring refill
 //     and combine), so a CTA that starts several units takes fewer pages.
