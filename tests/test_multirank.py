@@ -66,3 +66,17 @@ def test_reference_arm_prints_one_contract_line():
     assert res["impl"] == "reference" and res["unit"] == "GB/s" and res["value"] > 0
     assert res["cpu_baseline"]["kind"] == "oracle" and res["cpu_baseline"]["cores"] >= 1
     assert res["e2e"]["h2d_bytes_per_step"] == 0 and res["metric"] == bench.METRIC
+
+
+def test_kernel_hash_covers_every_decode_source():
+    """The roofline's DRAM traffic is looked up by a hash of the decode kernel sources; every
+    source of the partial and merge kernels must be part of it, so that a changed kernel never
+    reuses a stale capture."""
+    import glob
+    csrc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                        "mixed_format_paged_mkv_b200", "csrc")
+    decode = {os.path.basename(f) for f in glob.glob(os.path.join(csrc, "decode*"))}
+    import inspect
+    src = inspect.getsource(bench.kernel_hash)
+    missing = [f for f in sorted(decode | {"device_util.cuh", "mkv_internal.h"}) if f not in src]
+    assert not missing, missing
