@@ -218,6 +218,13 @@ __device__ __forceinline__ uint32_t hmax2_u32(uint32_t a, uint32_t b) {
   asm("max.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
 }
+// Per-half maximum of two bf16x2 words (a NaN half yields the other operand's half, as fmaxf;
+// subnormals kept).
+__device__ __forceinline__ uint32_t bmax2_u32(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
 // Two floats -> f16x2 (lo in the low half), round to nearest even.
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);

@@ -321,10 +321,11 @@ __global__ void __launch_bounds__(256) pack_kernel(const __grid_constant__ PackP
                        (static_cast<uint32_t>(src[8 * k + 2 * e + 1]) << 16);
     }
   }
-  float amax = 0.f;
+  // largest magnitude, two bf16 values per operation (|x| by clearing the sign bits)
+  uint32_t mx = 0u;
 #pragma unroll
-  for (int e = 0; e < 16; ++e)
-    amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[e])), fabsf(bf16_hi(w[e]))));
+  for (int e = 0; e < 16; ++e) mx = bmax2_u32(mx, w[e] & 0x7fff7fffu);
+  const float amax = fmaxf(bf16_lo(mx), bf16_hi(mx));
   // codes in the bf16 domain: x >= k*s is m >= ceil(t_k / 2^16) and |x| > k*s is
   // m >= floor(t_k / 2^16) + 1, with m the bf16 magnitude bits and t_k the fp32 bits of k*s
   uint32_t w0, w1, w2;
