@@ -8,7 +8,8 @@ whenever the barrier's completed-phase count has the other parity -- including w
 f - 1 has not completed yet.  The kernel therefore requires that fill f - 1 of a stage was
 consumed by the same warp (NST a multiple of PW), so it has always completed.  This test
 replays random interleavings and checks that no wait is ever ambiguous for the ring shapes
-the kernel uses, and that a shape violating the rule is caught."""
+the kernel uses, that a shape violating the rule is caught, and that a unit ends with every copy
+landed and consumed (so a CTA can re-initialise its barriers for its next unit)."""
 import random
 
 import pytest
@@ -57,6 +58,9 @@ def replay(count, nst, pw, seed):
                 released[i] = True
                 nxt[m] += pw
                 del waiting[m]
+    # a unit ends with no copy in flight and every copy consumed: the kernel may then
+    # invalidate and re-initialise the stage barriers for the CTA's next unit
+    assert issued == count and not in_flight and not waiting
     return ambiguous
 
 
@@ -143,6 +147,7 @@ def replay_team(count, nst, tw, seed):
                 if step[w] == min(tw, count - b):
                     batch[w] += tw
                     step[w] = "k"
+    assert issued == count and not in_flight   # as above: the barriers can be re-initialised
     return ambiguous
 
 
