@@ -392,7 +392,8 @@ bool cut_launch(const mkv_pool* p, const int32_t* seq_ids, int32_t s0, int32_t s
   const int Hkv = p->cfg.num_kv_heads;
   const int64_t slots =
       static_cast<int64_t>(plan_sms(p)) * partial_ctas_per_sm(p->cfg.head_dim, NC, mode);
-  int64_t U = std::max<int64_t>(1, slots / Hkv);
+  // CTAs of the wave per KV head; a launch holds at most kDecodeMaxUnits units
+  int64_t U = std::max<int64_t>(1, std::min<int64_t>(slots / Hkv, kDecodeMaxUnits - 2));
   ld->s0 = s0;
   ld->s1 = s1;
   ld->n_ctas = 0;
