@@ -170,10 +170,13 @@ MKV_API int mkv_decode_workspace_bytes(mkv_pool_t pool, const int32_t* seq_ids,
 /* The work units mkv_decode_attention would cut for this call (host computation; also on
  * host-only pools), for inspection and tests.  A unit is the pages of one format (0 FP8, 1 TQ3,
  * 2 BF16) inside a logical page range of one sequence, and yields one partial state per query
- * column and KV head.  Per launch (at most 256 sequences), a grid's pages -- all sequences'
- * pages of its format, or of both for the fused grid, in call order -- are cut into CTAs of
- * equal cost; a CTA (of each KV head) takes the units of its share one after another, so it
- * may span sequences.  units_out (host int32 [cap][6]) receives, CTA by CTA: {call position of
+ * column and KV head.  A call is split into launches of whole sequences (at most 256, and
+ * fewer when their pages need more than 1536 units of 512 pages), each sized for one wave.
+ * Within a launch each (sequence, format) group is cut into equal units, one CTA (of each KV
+ * head) per unit; where that leaves the wave badly balanced, a grid's pages -- all sequences'
+ * pages of its format, or of both for the fused grid, in call order -- are instead cut into
+ * CTAs of equal cost, and a CTA takes the units of its share one after another, so it may
+ * span sequences.  units_out (host int32 [cap][6]) receives, CTA by CTA: {call position of
  * the sequence, format, first logical page, end logical page (exclusive), pages of that format
  * in the range, CTA number (counted on across launches)}; with units_out NULL the call only
  * counts.  *n_units receives the unit count, also when it exceeds cap (then INVALID_ARG and
@@ -188,8 +191,8 @@ MKV_API int mkv_decode_plan(mkv_pool_t pool, const int32_t* seq_ids, int32_t n_s
  * parciais são combinados"): for sequence seq_ids[i] of length L, query j < q_len (the new
  * tokens are the last q_len positions), query head hq (KV head hq / (num_q_heads/Hkv)):
  *     out[i][j][hq][:] = sum_t softmax_t(sm_scale * q . K_t) V_t   over t <= L - q_len + j
- * with K, V the dequantised cache.  Per group of up to 256 sequences, the partial grids and a
- * merge: every sequence is cut into units of one page format and a logical page range; each
+ * with K, V the dequantised cache.  Per launch of whole sequences (see mkv_decode_plan), the
+ * partial grids and a merge: every sequence is cut into units of one page format and a logical page range; each
  * format has its own partial-attention code producing (running max, denominator, unnormalised
  * accumulator) per query column of a unit; the merge kernel combines all partial states of a
  * (sequence, KV head, column) with global normalisation.  No dense copy of the cache is made;
@@ -199,8 +202,8 @@ MKV_API int mkv_decode_plan(mkv_pool_t pool, const int32_t* seq_ids, int32_t n_s
  *   workspace device scratch of ws_bytes >= mkv_decode_workspace_bytes(...), 256-B aligned
  * Constraints: num_q_heads % Hkv == 0, q_len * (num_q_heads / Hkv) <= 32 (else UNSUPPORTED),
  * n_seqs <= max_seqs (rows may repeat), at most 1536 x 512 pages of one format per sequence
- * and 1536 work units per group of 256 sequences (else UNSUPPORTED: a unit holds at most 512
- * pages).
+ * (else UNSUPPORTED: a launch holds 1536 work units of at most 512 pages; the call is split
+ * into as many launches as its sequences need).
  * Errors: BAD_SEQ, EMPTY_CONTEXT, INVALID_ARG, UNSUPPORTED, WORKSPACE_TOO_SMALL, CUDA. */
 MKV_API int mkv_decode_attention(mkv_pool_t pool, const int32_t* seq_ids, int32_t n_seqs,
                                  int32_t q_len, const void* q_bf16, int32_t num_q_heads,
